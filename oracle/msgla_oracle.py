@@ -1,0 +1,195 @@
+"""Plain fp64 CPU oracle of the MS-GLA layer forward pass.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module. The product (the CUDA library and its binding) never calls it, and it
+shares no code with the product: it depends on numpy alone.
+
+What it computes follows "MS-GLA: Multi-Scale Gated Linear Attention" as
+summarised in the MS-GLA reading notes (arXiv 2609.35664v1):
+
+* Sec. 2.1 (the paper's Eqs. (2), (5), (6)): the GLA recurrence in row-vector
+  form, S_t = Diag(alpha_t) S_{t-1} + k_t^T v_t and o_t = q_t S_t, with
+  q_t, k_t in R^{1 x d_k}, v_t in R^{1 x d_v}, S_t in R^{d_k x d_v}; alpha_t in
+  (0,1)^{d_k} comes from a low-rank projection of the hidden state followed by
+  a sigmoid-type map.
+* Sec. 3.1, Eq. (8): non-overlapping mean pooling over s adjacent rows, pooled
+  length ceil(L/s), the incomplete tail block averaged over its valid rows
+  (no padding mask: every row inside L is valid).
+* Sec. 3.2, Eq. (9): the H heads are split over the scales (sum_s h_s = H);
+  each branch has its own q/k/v/gate/output projections.
+* Sec. 3.3: causal hold -- each coarse output is repeated s times and shifted
+  right by s-1 with zero fill, i.e. position t reads pooled row
+  floor((t+1)/s) - 1, or zero when that index is negative.
+* Sec. 3.3, Eqs. (10)-(11): w_t = softmax(W_fuse x_t + b_fuse) from the
+  unpooled row x_t, and O_t = sum_s w_{t,s} Yhat^(s)_t.
+
+Readings where the notes leave a step open (each is also listed in the design
+notes of this repository):
+* gate form: log alpha = logsigmoid(g W_g2^T + b_g) / gate_normalizer with
+  g = xbar W_g1^T of rank r (the notes only say "low-rank + sigmoid-like");
+* output projection before the hold (the two orders are identical: the hold
+  is a row gather);
+* o_t = qk_scale * q_t S_t with qk_scale = 1 by default (the notes' equation
+  has no scale);
+* no per-branch normalisation and no output gate (the notes list a
+  per-branch "normalisation" without defining it).
+
+Every step is written token by token or row by row; numpy's matmul is used as
+a library primitive for the per-row projections only.
+
+Parity pins (tests/test_oracle.py): brute-force quadratic form of the GLA
+recurrence, alpha = 1 reducing to causal (Q K^T) V, the single-scale layer
+reducing to plain GLA + W_o, the constant-input geometric closed form, the
+worked s = 4 hold table and pooling example of Sec. 3.1/3.3, causality,
+half-life, the 11/16 update count and the simplex property of the fusion
+weights.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+# ---------------------------------------------------------------------------
+# Sec. 3.1, Eq. (8): non-overlapping mean pooling (mask M = 1 inside L)
+# ---------------------------------------------------------------------------
+def pool(X: np.ndarray, s: int) -> np.ndarray:
+    """Mean of each block of s consecutive rows; X is [L, d] -> [ceil(L/s), d].
+
+    The incomplete tail block (L not divisible by s) is the mean of its valid
+    rows: Eq. (8) with M = 1 for rows inside L and 0 for the right padding,
+    denominator max(1, sum M).
+    """
+    L = X.shape[0]
+    n = -(-L // s)
+    out = np.zeros((n, X.shape[1]), dtype=np.float64)
+    for i in range(n):
+        rows = [i * s + j for j in range(s) if i * s + j < L]
+        acc = np.zeros(X.shape[1], dtype=np.float64)
+        for r in rows:
+            acc += X[r]
+        out[i] = acc / max(1, len(rows))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Sec. 2.1 gate: low-rank projection + sigmoid-type map (form fixed above)
+# ---------------------------------------------------------------------------
+def logsigmoid(z: np.ndarray) -> np.ndarray:
+    """log(1 / (1 + exp(-z))) evaluated without overflow."""
+    return -np.logaddexp(0.0, -z)
+
+
+def branch_projections(Xp: np.ndarray, br: dict, gate_normalizer: float):
+    """q, k, v and log alpha of one branch from its pooled rows Xp [n, d].
+
+    q = Xp W_q^T, k = Xp W_k^T, v = Xp W_v^T (heads side by side along the
+    feature axis), log alpha = logsigmoid((Xp W_g1^T) W_g2^T + b_g) / normalizer.
+    """
+    q = Xp @ br["Wq"].T
+    k = Xp @ br["Wk"].T
+    v = Xp @ br["Wv"].T
+    g = Xp @ br["Wg1"].T
+    log_alpha = logsigmoid(g @ br["Wg2"].T + br["bg"]) / gate_normalizer
+    return q, k, v, log_alpha
+
+
+# ---------------------------------------------------------------------------
+# Sec. 2.1: GLA recurrence, one head, token by token
+# ---------------------------------------------------------------------------
+def gla_recurrent(q: np.ndarray, k: np.ndarray, v: np.ndarray, log_alpha: np.ndarray,
+                  qk_scale: float = 1.0, counter: list | None = None) -> np.ndarray:
+    """S_0 = 0; for each step t: S_t = Diag(alpha_t) S_{t-1} + k_t^T v_t and
+    o_t = qk_scale * q_t S_t. q, k, log_alpha are [n, d_k]; v is [n, d_v]."""
+    n, dk = q.shape
+    dv = v.shape[1]
+    S = np.zeros((dk, dv), dtype=np.float64)
+    o = np.zeros((n, dv), dtype=np.float64)
+    alpha = np.exp(log_alpha)
+    for t in range(n):
+        S = alpha[t][:, None] * S + np.outer(k[t], v[t])
+        o[t] = qk_scale * (q[t] @ S)
+        if counter is not None:
+            counter[0] += 1
+    return o
+
+
+# ---------------------------------------------------------------------------
+# Sec. 3.3: causal hold (repeat s times, shift right by s-1, zero fill)
+# ---------------------------------------------------------------------------
+def hold_index(t: int, s: int) -> int:
+    """Pooled row read at original position t, or -1 for the zero fill."""
+    return (t + 1) // s - 1
+
+
+def hold(Y: np.ndarray, s: int, L: int) -> np.ndarray:
+    """Yhat [L, d] from the pooled branch output Y [ceil(L/s), d]."""
+    out = np.zeros((L, Y.shape[1]), dtype=np.float64)
+    for t in range(L):
+        i = hold_index(t, s)
+        if i >= 0:
+            out[t] = Y[i]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Sec. 3.3, Eqs. (10)-(11): input-dependent fusion
+# ---------------------------------------------------------------------------
+def fusion_weights(X: np.ndarray, Wfuse: np.ndarray, bfuse: np.ndarray) -> np.ndarray:
+    """w_t = softmax(W_fuse x_t + b_fuse) for every row of X [L, d]."""
+    z = X @ Wfuse.T + bfuse
+    z = z - z.max(axis=1, keepdims=True)
+    e = np.exp(z)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+# ---------------------------------------------------------------------------
+# whole layer
+# ---------------------------------------------------------------------------
+def layer_forward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: int,
+                  gate_normalizer: float = 16.0, qk_scale: float = 1.0,
+                  intermediates: bool = False, counter: list | None = None):
+    """MS-GLA layer forward for X [B, L, d] (float64).
+
+    ``weights`` holds ``branches`` (per scale: Wq, Wk, Wv, Wg1, Wg2, bg, Wo)
+    and ``Wfuse``, ``bfuse``. Returns O [B, L, d]; with ``intermediates`` also a
+    dict of per-branch pooled rows, q, k, v, log alpha, o and Y plus the fusion
+    weights w, each with a leading batch axis.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    B, L, d = X.shape
+    assert len(scales) == len(heads) == len(weights["branches"])
+    O = np.zeros((B, L, d), dtype=np.float64)
+    inter = {"w": [], "branches": [dict(Xp=[], q=[], k=[], v=[], log_alpha=[], o=[], Y=[])
+                                   for _ in scales]}
+    for b in range(B):
+        w = fusion_weights(X[b], weights["Wfuse"], weights["bfuse"])
+        inter["w"].append(w)
+        for j, (s, h) in enumerate(zip(scales, heads)):
+            br = weights["branches"][j]
+            Xp = pool(X[b], s)
+            q, k, v, la = branch_projections(Xp, br, gate_normalizer)
+            o = np.zeros((Xp.shape[0], h * d_v), dtype=np.float64)
+            for hh in range(h):
+                ck, cv = slice(hh * d_k, (hh + 1) * d_k), slice(hh * d_v, (hh + 1) * d_v)
+                o[:, cv] = gla_recurrent(q[:, ck], k[:, ck], v[:, cv], la[:, ck],
+                                         qk_scale=qk_scale, counter=counter)
+            Y = o @ br["Wo"].T
+            O[b] += w[:, j:j + 1] * hold(Y, s, L)
+            if intermediates:
+                for name, val in (("Xp", Xp), ("q", q), ("k", k), ("v", v),
+                                  ("log_alpha", la), ("o", o), ("Y", Y)):
+                    inter["branches"][j][name].append(val)
+    if not intermediates:
+        return O
+    inter["w"] = np.stack(inter["w"])
+    for br in inter["branches"]:
+        for name in list(br):
+            br[name] = np.stack(br[name]) if br[name] else None
+    return O, inter
+
+
+def state_updates(L: int, scales, heads) -> int:
+    """Number of per-head state updates the layer performs on one sequence of
+    length L (each branch updates its h_s states once per pooled step)."""
+    return sum(h * (-(-L // s)) for s, h in zip(scales, heads))
