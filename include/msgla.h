@@ -1,0 +1,151 @@
+/*
+ * msgla.h -- C ABI of the MS-GLA (multi-scale gated linear attention) layer
+ * forward pass on NVIDIA B200 (sm_100a).
+ *
+ * The layer (MS-GLA reading notes, arXiv 2609.35664v1, Secs. 2.1 and 3.1-3.3):
+ *   for every scale s of the scale set S, with h_s heads (sum_s h_s = H, Eq. (9)):
+ *     Xbar^(s)_i = mean of rows i*s .. i*s+s-1 of X        (Sec. 3.1, Eq. (8))
+ *     q, k = Xbar W_q^T, Xbar W_k^T      [per head d_k wide]
+ *     v    = Xbar W_v^T                  [per head d_v wide]
+ *     log alpha = logsigmoid((Xbar W_g1^T) W_g2^T + b_g) / gate_normalizer
+ *     S_t = Diag(alpha_t) S_{t-1} + k_t^T v_t,  o_t = qk_scale * q_t S_t  (Sec. 2.1)
+ *     Y^(s) = o W_o^T                                        (Sec. 3.2)
+ *     Yhat^(s)_t = Y^(s)_{floor((t+1)/s)-1}, zero when that index is < 0 (Sec. 3.3)
+ *   w_t = softmax(W_fuse x_t + b_fuse),  O_t = sum_s w_{t,s} Yhat^(s)_t  (Eqs. (10)-(11))
+ *
+ * Conventions
+ *   - Matrices are row-major with PyTorch Linear layout [out, in] (y = x W^T).
+ *   - "device" pointers are CUDA global memory of the handle's device; "host"
+ *     pointers are ordinary (preferably pinned) host memory.
+ *   - bf16 = IEEE-754 bfloat16 stored as uint16; f32 = IEEE float.
+ *   - Every call returns an msgla_status (0 = success, negative = error), except
+ *     msgla_destroy and msgla_status_string. msgla_last_error() gives a message
+ *     for the last failing call on the calling thread.
+ *   - Calls are not thread-safe on one handle. A handle may be used with one
+ *     stream at a time (its device-side error flags are per handle).
+ */
+#ifndef MSGLA_H_
+#define MSGLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MSGLA_MAX_SCALES 8
+
+typedef enum msgla_status {
+  MSGLA_OK = 0,
+  MSGLA_ERR_INVALID_ARG = -1,    /* null pointer, bad size, inconsistent config       */
+  MSGLA_ERR_UNSUPPORTED = -2,    /* valid but outside what the kernels implement      */
+  MSGLA_ERR_CUDA = -3,           /* a CUDA runtime/driver call failed                 */
+  MSGLA_ERR_DEVICE_TIMEOUT = -4, /* a bounded wait inside a kernel gave up            */
+  MSGLA_ERR_RANGE = -5,          /* a value left the fp16 range of an internal operand */
+  MSGLA_ERR_WORKSPACE = -6       /* workspace missing, too small or misaligned        */
+} msgla_status;
+
+/* Layer configuration (Sec. 3.2 of the notes: scale set, head split, widths). */
+typedef struct msgla_config {
+  int d;                         /* model width; multiple of 64, 64..8192                 */
+  int n_scales;                  /* |S|, 1..MSGLA_MAX_SCALES                              */
+  int scales[MSGLA_MAX_SCALES];  /* pooling factors, strictly increasing, 1..64           */
+  int heads[MSGLA_MAX_SCALES];   /* h_s >= 1 for each scale; H = sum of heads             */
+  int d_k;                       /* key width per head, 1..256                            */
+  int d_v;                       /* value width per head, 1..1024                         */
+  int gate_rank;                 /* rank r of the gate projection, 1..64                  */
+  int chunk;                     /* chunk length of the chunkwise GLA kernel: 0 or 64.
+                                    A compute parameter with no effect on the result
+                                    beyond rounding (Sec. 3.4 of the notes).             */
+  float gate_normalizer;         /* log alpha = logsigmoid(.) / gate_normalizer (> 0)     */
+  float qk_scale;                /* o_t = qk_scale * q_t S_t                              */
+} msgla_config;
+
+/* Weights: DEVICE pointers on the handle's device, read during msgla_create only
+ * (the handle keeps its own packed copies; the caller may free these after).
+ * Per scale j (index into msgla_config.scales):
+ *   Wq[j]  bf16 [h_j*d_k, d]     Wk[j] bf16 [h_j*d_k, d]    Wv[j] bf16 [h_j*d_v, d]
+ *   Wg1[j] bf16 [gate_rank, d]   Wg2[j] f32 [h_j*d_k, gate_rank]   bg[j] f32 [h_j*d_k]
+ *   Wo[j]  bf16 [d, h_j*d_v]
+ * Heads are laid side by side: head h of scale j owns rows h*d_k..h*d_k+d_k-1 of
+ * Wq/Wk/Wg2/bg, rows h*d_v.. of Wv and columns h*d_v.. of Wo.
+ *   Wfuse  bf16 [n_scales, d]    bfuse f32 [n_scales] (NULL = zeros)
+ * bg[j] may be NULL (zeros). */
+typedef struct msgla_weights {
+  const void*  Wq[MSGLA_MAX_SCALES];
+  const void*  Wk[MSGLA_MAX_SCALES];
+  const void*  Wv[MSGLA_MAX_SCALES];
+  const void*  Wg1[MSGLA_MAX_SCALES];
+  const float* Wg2[MSGLA_MAX_SCALES];
+  const float* bg[MSGLA_MAX_SCALES];
+  const void*  Wo[MSGLA_MAX_SCALES];
+  const void*  Wfuse;
+  const float* bfuse;
+} msgla_weights;
+
+typedef struct msgla_handle msgla_handle;
+
+/* Create a layer on CUDA device `device`. Validates the configuration, packs the
+ * weights into handle-owned device buffers (converted to fp16 where a tensor-core
+ * operand pairs them with fp16 data; a weight whose magnitude exceeds 65504 is
+ * rejected with MSGLA_ERR_RANGE) and synchronises the device.
+ * On success *out owns device memory until msgla_destroy. On error *out = NULL. */
+int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weights* w,
+                 int device);
+
+/* Free everything the handle owns. NULL-safe. Synchronises the handle's device. */
+void msgla_destroy(msgla_handle* h);
+
+/* Bytes of device workspace msgla_forward needs for a [B, L, d] input.
+ * B >= 0, L >= 0 (B*L = 0 gives 0 bytes). */
+int msgla_workspace_size(const msgla_handle* h, int B, int L, size_t* bytes);
+
+/* Layer forward: O = MS-GLA(X).
+ *   X  device bf16 [B, L, d], row-major, 16-byte aligned, not written.
+ *   O  device bf16 [B, L, d], row-major, 16-byte aligned; may not alias X.
+ *   workspace  device buffer of at least msgla_workspace_size bytes, 256-byte
+ *              aligned, owned by the caller; its contents on entry do not matter.
+ *   stream     cudaStream_t (NULL = legacy default stream).
+ * Asynchronous: returns after enqueuing the kernels on `stream`. Errors found by
+ * the kernels (timeouts, fp16 range) are latched in the handle and reported by
+ * msgla_sync_status (and by the next msgla_forward). B*L = 0 launches nothing. */
+int msgla_forward(msgla_handle* h, const void* X, int B, int L, void* O,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace for msgla_forward_host: msgla_workspace_size plus room to stage X and O. */
+int msgla_workspace_size_host(const msgla_handle* h, int B, int L, size_t* bytes);
+
+/* Host-buffer forward: copies X (HOST bf16 [B, L, d]) to the device part of
+ * `workspace`, runs the layer, copies O back to HOST bf16 [B, L, d] and
+ * synchronises `stream`. Pinned host memory gives the fastest copies. Returns the
+ * status of the whole call, including device-side errors. */
+int msgla_forward_host(msgla_handle* h, const void* X_host, int B, int L, void* O_host,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise the handle's device and return (then clear) the first device-side
+ * error latched since the previous call: MSGLA_OK, MSGLA_ERR_DEVICE_TIMEOUT or
+ * MSGLA_ERR_RANGE; MSGLA_ERR_CUDA if the synchronisation itself failed. */
+int msgla_sync_status(msgla_handle* h);
+
+/* Intermediate tensors inside the workspace of a forward with the same B and L
+ * (for inspection by tests and tools; valid after the forward completes).
+ * `which`: 0 pooled X (fp16 [B, n_s, d]; scales > 1 only), 1 q (fp16 [B, n_s, h*dkp]),
+ * 2 k, 3 v (fp16 [B, n_s, h*dvp]), 4 gate low-rank g (f32 [B, n_s, rp]),
+ * 5 o (fp16 [B, n_s, h*dvp]), 6 Y (fp16 [B, n_s, d]; branches whose output is
+ * materialised), 7 fusion weights w (f32 [B, L, n_scales]; `scale_index` ignored).
+ * dkp, dvp and rp are the padded widths reported in dims[2] (columns). Padding
+ * columns hold zeros. A tensor that does not exist gives MSGLA_ERR_INVALID_ARG. */
+int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index, int which,
+                           size_t* offset, int dims[3]);
+
+/* Static description of an error code. */
+const char* msgla_status_string(int status);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char* msgla_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSGLA_H_ */

@@ -1,0 +1,693 @@
+// msgla_abi.cu -- host side of the C ABI declared in include/msgla.h.
+//
+// Launch sequence of one forward (MS-GLA reading notes, Sec. 3):
+//   1. pool_fuse   pooled rows for every scale s > 1 (fp16) and the fusion
+//                  weights w (fp32), one pass over X
+//   2. gemm        q | k | v | low-rank gate of every branch (grouped launch)
+//   3. gate        log alpha, in-chunk cumulative sums, scaled q/k, chunk decays
+//   4. gla         chunkwise GLA of every branch and head (grouped launch)
+//   5. gemm        Y^(s) = o W_o^T of the coarse branches (fp16)
+//   6. gemm        Y^(1) = o W_o^T of the scale-1 branch fused with the causal
+//                  hold of the coarse Y^(s) and the fusion weights -> O (bf16)
+//      (without a scale-1 branch: all Y^(s) in step 5, then hold_fuse)
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/msgla.h"
+#include "msgla_internal.h"
+#include "sm100_ptx.cuh"
+
+using namespace msgla;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+#define CUDA_TRY(expr)                                                                                   \
+  do {                                                                                                   \
+    cudaError_t e_ = (expr);                                                                             \
+    if (e_ != cudaSuccess) return fail(MSGLA_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+int gcd(int a, int b) { return b == 0 ? a : gcd(b, a % b); }
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 16-bit row-major [batch][rows][inner] with a {64, box_rows, 1} box and 128B swizzle.
+bool encode_3d(CUtensorMap* m, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+               uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base),
+            dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool encode_2d(CUtensorMap* m, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base),
+            dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess) ok = true;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+}  // namespace
+
+// ---------------------------------------------------------------- handle
+struct Branch {
+  int scale, heads;
+  int np;             // packed projection rows: h(2 dkp + dvp) + rp
+  void* Bproj;        // [np, d] bf16 (scale 1) or fp16
+  float* Wg2p;        // [h dkp, rp]
+  float* bgp;         // [h dkp]
+  __half* Wop;        // [d, h dvp]
+};
+
+struct msgla_handle {
+  msgla_config cfg;
+  int device;
+  int dkp, dvp, rp, n_scales, main_index, pool_rows;
+  Branch br[MSGLA_MAX_SCALES];
+  __nv_bfloat16* Wfuse;
+  float* bfuse;
+  int* d_err;  // device error word
+};
+
+namespace {
+
+struct Region {
+  size_t off = 0, bytes = 0;
+};
+struct BranchWs {
+  int rows, n_chunks;
+  Region Xp, q, k, qs, ks, v, g, gamma, o, Y;
+};
+struct Workspace {
+  BranchWs br[MSGLA_MAX_SCALES];
+  Region w;
+  size_t total = 0;
+};
+
+void add(Region& r, size_t& cur, size_t bytes) {
+  r.off = cur;
+  r.bytes = bytes;
+  cur = round_up(cur + bytes, 256);
+}
+
+Workspace layout(const msgla_handle* h, int B, int L) {
+  Workspace ws;
+  size_t cur = 0;
+  const size_t BB = static_cast<size_t>(B);
+  const int d = h->cfg.d;
+  for (int j = 0; j < h->n_scales; ++j) {
+    const Branch& b = h->br[j];
+    BranchWs& w = ws.br[j];
+    w.rows = ceil_div(L, b.scale);
+    w.n_chunks = ceil_div(w.rows, kChunk);
+    const size_t n = BB * w.rows;
+    if (b.scale > 1) add(w.Xp, cur, n * d * 2);
+    add(w.q, cur, n * b.heads * h->dkp * 2);
+    add(w.k, cur, n * b.heads * h->dkp * 2);
+    add(w.qs, cur, n * b.heads * h->dkp * 2);
+    add(w.ks, cur, n * b.heads * h->dkp * 2);
+    add(w.v, cur, n * b.heads * h->dvp * 2);
+    add(w.g, cur, n * h->rp * 4);
+    add(w.gamma, cur, BB * w.n_chunks * b.heads * h->dkp * 4);
+    add(w.o, cur, n * b.heads * h->dvp * 2);
+    if (j != h->main_index) add(w.Y, cur, n * d * 2);
+  }
+  add(ws.w, cur, BB * L * h->n_scales * 4);
+  ws.total = cur;
+  return ws;
+}
+
+int validate(const msgla_config* c) {
+  if (!c) return fail(MSGLA_ERR_INVALID_ARG, "config is NULL");
+  if (c->d < 64 || c->d > 8192 || c->d % 64)
+    return fail(MSGLA_ERR_UNSUPPORTED, "d=%d: must be a multiple of 64 in [64, 8192]", c->d);
+  if (c->n_scales < 1 || c->n_scales > MSGLA_MAX_SCALES)
+    return fail(MSGLA_ERR_INVALID_ARG, "n_scales=%d outside [1, %d]", c->n_scales, MSGLA_MAX_SCALES);
+  int H = 0;
+  for (int j = 0; j < c->n_scales; ++j) {
+    if (c->scales[j] < 1 || c->scales[j] > 64)
+      return fail(MSGLA_ERR_INVALID_ARG, "scales[%d]=%d outside [1, 64]", j, c->scales[j]);
+    if (j > 0 && c->scales[j] <= c->scales[j - 1])
+      return fail(MSGLA_ERR_INVALID_ARG, "scales must be strictly increasing");
+    if (c->heads[j] < 1) return fail(MSGLA_ERR_INVALID_ARG, "heads[%d]=%d must be >= 1", j, c->heads[j]);
+    H += c->heads[j];
+  }
+  if (H > 64) return fail(MSGLA_ERR_UNSUPPORTED, "H=%d heads: at most 64", H);
+  if (c->d_k < 1 || c->d_k > 256) return fail(MSGLA_ERR_UNSUPPORTED, "d_k=%d outside [1, 256]", c->d_k);
+  if (c->d_v < 1 || c->d_v > 1024) return fail(MSGLA_ERR_UNSUPPORTED, "d_v=%d outside [1, 1024]", c->d_v);
+  if (c->gate_rank < 1 || c->gate_rank > 32)
+    return fail(MSGLA_ERR_UNSUPPORTED, "gate_rank=%d outside [1, 32]", c->gate_rank);
+  if (c->chunk != 0 && c->chunk != kChunk)
+    return fail(MSGLA_ERR_UNSUPPORTED, "chunk=%d: the GLA kernel runs 64-row chunks (pass 0 or 64)", c->chunk);
+  if (!(c->gate_normalizer > 0.f) || !std::isfinite(c->gate_normalizer))
+    return fail(MSGLA_ERR_INVALID_ARG, "gate_normalizer must be finite and > 0");
+  if (!std::isfinite(c->qk_scale)) return fail(MSGLA_ERR_INVALID_ARG, "qk_scale must be finite");
+  int lcm = 1;
+  for (int j = 0; j < c->n_scales; ++j)
+    if (c->scales[j] > 1) lcm = lcm / gcd(lcm, c->scales[j]) * c->scales[j];
+  if (lcm > 64)
+    return fail(MSGLA_ERR_UNSUPPORTED, "least common multiple of the scales is %d (at most 64)", lcm);
+  return MSGLA_OK;
+}
+
+void free_handle(msgla_handle* h) {
+  if (!h) return;
+  for (int j = 0; j < MSGLA_MAX_SCALES; ++j) {
+    cudaFree(h->br[j].Bproj);
+    cudaFree(h->br[j].Wg2p);
+    cudaFree(h->br[j].bgp);
+    cudaFree(h->br[j].Wop);
+  }
+  cudaFree(h->Wfuse);
+  cudaFree(h->bfuse);
+  cudaFree(h->d_err);
+  delete h;
+}
+
+template <class T>
+int dmalloc_zero(T** p, size_t bytes) {
+  *p = nullptr;
+  CUDA_TRY(cudaMalloc(reinterpret_cast<void**>(p), bytes));
+  CUDA_TRY(cudaMemset(*p, 0, bytes));
+  return MSGLA_OK;
+}
+
+int create_impl(msgla_handle* h, const msgla_weights* w) {
+  const msgla_config& c = h->cfg;
+  const int d = c.d, dk = c.d_k, dv = c.d_v, r = c.gate_rank;
+  int* d_over = nullptr;
+  int st = dmalloc_zero(&d_over, sizeof(int));
+  if (st) return st;
+  struct Free {
+    int* p;
+    ~Free() { cudaFree(p); }
+  } free_over{d_over};
+  for (int j = 0; j < h->n_scales; ++j) {
+    Branch& b = h->br[j];
+    if (!w->Wq[j] || !w->Wk[j] || !w->Wv[j] || !w->Wg1[j] || !w->Wg2[j] || !w->Wo[j])
+      return fail(MSGLA_ERR_INVALID_ARG, "weights of scale index %d: NULL pointer", j);
+    const int hh = b.heads;
+    const bool bf = (b.scale == 1);
+    const size_t esz = 2;
+    if ((st = dmalloc_zero(&b.Bproj, static_cast<size_t>(b.np) * d * esz))) return st;
+    if ((st = dmalloc_zero(&b.Wg2p, static_cast<size_t>(hh) * h->dkp * h->rp * 4))) return st;
+    if ((st = dmalloc_zero(&b.bgp, static_cast<size_t>(hh) * h->dkp * 4))) return st;
+    if ((st = dmalloc_zero(&b.Wop, static_cast<size_t>(d) * hh * h->dvp * 2))) return st;
+    auto put_rows = [&](const void* src, int src_row0, int nrows, int dst_row0) -> cudaError_t {
+      const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(src) + static_cast<size_t>(src_row0) * d;
+      if (bf)
+        return launch_bf16_copy_rows(s, d, nrows, d,
+                                     static_cast<__nv_bfloat16*>(b.Bproj) + static_cast<size_t>(dst_row0) * d, d, 0);
+      return launch_bf16_to_f16_rows(s, d, nrows, d, static_cast<__half*>(b.Bproj) + static_cast<size_t>(dst_row0) * d,
+                                     d, d_over, 0);
+    };
+    for (int x = 0; x < hh; ++x) {
+      CUDA_TRY(put_rows(w->Wq[j], x * dk, dk, x * h->dkp));
+      CUDA_TRY(put_rows(w->Wk[j], x * dk, dk, hh * h->dkp + x * h->dkp));
+      CUDA_TRY(put_rows(w->Wv[j], x * dv, dv, 2 * hh * h->dkp + x * h->dvp));
+      CUDA_TRY(cudaMemcpy2D(b.Wg2p + static_cast<size_t>(x) * h->dkp * h->rp, h->rp * 4,
+                            w->Wg2[j] + static_cast<size_t>(x) * dk * r, r * 4, r * 4, dk, cudaMemcpyDeviceToDevice));
+      if (w->bg[j])
+        CUDA_TRY(cudaMemcpy(b.bgp + static_cast<size_t>(x) * h->dkp, w->bg[j] + static_cast<size_t>(x) * dk, dk * 4,
+                            cudaMemcpyDeviceToDevice));
+      CUDA_TRY(launch_bf16_to_f16_rows(static_cast<const __nv_bfloat16*>(w->Wo[j]) + static_cast<size_t>(x) * dv,
+                                       hh * dv, d, dv, b.Wop + static_cast<size_t>(x) * h->dvp, hh * h->dvp, d_over,
+                                       0));
+    }
+    CUDA_TRY(put_rows(w->Wg1[j], 0, r, hh * (2 * h->dkp + h->dvp)));
+  }
+  if (!w->Wfuse) return fail(MSGLA_ERR_INVALID_ARG, "Wfuse is NULL");
+  if ((st = dmalloc_zero(&h->Wfuse, static_cast<size_t>(h->n_scales) * d * 2))) return st;
+  if ((st = dmalloc_zero(&h->bfuse, static_cast<size_t>(h->n_scales) * 4))) return st;
+  CUDA_TRY(cudaMemcpy(h->Wfuse, w->Wfuse, static_cast<size_t>(h->n_scales) * d * 2, cudaMemcpyDeviceToDevice));
+  if (w->bfuse) CUDA_TRY(cudaMemcpy(h->bfuse, w->bfuse, h->n_scales * 4, cudaMemcpyDeviceToDevice));
+  if ((st = dmalloc_zero(&h->d_err, sizeof(int)))) return st;
+  CUDA_TRY(cudaDeviceSynchronize());
+  int over = 0;
+  CUDA_TRY(cudaMemcpy(&over, d_over, sizeof(int), cudaMemcpyDeviceToHost));
+  if (over) return fail(MSGLA_ERR_RANGE, "%d weight values exceed the fp16 range (|w| > 65504)", over);
+  return MSGLA_OK;
+}
+
+int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* wsp, size_t ws_bytes,
+                 cudaStream_t st) {
+  const msgla_config& c = h->cfg;
+  const int d = c.d;
+  const Workspace ws = layout(h, B, L);
+  if (!wsp || ws_bytes < ws.total)
+    return fail(MSGLA_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, ws.total);
+  if (reinterpret_cast<uintptr_t>(wsp) % 256) return fail(MSGLA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  uint8_t* base = static_cast<uint8_t*>(wsp);
+  auto at = [&](const Region& r) { return static_cast<void*>(base + r.off); };
+  const int ns = h->n_scales;
+
+  // 1. pooling + fusion weights
+  PoolParams pp{};
+  pp.X = static_cast<const __nv_bfloat16*>(X);
+  pp.B = B;
+  pp.L = L;
+  pp.d = d;
+  pp.n_scales = ns;
+  for (int j = 0; j < ns; ++j) {
+    pp.scales[j] = h->br[j].scale;
+    pp.Xp[j] = h->br[j].scale > 1 ? static_cast<__half*>(at(ws.br[j].Xp)) : nullptr;
+  }
+  pp.Wfuse = h->Wfuse;
+  pp.bfuse = h->bfuse;
+  pp.w = static_cast<float*>(at(ws.w));
+  pp.block_rows = h->pool_rows;
+  pp.err = h->d_err;
+  CUDA_TRY(launch_pool_fuse(pp, st));
+
+  // 2. projections (grouped over branches)
+  static thread_local GemmParams gp;
+  memset(&gp, 0, sizeof(gp));
+  gp.err = h->d_err;
+  int tiles = 0;
+  for (int j = 0; j < ns; ++j) {
+    const Branch& b = h->br[j];
+    const BranchWs& bw = ws.br[j];
+    GemmTask& t = gp.task[j];
+    const bool bf = (b.scale == 1);
+    if (!encode_3d(&t.tmA, bf, bf ? X : at(bw.Xp), d, bw.rows, B, kGemmBM) ||
+        !encode_2d(&t.tmB, bf, b.Bproj, d, b.np, 256))
+      return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (projection, scale %d)", b.scale);
+    t.rows = bw.rows;
+    t.m_tiles = ceil_div(bw.rows, kGemmBM);
+    t.n_tiles = ceil_div(b.np, 256);
+    t.N = b.np;
+    t.K = d;
+    t.tile_begin = tiles;
+    t.ab_bf16 = bf ? 1 : 0;
+    t.epi = kEpiProj;
+    t.nq = t.nk = b.heads * h->dkp;
+    t.nv = b.heads * h->dvp;
+    t.ng = h->rp;
+    t.q = static_cast<__half*>(at(bw.q));
+    t.k = static_cast<__half*>(at(bw.k));
+    t.v = static_cast<__half*>(at(bw.v));
+    t.g = static_cast<float*>(at(bw.g));
+    tiles += B * t.m_tiles * t.n_tiles;
+  }
+  gp.n_tasks = ns;
+  gp.total_tiles = tiles;
+  CUDA_TRY(launch_gemm(gp, 256, st));
+
+  // 3. gates
+  for (int j = 0; j < ns; ++j) {
+    const Branch& b = h->br[j];
+    const BranchWs& bw = ws.br[j];
+    GateParams g{};
+    g.q = static_cast<const __half*>(at(bw.q));
+    g.k = static_cast<const __half*>(at(bw.k));
+    g.g = static_cast<const float*>(at(bw.g));
+    g.Wg2 = b.Wg2p;
+    g.bg = b.bgp;
+    g.qs = static_cast<__half*>(at(bw.qs));
+    g.ks = static_cast<__half*>(at(bw.ks));
+    g.gamma = static_cast<float*>(at(bw.gamma));
+    g.B = B;
+    g.rows = bw.rows;
+    g.heads = b.heads;
+    g.dkp = h->dkp;
+    g.rp = h->rp;
+    g.n_chunks = bw.n_chunks;
+    g.inv_normalizer = 1.f / c.gate_normalizer;
+    g.err = h->d_err;
+    CUDA_TRY(launch_gate(g, st));
+  }
+
+  // 4. chunkwise GLA (grouped over branches; longest sequences first)
+  static thread_local GlaParams lp;
+  memset(&lp, 0, sizeof(lp));
+  lp.err = h->d_err;
+  lp.qk_scale = c.qk_scale;
+  int ctas = 0;
+  for (int j = 0; j < ns; ++j) {
+    const Branch& b = h->br[j];
+    const BranchWs& bw = ws.br[j];
+    GlaTask& t = lp.task[j];
+    if (!encode_3d(&t.tmQ, false, at(bw.qs), b.heads * h->dkp, bw.rows, B, kChunk) ||
+        !encode_3d(&t.tmK, false, at(bw.ks), b.heads * h->dkp, bw.rows, B, kChunk) ||
+        !encode_3d(&t.tmV, false, at(bw.v), b.heads * h->dvp, bw.rows, B, kChunk))
+      return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (gla, scale %d)", b.scale);
+    t.gamma = static_cast<const float*>(at(bw.gamma));
+    t.o = static_cast<__half*>(at(bw.o));
+    t.rows = bw.rows;
+    t.n_chunks = bw.n_chunks;
+    t.heads = b.heads;
+    t.dkp = h->dkp;
+    t.dvp = h->dvp;
+    t.v_tiles = h->dvp / kGlaTile;
+    t.cta_begin = ctas;
+    ctas += B * b.heads * t.v_tiles;
+  }
+  lp.n_tasks = ns;
+  lp.total_ctas = ctas;
+  CUDA_TRY(launch_gla(lp, st));
+
+  // 5. coarse branches: Y^(s) = o W_o^T (fp16)
+  memset(&gp, 0, sizeof(gp));
+  gp.err = h->d_err;
+  tiles = 0;
+  int nt = 0;
+  for (int j = 0; j < ns; ++j) {
+    if (j == h->main_index) continue;
+    const Branch& b = h->br[j];
+    const BranchWs& bw = ws.br[j];
+    GemmTask& t = gp.task[nt++];
+    if (!encode_3d(&t.tmA, false, at(bw.o), b.heads * h->dvp, bw.rows, B, kGemmBM) ||
+        !encode_2d(&t.tmB, false, b.Wop, b.heads * h->dvp, d, 256))
+      return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (output, scale %d)", b.scale);
+    t.rows = bw.rows;
+    t.m_tiles = ceil_div(bw.rows, kGemmBM);
+    t.n_tiles = ceil_div(d, 256);
+    t.N = d;
+    t.K = b.heads * h->dvp;
+    t.tile_begin = tiles;
+    t.ab_bf16 = 0;
+    t.epi = kEpiStoreF16;
+    t.y = static_cast<__half*>(at(bw.Y));
+    tiles += B * t.m_tiles * t.n_tiles;
+  }
+  if (nt > 0) {
+    gp.n_tasks = nt;
+    gp.total_tiles = tiles;
+    CUDA_TRY(launch_gemm(gp, 256, st));
+  }
+
+  // 6. scale-1 branch fused with hold + fusion, or the stand-alone hold + fusion
+  if (h->main_index >= 0) {
+    memset(&gp, 0, sizeof(gp));
+    gp.err = h->d_err;
+    const int j = h->main_index;
+    const Branch& b = h->br[j];
+    const BranchWs& bw = ws.br[j];
+    GemmTask& t = gp.task[0];
+    if (!encode_3d(&t.tmA, false, at(bw.o), b.heads * h->dvp, bw.rows, B, kGemmBM) ||
+        !encode_2d(&t.tmB, false, b.Wop, b.heads * h->dvp, d, 256))
+      return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (output, scale 1)");
+    t.rows = bw.rows;
+    t.m_tiles = ceil_div(bw.rows, kGemmBM);
+    t.n_tiles = ceil_div(d, 256);
+    t.N = d;
+    t.K = b.heads * h->dvp;
+    t.tile_begin = 0;
+    t.ab_bf16 = 0;
+    t.epi = kEpiFuse;
+    t.out = static_cast<__nv_bfloat16*>(O);
+    t.w = static_cast<const float*>(at(ws.w));
+    t.n_scales = ns;
+    t.main_index = j;
+    int nc = 0;
+    for (int q = 0; q < ns; ++q) {
+      if (q == j) continue;
+      t.coarse_scale[nc] = h->br[q].scale;
+      t.coarse_index[nc] = q;
+      t.coarse_rows[nc] = ws.br[q].rows;
+      t.coarse_y[nc] = static_cast<const __half*>(at(ws.br[q].Y));
+      ++nc;
+    }
+    t.n_coarse = nc;
+    gp.n_tasks = 1;
+    gp.total_tiles = B * t.m_tiles * t.n_tiles;
+    CUDA_TRY(launch_gemm(gp, 256, st));
+  } else {
+    HoldFuseParams hp{};
+    for (int j = 0; j < ns; ++j) {
+      hp.Y[j] = static_cast<const __half*>(at(ws.br[j].Y));
+      hp.scales[j] = h->br[j].scale;
+      hp.rows[j] = ws.br[j].rows;
+    }
+    hp.w = static_cast<const float*>(at(ws.w));
+    hp.out = static_cast<__nv_bfloat16*>(O);
+    hp.B = B;
+    hp.L = L;
+    hp.d = d;
+    hp.n_scales = ns;
+    CUDA_TRY(launch_hold_fuse(hp, st));
+  }
+  return MSGLA_OK;
+}
+
+int check_forward_args(const msgla_handle* h, int B, int L) {
+  if (!h) return fail(MSGLA_ERR_INVALID_ARG, "handle is NULL");
+  if (B < 0 || L < 0) return fail(MSGLA_ERR_INVALID_ARG, "B=%d, L=%d must be >= 0", B, L);
+  if (static_cast<long long>(B) * L * h->cfg.d > (1ll << 34))
+    return fail(MSGLA_ERR_UNSUPPORTED, "B*L*d = %lld elements is beyond the supported size",
+                static_cast<long long>(B) * L * h->cfg.d);
+  if (L > (1 << 24)) return fail(MSGLA_ERR_UNSUPPORTED, "L=%d beyond 2^24", L);
+  if (B > 65535) return fail(MSGLA_ERR_UNSUPPORTED, "B=%d beyond 65535", B);
+  return MSGLA_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- C ABI
+extern "C" {
+
+int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weights* w, int device) {
+  if (!out) return fail(MSGLA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  int st = validate(cfg);
+  if (st) return st;
+  if (!w) return fail(MSGLA_ERR_INVALID_ARG, "weights are NULL");
+  int ndev = 0;
+  CUDA_TRY(cudaGetDeviceCount(&ndev));
+  if (device < 0 || device >= ndev) return fail(MSGLA_ERR_INVALID_ARG, "device %d of %d", device, ndev);
+  cudaDeviceProp prop;
+  CUDA_TRY(cudaGetDeviceProperties(&prop, device));
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(MSGLA_ERR_UNSUPPORTED, "device %d is sm_%d%d; the kernels are built for sm_100a", device, prop.major,
+                prop.minor);
+  if (!encode_fn()) return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  DeviceGuard guard(device);
+  if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", device);
+  msgla_handle* h = new msgla_handle();
+  memset(h->br, 0, sizeof(h->br));
+  h->Wfuse = nullptr;
+  h->bfuse = nullptr;
+  h->d_err = nullptr;
+  h->cfg = *cfg;
+  h->device = device;
+  h->n_scales = cfg->n_scales;
+  h->dkp = cfg->d_k <= 128 ? 128 : 256;
+  h->dvp = static_cast<int>(round_up(cfg->d_v, kGlaTile));
+  h->rp = static_cast<int>(round_up(cfg->gate_rank, 16));
+  h->main_index = -1;
+  int lcm = 1;
+  for (int j = 0; j < h->n_scales; ++j) {
+    h->br[j].scale = cfg->scales[j];
+    h->br[j].heads = cfg->heads[j];
+    h->br[j].np = cfg->heads[j] * (2 * h->dkp + h->dvp) + h->rp;
+    if (cfg->scales[j] == 1) h->main_index = j;
+    else lcm = lcm / gcd(lcm, cfg->scales[j]) * cfg->scales[j];
+  }
+  h->pool_rows = lcm;
+  while (h->pool_rows < 32) h->pool_rows *= 2;
+  st = create_impl(h, w);
+  if (st) {
+    const std::string msg = g_last_error;
+    free_handle(h);
+    g_last_error = msg;
+    return st;
+  }
+  *out = h;
+  return MSGLA_OK;
+}
+
+void msgla_destroy(msgla_handle* h) {
+  if (!h) return;
+  DeviceGuard guard(h->device);
+  cudaDeviceSynchronize();
+  free_handle(h);
+}
+
+int msgla_workspace_size(const msgla_handle* h, int B, int L, size_t* bytes) {
+  if (!bytes) return fail(MSGLA_ERR_INVALID_ARG, "bytes is NULL");
+  int st = check_forward_args(h, B, L);
+  if (st) return st;
+  *bytes = (B == 0 || L == 0) ? 0 : layout(h, B, L).total;
+  return MSGLA_OK;
+}
+
+int msgla_workspace_size_host(const msgla_handle* h, int B, int L, size_t* bytes) {
+  int st = msgla_workspace_size(h, B, L, bytes);
+  if (st) return st;
+  if (B > 0 && L > 0) *bytes += 2 * round_up(static_cast<size_t>(B) * L * h->cfg.d * 2, 256);
+  return MSGLA_OK;
+}
+
+int msgla_forward(msgla_handle* h, const void* X, int B, int L, void* O, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  int st = check_forward_args(h, B, L);
+  if (st) return st;
+  if (B == 0 || L == 0) return MSGLA_OK;
+  if (!X || !O) return fail(MSGLA_ERR_INVALID_ARG, "X or O is NULL");
+  if (reinterpret_cast<uintptr_t>(X) % 16 || reinterpret_cast<uintptr_t>(O) % 16)
+    return fail(MSGLA_ERR_INVALID_ARG, "X and O must be 16-byte aligned");
+  const size_t nbytes = static_cast<size_t>(B) * L * h->cfg.d * 2;
+  const uint8_t* x0 = static_cast<const uint8_t*>(X);
+  const uint8_t* o0 = static_cast<const uint8_t*>(O);
+  if (x0 < o0 + nbytes && o0 < x0 + nbytes) return fail(MSGLA_ERR_INVALID_ARG, "O overlaps X");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
+  return forward_impl(h, X, B, L, O, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int msgla_forward_host(msgla_handle* h, const void* X_host, int B, int L, void* O_host, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  int st = check_forward_args(h, B, L);
+  if (st) return st;
+  if (B == 0 || L == 0) return MSGLA_OK;
+  if (!X_host || !O_host) return fail(MSGLA_ERR_INVALID_ARG, "X or O is NULL");
+  size_t need = 0;
+  msgla_workspace_size_host(h, B, L, &need);
+  if (!workspace || workspace_bytes < need)
+    return fail(MSGLA_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(MSGLA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
+  const size_t nbytes = static_cast<size_t>(B) * L * h->cfg.d * 2;
+  const size_t core = layout(h, B, L).total;
+  uint8_t* Xd = static_cast<uint8_t*>(workspace) + core;
+  uint8_t* Od = Xd + round_up(nbytes, 256);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUDA_TRY(cudaMemcpyAsync(Xd, X_host, nbytes, cudaMemcpyHostToDevice, s));
+  st = forward_impl(h, Xd, B, L, Od, workspace, core, s);
+  if (st) return st;
+  CUDA_TRY(cudaMemcpyAsync(O_host, Od, nbytes, cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(cudaStreamSynchronize(s));
+  int err = 0;
+  CUDA_TRY(cudaMemcpy(&err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (err) {
+    CUDA_TRY(cudaMemset(h->d_err, 0, sizeof(int)));
+    return err == kDevTimeout ? fail(MSGLA_ERR_DEVICE_TIMEOUT, "a bounded wait inside a kernel timed out")
+                              : fail(MSGLA_ERR_RANGE, "an internal fp16 operand overflowed");
+  }
+  return MSGLA_OK;
+}
+
+int msgla_sync_status(msgla_handle* h) {
+  if (!h) return fail(MSGLA_ERR_INVALID_ARG, "handle is NULL");
+  DeviceGuard guard(h->device);
+  CUDA_TRY(cudaDeviceSynchronize());
+  int err = 0;
+  CUDA_TRY(cudaMemcpy(&err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (!err) return MSGLA_OK;
+  CUDA_TRY(cudaMemset(h->d_err, 0, sizeof(int)));
+  if (err == kDevTimeout) return fail(MSGLA_ERR_DEVICE_TIMEOUT, "a bounded wait inside a kernel timed out");
+  return fail(MSGLA_ERR_RANGE, "an internal fp16 operand overflowed");
+}
+
+int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index, int which, size_t* offset,
+                           int dims[3]) {
+  if (!h || !offset || !dims) return fail(MSGLA_ERR_INVALID_ARG, "NULL argument");
+  int st = check_forward_args(h, B, L);
+  if (st) return st;
+  if (B == 0 || L == 0) return fail(MSGLA_ERR_INVALID_ARG, "empty input has no workspace");
+  const Workspace ws = layout(h, B, L);
+  if (which == 7) {
+    *offset = ws.w.off;
+    dims[0] = B;
+    dims[1] = L;
+    dims[2] = h->n_scales;
+    return MSGLA_OK;
+  }
+  if (scale_index < 0 || scale_index >= h->n_scales) return fail(MSGLA_ERR_INVALID_ARG, "scale_index out of range");
+  const BranchWs& bw = ws.br[scale_index];
+  const Branch& b = h->br[scale_index];
+  const Region* r = nullptr;
+  int cols = 0;
+  switch (which) {
+    case 0: r = &bw.Xp; cols = h->cfg.d; break;
+    case 1: r = &bw.q; cols = b.heads * h->dkp; break;
+    case 2: r = &bw.k; cols = b.heads * h->dkp; break;
+    case 3: r = &bw.v; cols = b.heads * h->dvp; break;
+    case 4: r = &bw.g; cols = h->rp; break;
+    case 5: r = &bw.o; cols = b.heads * h->dvp; break;
+    case 6: r = &bw.Y; cols = h->cfg.d; break;
+    default: return fail(MSGLA_ERR_INVALID_ARG, "which=%d unknown", which);
+  }
+  if (r->bytes == 0) return fail(MSGLA_ERR_INVALID_ARG, "tensor %d does not exist for scale index %d", which,
+                                 scale_index);
+  *offset = r->off;
+  dims[0] = B;
+  dims[1] = bw.rows;
+  dims[2] = cols;
+  return MSGLA_OK;
+}
+
+const char* msgla_status_string(int status) {
+  switch (status) {
+    case MSGLA_OK: return "ok";
+    case MSGLA_ERR_INVALID_ARG: return "invalid argument";
+    case MSGLA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MSGLA_ERR_CUDA: return "CUDA error";
+    case MSGLA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MSGLA_ERR_RANGE: return "value outside the fp16 range of an internal operand";
+    case MSGLA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    default: return "unknown status";
+  }
+}
+
+const char* msgla_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,127 @@
+// msgla_internal.h -- parameter blocks shared by the host side of the C ABI and
+// the sm_100a kernels. Not part of the public interface.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+namespace msgla {
+
+// Fixed tile constants.
+constexpr int kGemmBM = 128;     // GEMM rows per tile (tcgen05 M)
+constexpr int kGemmBK = 64;      // GEMM K per stage (one 128-byte swizzle atom of 16-bit data)
+constexpr int kChunk = 64;       // chunk length of the chunkwise GLA kernel
+constexpr int kGlaTile = 128;    // value columns per GLA CTA (tcgen05 M of the output MMA)
+constexpr int kMaxTasks = 8;     // GEMM tasks per grouped launch
+constexpr int kMaxScales = 8;
+
+enum EpiKind : int {
+  kEpiProj = 0,      // split columns into q | k | v (fp16) | g (fp32)
+  kEpiStoreF16 = 1,  // plain fp16 store
+  kEpiFuse = 2,      // O = w_main * acc + sum_coarse w_s * held Y_s  (bf16)
+};
+
+// One GEMM D[rows x N] = A[rows x K] * B[N x K]^T per batch, tiled 128 x BN.
+struct alignas(64) GemmTask {
+  CUtensorMap tmA;  // 3D {K, rows, B}, box {64, 128, 1}, 128B swizzle
+  CUtensorMap tmB;  // 2D {K, N}, box {64, BN}, 128B swizzle
+  int rows, m_tiles, n_tiles, N, K, tile_begin, ab_bf16, epi;
+  // kEpiProj
+  int nq, nk, nv, ng;
+  __half* q;
+  __half* k;
+  __half* v;
+  float* g;
+  // kEpiStoreF16
+  __half* y;
+  // kEpiFuse (rows == L, the branch with scale 1)
+  __nv_bfloat16* out;
+  const float* w;   // [B, L, n_scales]
+  int n_scales, main_index, n_coarse, pad_;
+  int coarse_scale[kMaxScales];
+  int coarse_index[kMaxScales];
+  int coarse_rows[kMaxScales];
+  const __half* coarse_y[kMaxScales];
+};
+
+struct GemmParams {
+  GemmTask task[kMaxTasks];
+  int n_tasks;
+  int total_tiles;
+  int* err;
+};
+
+// Chunkwise GLA over one or more branches.
+struct alignas(64) GlaTask {
+  CUtensorMap tmQ;  // 3D {h*dkp, n_s, B}, box {64, 64, 1}
+  CUtensorMap tmK;  // same shape as tmQ
+  CUtensorMap tmV;  // 3D {h*dvp, n_s, B}, box {64, 64, 1}
+  const float* gamma;  // [B, n_chunks, h*dkp]
+  __half* o;           // [B, n_s, h*dvp]
+  int rows, n_chunks, heads, dkp, dvp, v_tiles, cta_begin, pad_;
+};
+
+struct GlaParams {
+  GlaTask task[kMaxScales];
+  int n_tasks;
+  int total_ctas;
+  float qk_scale;
+  int* err;
+};
+
+// ---------------------------------------------------------------- launchers
+// (each returns the cudaError_t of the launch)
+cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st);
+cudaError_t launch_gla(const GlaParams& p, cudaStream_t st);
+
+// pooled rows (fp16) for scales > 1 and fusion weights w = softmax(W_fuse x + b)
+struct PoolParams {
+  const __nv_bfloat16* X;  // [B, L, d]
+  int B, L, d, n_scales;
+  int scales[kMaxScales];
+  __half* Xp[kMaxScales];  // [B, n_s, d] or null (scale 1)
+  const __nv_bfloat16* Wfuse;  // [n_scales, d]
+  const float* bfuse;          // [n_scales]
+  float* w;                    // [B, L, n_scales]
+  int block_rows;              // rows per CTA (multiple of every scale > 1)
+  int* err;
+};
+cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st);
+
+// gates: log alpha, chunk-local cumulative sums, scaled q/k and chunk decays
+struct GateParams {
+  const __half* q;   // [B, n_s, h*dkp]
+  const __half* k;
+  const float* g;    // [B, n_s, rp]
+  const float* Wg2;  // [h*dkp, rp]
+  const float* bg;   // [h*dkp]
+  __half* qs;        // q * exp(b)
+  __half* ks;        // k * exp(-b)
+  float* gamma;      // [B, n_chunks, h*dkp] = exp(b at the chunk's last row)
+  int B, rows, heads, dkp, rp, n_chunks;
+  float inv_normalizer;
+  int* err;
+};
+cudaError_t launch_gate(const GateParams& p, cudaStream_t st);
+
+// hold + fuse from materialised branch outputs (used when no branch has scale 1)
+struct HoldFuseParams {
+  const __half* Y[kMaxScales];  // [B, n_s, d]
+  int scales[kMaxScales];
+  int rows[kMaxScales];
+  const float* w;               // [B, L, n_scales]
+  __nv_bfloat16* out;           // [B, L, d]
+  int B, L, d, n_scales;
+};
+cudaError_t launch_hold_fuse(const HoldFuseParams& p, cudaStream_t st);
+
+// bf16 -> fp16 with an overflow count; bf16 -> bf16 copy into a strided block
+cudaError_t launch_bf16_to_f16_rows(const __nv_bfloat16* src, int src_ld, int rows, int cols, __half* dst,
+                                    int dst_ld, int* overflow, cudaStream_t st);
+cudaError_t launch_bf16_copy_rows(const __nv_bfloat16* src, int src_ld, int rows, int cols, __nv_bfloat16* dst,
+                                  int dst_ld, cudaStream_t st);
+
+}  // namespace msgla
