@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the MS-GLA layer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one MS-GLA layer forward over one batch of the 340M-shaped layer
+(B=8, L=2048, d=1024, scales {1,2,4} with heads [2,1,1], d_k=256, d_v=512) on
+seeded synthetic inputs (see scale_gated_linear_b200/workloads.py). With N > 1
+(one process per GPU under torch.distributed.run) every rank runs its own batch
+of 8 sequences: batch sequences are independent, so the work is sharded by
+sequence with no collective on the data path ("scaling": "weak").
+
+Prints one JSON line on rank 0. Timing: W untimed warm-up steps, then K timed
+steps, each bracketed by CUDA events on the launching stream with a 256 MiB
+write between steps to flush the 126 MB L2; the per-kernel events of
+msgla_forward_profiled give the dominant kernel's duration for the roofline.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MS-GLA layer fwd tokens/sec @d=1024,L=2048"
+UNIT = "tokens/s"
+WORKLOAD = "msgla_340m"
+BASELINE_WORKLOAD = "gla_340m"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+# --------------------------------------------------------------------- helpers
+def shard_rows(global_rows: int, rank: int, world: int) -> range:
+    """Contiguous block of batch rows owned by `rank` (weak scaling gives every rank
+    the same count; any remainder goes to the lowest ranks)."""
+    base, rem = divmod(global_rows, world)
+    start = rank * base + min(rank, rem)
+    return range(start, start + base + (1 if rank < rem else 0))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_counts(w, B: int, L: int) -> dict:
+    """Algorithmic FLOPs (tensor work) and bytes per kernel of one forward.
+
+    FLOPs count only what the layer computes (pooled-length projections, the
+    chunkwise GLA count 4 d_k d_v + C (d_k + d_v) per head and pooled step, the
+    output projection at pooled length); bytes count each kernel's compulsory
+    global-memory traffic."""
+    C = 64
+    r = w.gate_rank
+    out = {}
+    rows = {s: B * math.ceil(L / s) for s in w.scales}
+    out["proj_gemm"] = {"flops": sum(rows[s] * 2 * w.d * (h * (2 * w.d_k + w.d_v) + r)
+                                     for s, h in zip(w.scales, w.heads))}
+    out["gla"] = {"flops": sum(rows[s] * h * (4 * w.d_k * w.d_v + C * (w.d_k + w.d_v))
+                               for s, h in zip(w.scales, w.heads))}
+    coarse = [(s, h) for s, h in zip(w.scales, w.heads) if s != 1]
+    if coarse and 1 in w.scales:
+        out["out_gemm_coarse"] = {"flops": sum(rows[s] * 2 * h * w.d_v * w.d for s, h in coarse)}
+    if 1 in w.scales:
+        h1 = dict(zip(w.scales, w.heads))[1]
+        out["out_gemm_fused"] = {"flops": rows[1] * 2 * h1 * w.d_v * w.d}
+    else:
+        out["out_gemm_coarse"] = {"flops": sum(rows[s] * 2 * h * w.d_v * w.d for s, h in coarse)}
+    out["pool_fuse"] = {"bytes": B * L * w.d * 2 + sum(rows[s] * w.d * 2 for s in w.scales if s > 1)
+                        + B * L * len(w.scales) * 4}
+    out["gate"] = {"bytes": sum(rows[s] * (h * w.d_k * 2 * 2 * 2 + r * 4)
+                                + math.ceil(rows[s] / B / C) * B * h * w.d_k * 4
+                                for s, h in zip(w.scales, w.heads))}
+    total_flops = sum(v.get("flops", 0) for v in out.values())
+    weights = sum(h * (2 * w.d_k + w.d_v) * w.d * 2 + r * w.d * 2 + h * w.d_k * r * 4 + w.d * h * w.d_v * 2
+                  for s, h in zip(w.scales, w.heads))
+    layer_bytes = 2 * B * L * w.d * 2 + weights
+    return {"kernels": out, "total_flops": total_flops, "layer_bytes": layer_bytes}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "scale_gated_linear_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None if
+    there is none or the kernel sources changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("source_hash") != kernel_source_hash():
+        return None
+    return t.get("kernels", {}).get(workload, {}).get(kernel)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 9 and (self.uuid is None or self.uuid in parts[0]):
+                self.rows.append(parts)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def numpy_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, inp, rows_budget_s: float, prefix: int | None = None):
+    """Run the fp64 oracle on whole batch rows (or a prefix of them) until about
+    `rows_budget_s` seconds have passed. Returns (tokens, seconds, description)."""
+    import numpy as np
+
+    import oracle
+    from scale_gated_linear_b200 import workloads as wl
+    f = wl.to_float64(inp)
+    L = f["X"].shape[1] if prefix is None else prefix
+    done, t0 = 0, time.perf_counter()
+    for b in range(f["X"].shape[0]):
+        oracle.layer_forward(f["X"][b:b + 1, :L], f, w.scales, w.heads, w.d_k, w.d_v,
+                             gate_normalizer=w.gate_normalizer)
+        done += 1
+        if time.perf_counter() - t0 >= rows_budget_s:
+            break
+    dt = time.perf_counter() - t0
+    desc = f"{done} batch row(s) x {L} positions of {w.name} (B={w.B}, L={w.L}), fp64 oracle, numpy"
+    return done * L, dt, desc
+
+
+# --------------------------------------------------------------------- reference arm
+def run_reference(args) -> int:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from scale_gated_linear_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    inp = wl.make_inputs(w, B=1)
+    prefix = min(w.L, args.ref_prefix)
+    times = []
+    for k in range(args.warmup + args.steps):
+        tok, dt, desc = oracle_sample(w, inp, 0.0, prefix=prefix)
+        if k >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = len(times) * prefix / total
+    cores = numpy_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: one sequence prefix of {prefix} of B={w.B} x L={w.L}, d={w.d}, "
+                               f"scales {list(w.scales)} heads {list(w.heads)}, d_k={w.d_k}, d_v={w.d_v}",
+                   "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: first {prefix} positions of one batch row (fp64 numpy oracle)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------- our arm
+def time_layer(layer, X, O, ws, steps: int, warmup: int, flush, n_events: int):
+    import torch
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(steps)]
+    wev = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
+    for _ in range(warmup):
+        flush()
+        layer.forward_profiled(X, O, ws, wev, stream)
+    return ev
+
+
+def run_ours(args) -> int:
+    import torch
+    import torch.distributed as dist
+
+    from scale_gated_linear_b200 import MSGLA
+    from scale_gated_linear_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = wl.WORKLOADS[args.workload]
+    peaks, peak_kind = load_peaks()
+    cpu_line = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp0 = wl.make_inputs(w, B=min(w.B, 4))
+        tok, dt, desc = oracle_sample(w, inp0, args.cpu_seconds)
+        cpu_line = {"value": tok / dt, "unit": UNIT, "cores": numpy_threads(), "kind": "oracle", "sample": desc}
+
+    def measure(wk, steps, warmup, e2e: bool):
+        inp = wl.make_inputs(wk)
+        if rank > 0:  # this rank's own batch of sequences (same weights)
+            g = torch.Generator().manual_seed(wk.seed * 1000 + rank)
+            X = torch.randn(wk.B, wk.L, wk.d, generator=g)
+            inp["X"] = (X / X.pow(2).mean(-1, keepdim=True).sqrt()).to(torch.bfloat16)
+        layer = MSGLA.from_workload(wk, inp, device=local)
+        X = inp["X"].to(dev)
+        O = torch.empty_like(X)
+        ws = layer.alloc_workspace(wk.B, wk.L)
+        flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        flush = lambda: flush_buf.fill_(1)
+        names = layer.launch_names()
+        n_ev = len(names) + 1
+        ev = time_layer(layer, X, O, ws, steps, warmup, flush, n_ev)
+        torch.cuda.synchronize()
+        layer.check_status()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        sampler = ClockSampler(getattr(torch.cuda.get_device_properties(dev), "uuid", None)
+                               and str(torch.cuda.get_device_properties(dev).uuid))
+        sampler.start()
+        time.sleep(0.3)
+        launches = 0
+        stream = torch.cuda.current_stream()
+        for k in range(steps):
+            flush()
+            launches += layer.forward_profiled(X, O, ws, ev[k], stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        clocks = sampler.stop()
+        layer.check_status()
+        step_ms = [ev[k][0].elapsed_time(ev[k][-1]) for k in range(steps)]
+        kern_ms = {n: [ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)] for i, n in enumerate(names)}
+        total_ms = max_over_ranks(sum(step_ms), world, dev)
+        res = {"total_ms": total_ms, "step_ms": step_ms, "kern_ms": kern_ms, "launches": launches,
+               "clocks": clocks, "tokens_per_step": wk.B * wk.L}
+        if e2e:
+            wsh = layer.alloc_workspace(wk.B, wk.L, host_staging=True)
+            Xh = inp["X"].pin_memory()
+            Oh = torch.empty_like(Xh).pin_memory()
+            for _ in range(max(1, warmup)):
+                layer.forward_host(Xh, Oh, wsh)
+            e_ms = []
+            for _ in range(steps):
+                flush()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                layer.forward_host(Xh, Oh, wsh, stream)
+                b.record(stream)
+                b.synchronize()
+                e_ms.append(a.elapsed_time(b))
+            res["e2e_ms"] = max_over_ranks(sum(e_ms), world, dev)
+            res["io_bytes"] = Xh.numel() * 2
+            del wsh
+        layer.close()
+        del ws, flush_buf
+        torch.cuda.empty_cache()
+        return res
+
+    r = measure(w, args.steps, args.warmup, e2e=not args.no_e2e)
+    tokens = r["tokens_per_step"] * args.steps * world
+    value = tokens / (r["total_ms"] / 1e3)
+    counts = algorithmic_counts(w, w.B, w.L)
+    mean_k = {n: statistics.mean(v) for n, v in r["kern_ms"].items()}
+    dominant = max(mean_k, key=mean_k.get)
+    kc = counts["kernels"][dominant]
+    if "flops" in kc:
+        achieved = kc["flops"] / (mean_k[dominant] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
+    else:
+        achieved = kc["bytes"] / (mean_k[dominant] * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
+    roof.update({"kernel": dominant, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst)"
+                 if peak_kind == "measured" else "fallback", "traffic": traffic_for(dominant, w.name),
+                 "kernel_ms": mean_k[dominant]})
+    step_ms = r["total_ms"] / args.steps
+    path_tf = counts["total_flops"] / (step_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16/bf16 tensor-core operands, f32 accumulate; bf16 in/out",
+        "data": "synthetic (seeded N(0,1) rows RMS-normalised, weights N(0,0.02))",
+        "config": {"workload": f"{w.name}: B={w.B} per GPU, L={w.L}, d={w.d}, scales {list(w.scales)} heads "
+                               f"{list(w.heads)}, d_k={w.d_k}, d_v={w.d_v}, gate rank {w.gate_rank}, chunk 64",
+                   "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"sequence-sharded x{world}",
+                   "l2": "flushed between timed steps (256 MiB write)"},
+        "roofline": roof,
+        "path_roofline": {"bound": "tensor", "achieved": path_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                          "frac": path_tf / peaks["bf16_tflops"], "flops_per_step": counts["total_flops"]},
+        "kernel_ms": mean_k,
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+    }
+    if "e2e_ms" in r:
+        line["e2e"] = {"value": tokens / (r["e2e_ms"] / 1e3), "unit": UNIT,
+                       "h2d_bytes_per_step": r["io_bytes"], "d2h_bytes_per_step": r["io_bytes"]}
+    if world == 1 and not args.no_gla_baseline:
+        g = measure(wl.WORKLOADS[BASELINE_WORKLOAD], max(3, args.steps // 2), args.warmup, e2e=False)
+        g_ms = g["total_ms"] / max(3, args.steps // 2)
+        line["gla_baseline"] = {"workload": BASELINE_WORKLOAD, "value": g["tokens_per_step"] / (g_ms * 1e-3),
+                                "unit": UNIT, "ms_per_step": g_ms, "time_ratio_msgla_over_gla": step_ms / g_ms}
+    if cpu_line is not None:
+        line["cpu_baseline"] = cpu_line
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gla-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU oracle baseline")
+    ap.add_argument("--ref-prefix", type=int, default=512, help="positions per reference-arm step")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -54,7 +54,7 @@ typedef struct msgla_config {
   int heads[MSGLA_MAX_SCALES];   /* h_s >= 1 for each scale; H = sum of heads             */
   int d_k;                       /* key width per head, 1..256                            */
   int d_v;                       /* value width per head, 1..1024                         */
-  int gate_rank;                 /* rank r of the gate projection, 1..64                  */
+  int gate_rank;                 /* rank r of the gate projection, 1..32                  */
   int chunk;                     /* chunk length of the chunkwise GLA kernel: 0 or 64.
                                     A compute parameter with no effect on the result
                                     beyond rounding (Sec. 3.4 of the notes).             */
@@ -109,9 +109,23 @@ int msgla_workspace_size(const msgla_handle* h, int B, int L, size_t* bytes);
  *   stream     cudaStream_t (NULL = legacy default stream).
  * Asynchronous: returns after enqueuing the kernels on `stream`. Errors found by
  * the kernels (timeouts, fp16 range) are latched in the handle and reported by
- * msgla_sync_status (and by the next msgla_forward). B*L = 0 launches nothing. */
+ * msgla_sync_status. B*L = 0 launches nothing. */
 int msgla_forward(msgla_handle* h, const void* X, int B, int L, void* O,
                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* msgla_forward that also records CUDA events around its kernels, for timing each
+ * kernel on `stream` with events. `events` holds caller-created cudaEvent_t
+ * handles: events[0] is recorded before the first kernel and events[i+1] after
+ * the i-th kernel. The kernels of one forward, in launch order, are:
+ *   pool_fuse, proj_gemm, gate (all scales), gla,
+ *   out_gemm_coarse (only when a scale-1 branch and a coarser branch exist),
+ *   out_gemm_fused (scale-1 branch present) or, without a scale-1 branch,
+ *   out_gemm_coarse for all branches followed by hold_fuse.
+ * `max_events` is the length of `events` (it must be at least n_launches + 1);
+ * *n_launches receives the number of kernels launched. */
+int msgla_forward_profiled(msgla_handle* h, const void* X, int B, int L, void* O,
+                           void* workspace, size_t workspace_bytes, void* stream,
+                           void* const* events, int max_events, int* n_launches);
 
 /* Workspace for msgla_forward_host: msgla_workspace_size plus room to stage X and O. */
 int msgla_workspace_size_host(const msgla_handle* h, int B, int L, size_t* bytes);

@@ -107,6 +107,36 @@ class MSGLA:
 
     __call__ = forward
 
+    def launch_names(self):
+        """Kernel names of one forward, in launch order (see msgla_forward_profiled)."""
+        names = ["pool_fuse", "proj_gemm", "gate", "gla"]
+        if 1 in self.scales:
+            if len(self.scales) > 1:
+                names.append("out_gemm_coarse")
+            names.append("out_gemm_fused")
+        else:
+            names += ["out_gemm_coarse", "hold_fuse"]
+        return names
+
+    def forward_profiled(self, X, out, workspace, events, stream=None):
+        """forward() recording events[0] before the first kernel and events[i+1]
+        after kernel i (torch.cuda.Event objects with timing enabled). Returns the
+        number of kernels launched."""
+        import torch
+        B, L, d = X.shape
+        if stream is None:
+            stream = torch.cuda.current_stream(X.device)
+        for e in events:  # torch creates the underlying cudaEvent_t on first record
+            if not e.cuda_event:
+                e.record(stream)
+        arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        n = ctypes.c_int()
+        _lib.check(self._lib.msgla_forward_profiled(self._h, X.data_ptr(), B, L, out.data_ptr(),
+                                                    workspace.data_ptr(), workspace.numel(),
+                                                    ctypes.c_void_p(stream.cuda_stream), arr, len(events),
+                                                    ctypes.byref(n)))
+        return n.value
+
     def forward_host(self, X_host, O_host, workspace, stream=None):
         """Host-buffer forward: X_host, O_host are CPU bf16 [B, L, d] (pinned for
         speed); copies in, runs, copies out and synchronises."""

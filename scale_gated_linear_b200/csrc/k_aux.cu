@@ -128,52 +128,224 @@ __global__ void __launch_bounds__(kPoolThreads) pool_fuse_kernel(const PoolParam
   }
 }
 
-constexpr int kGateRows = kChunk;
-
-// grid (n_chunks, heads, B); block dkp/2 threads, two channels per thread.
-__global__ void gate_kernel(const GateParams p) {
-  extern __shared__ float gsm[];
-  float* g_s = gsm;                       // [64][rp]
-  float* w_s = gsm + kGateRows * p.rp;    // [dkp][rp]
-  const int c = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
-  const int t0 = c * kGateRows;
-  const int nrows = min(kGateRows, p.rows - t0);
-  const int ldk = p.heads * p.dkp;
-  for (int i = threadIdx.x; i < nrows * p.rp; i += blockDim.x)
-    g_s[i] = p.g[(static_cast<size_t>(b) * p.rows + t0) * p.rp + i];
-  for (int i = threadIdx.x; i < p.dkp * p.rp; i += blockDim.x)
-    w_s[i] = p.Wg2[static_cast<size_t>(head) * p.dkp * p.rp + i];
+// Streaming form for scale sets whose coarse scales all divide P (P <= 8): one
+// warp per block of P rows of one sequence. Each lane loads P x 16 bytes per
+// column group before using any of them (memory-level parallelism), forms the
+// pooled rows of every coarse scale and the partial fusion logits; the logits
+// are reduced across the warp once per row at the end.
+template <int P>
+__global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p) {
+  extern __shared__ float wf_s[];  // [n_scales][d] fp32
+  const int ns = p.n_scales;
+  for (int i = threadIdx.x; i < ns * p.d; i += blockDim.x) wf_s[i] = __bfloat162float(p.Wfuse[i]);
   __syncthreads();
-  const int a0 = 2 * threadIdx.x;
-  const int ch = head * p.dkp + a0;
-  const float bias0 = p.bg[ch], bias1 = p.bg[ch + 1];
-  const float* w0 = w_s + a0 * p.rp;
-  const float* w1 = w0 + p.rp;
-  float b0 = 0.f, b1 = 0.f;
-  bool bad = false;
-  for (int i = 0; i < nrows; ++i) {
-    float z0 = bias0, z1 = bias1;
-    const float* gi = g_s + i * p.rp;
-    for (int r = 0; r < p.rp; ++r) {
-      z0 = fmaf(gi[r], w0[r], z0);
-      z1 = fmaf(gi[r], w1[r], z1);
+  const int lane = threadIdx.x & 31;
+  const int blocks_per_seq = (p.L + P - 1) / P;
+  const size_t gw = blockIdx.x * static_cast<size_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (gw >= static_cast<size_t>(p.B) * blocks_per_seq) return;
+  const int b = static_cast<int>(gw / blocks_per_seq);
+  const int row0 = static_cast<int>(gw % blocks_per_seq) * P;
+  const int nrows = min(P, p.L - row0);
+  const __nv_bfloat16* Xb = p.X + (static_cast<size_t>(b) * p.L + row0) * p.d;
+  float part[P][kMaxScales];
+#pragma unroll
+  for (int r = 0; r < P; ++r)
+#pragma unroll
+    for (int j = 0; j < kMaxScales; ++j) part[r][j] = 0.f;
+  const int groups = p.d / 8;
+  for (int cg = lane; cg < groups; cg += 32) {
+    float x[P][8];
+#pragma unroll
+    for (int r = 0; r < P; ++r) {
+      if (r < nrows) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(Xb + static_cast<size_t>(r) * p.d) + cg);
+        bf16x8_to_f32(u, x[r]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[r][e] = 0.f;
+      }
     }
-    // logsigmoid(z) = min(z, 0) - log(1 + e^{-|z|})
-    b0 += (fminf(z0, 0.f) - log1pf(__expf(-fabsf(z0)))) * p.inv_normalizer;
-    b1 += (fminf(z1, 0.f) - log1pf(__expf(-fabsf(z1)))) * p.inv_normalizer;
-    const size_t idx = (static_cast<size_t>(b) * p.rows + t0 + i) * ldk + ch;
-    const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(p.q + idx));
-    const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(p.k + idx));
-    const float e0 = __expf(b0), e1 = __expf(b1);
-    const float ks0 = kf.x * __expf(-b0), ks1 = kf.y * __expf(-b1);
-    bad |= !(fabsf(ks0) <= 65504.f) || !(fabsf(ks1) <= 65504.f);
-    *reinterpret_cast<__half2*>(p.qs + idx) = __floats2half2_rn(qf.x * e0, qf.y * e1);
-    *reinterpret_cast<__half2*>(p.ks + idx) = __floats2half2_rn(ks0, ks1);
+#pragma unroll
+    for (int j = 0; j < kMaxScales; ++j) {
+      if (j >= ns) break;
+      const float4 wa = *reinterpret_cast<const float4*>(wf_s + j * p.d + cg * 8);
+      const float4 wb = *reinterpret_cast<const float4*>(wf_s + j * p.d + cg * 8 + 4);
+#pragma unroll
+      for (int r = 0; r < P; ++r)
+        part[r][j] += x[r][0] * wa.x + x[r][1] * wa.y + x[r][2] * wa.z + x[r][3] * wa.w + x[r][4] * wb.x +
+                      x[r][5] * wb.y + x[r][6] * wb.z + x[r][7] * wb.w;
+      const int s = p.scales[j];
+      if (s == 1) continue;
+      const int n_s = (p.L + s - 1) / s;
+      for (int i0 = 0; i0 < P; i0 += s) {
+        if (i0 >= nrows) break;
+        const int cnt = min(s, nrows - i0);
+        float m[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m[e] = 0.f;
+#pragma unroll
+        for (int r = 0; r < P; ++r)
+          if (r >= i0 && r < i0 + cnt)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m[e] += x[r][e];
+        const float inv = 1.f / static_cast<float>(cnt);
+        uint4 o;
+        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+        bool bad = false;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a0 = m[2 * e] * inv, a1 = m[2 * e + 1] * inv;
+          bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
+          ow[e] = pack_half2(a0, a1);
+        }
+        if (bad) atomicCAS(p.err, 0, kDevRange);
+        const int i = (row0 + i0) / s;
+        reinterpret_cast<uint4*>(p.Xp[j] + (static_cast<size_t>(b) * n_s + i) * p.d)[cg] = o;
+      }
+    }
   }
-  float* gm = p.gamma + (static_cast<size_t>(b) * p.n_chunks + c) * ldk + ch;
-  gm[0] = __expf(b0);
-  gm[1] = __expf(b1);
+#pragma unroll
+  for (int r = 0; r < P; ++r) {
+    float z[kMaxScales];
+    float zmax = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kMaxScales; ++j) {
+      float v = part[r][j];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      z[j] = v + ((j < ns && p.bfuse) ? p.bfuse[j] : 0.f);
+      if (j < ns) zmax = fmaxf(zmax, z[j]);
+    }
+    if (lane == 0 && r < nrows) {
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxScales; ++j) {
+        z[j] = j < ns ? __expf(z[j] - zmax) : 0.f;
+        sum += z[j];
+      }
+      float* wr = p.w + (static_cast<size_t>(b) * p.L + row0 + r) * ns;
+      for (int j = 0; j < ns; ++j) wr[j] = z[j] / sum;
+    }
+  }
+}
+
+constexpr int kGateThreads = 512;
+
+// One CTA per (branch, batch, head, chunk); 512 threads = (dkp/2 channel pairs) x
+// (row groups of 64/groups rows). Every thread issues all of its q/k loads first,
+// computes log alpha for its rows, a local cumulative sum, then adds the totals of
+// the preceding row groups (through shared memory) to get b, and writes
+// Qs = q e^{b}, Ks = k e^{-b}; gamma = e^{b at the chunk's last row}.
+template <int RP, int R>
+__global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constant__ GateParams p) {
+  extern __shared__ float gsm[];
+  constexpr int kGroups = kChunk / R;
+  const int dkp = p.dkp;
+  const int pairs = dkp / 2;  // == kGateThreads / kGroups
+  float* g_s = gsm;                  // [64][RP]
+  float* w_s = g_s + kChunk * RP;    // [dkp][RP]
+  float* tot = w_s + dkp * RP;       // [kGroups][dkp]
+  int bi = 0;
+#pragma unroll 1
+  for (int j = 1; j < p.n_branches; ++j)
+    if (static_cast<int>(blockIdx.x) >= p.br[j].block_begin) bi = j;
+  const GateBranch& P = p.br[bi];
+  const int local = blockIdx.x - P.block_begin;
+  const int c = local % P.n_chunks;
+  const int head = (local / P.n_chunks) % P.heads;
+  const int b = local / (P.n_chunks * P.heads);
+  const int t0 = c * kChunk;
+  const int nrows = min(kChunk, P.rows - t0);
+  const int ldk = P.heads * dkp;
+
+  const int pair = threadIdx.x % pairs, grp = threadIdx.x / pairs;
+  const int a0 = 2 * pair;
+  const int ch = head * dkp + a0;
+  const int r0 = grp * R;
+  // issue the q/k loads of this thread's rows first
+  __half2 qv[R], kv[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (r0 + r < nrows) {
+      const size_t idx = (static_cast<size_t>(b) * P.rows + t0 + r0 + r) * ldk + ch;
+      qv[r] = *reinterpret_cast<const __half2*>(P.q + idx);
+      kv[r] = *reinterpret_cast<const __half2*>(P.k + idx);
+    }
+  }
+  for (int i = threadIdx.x; i < nrows * RP; i += blockDim.x)
+    g_s[i] = P.g[(static_cast<size_t>(b) * P.rows + t0) * RP + i];
+  for (int i = threadIdx.x; i < dkp * RP; i += blockDim.x) w_s[i] = P.Wg2[static_cast<size_t>(head) * dkp * RP + i];
+  __syncthreads();
+  float w0[RP], w1[RP];
+#pragma unroll
+  for (int r = 0; r < RP; ++r) {
+    w0[r] = w_s[a0 * RP + r];
+    w1[r] = w_s[(a0 + 1) * RP + r];
+  }
+  const float bias0 = P.bg[ch], bias1 = P.bg[ch + 1];
+  float c0[R], c1[R];
+  float run0 = 0.f, run1 = 0.f;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (r0 + r < nrows) {
+      const float* gi = g_s + (r0 + r) * RP;
+      float z0 = bias0, z1 = bias1;
+#pragma unroll
+      for (int u = 0; u < RP; ++u) {
+        z0 = fmaf(gi[u], w0[u], z0);
+        z1 = fmaf(gi[u], w1[u], z1);
+      }
+      // logsigmoid(z) = min(z, 0) - log(1 + e^{-|z|})
+      run0 += (fminf(z0, 0.f) - log1pf(__expf(-fabsf(z0)))) * p.inv_normalizer;
+      run1 += (fminf(z1, 0.f) - log1pf(__expf(-fabsf(z1)))) * p.inv_normalizer;
+    }
+    c0[r] = run0;
+    c1[r] = run1;
+  }
+  tot[grp * dkp + a0] = run0;
+  tot[grp * dkp + a0 + 1] = run1;
+  __syncthreads();
+  float pre0 = 0.f, pre1 = 0.f, all0 = 0.f, all1 = 0.f;
+#pragma unroll
+  for (int g2 = 0; g2 < kGroups; ++g2) {
+    const float x0 = tot[g2 * dkp + a0], x1 = tot[g2 * dkp + a0 + 1];
+    if (g2 < grp) {
+      pre0 += x0;
+      pre1 += x1;
+    }
+    all0 += x0;
+    all1 += x1;
+  }
+  bool bad = false;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (r0 + r < nrows) {
+      const float b0 = pre0 + c0[r], b1 = pre1 + c1[r];
+      const float2 qf = __half22float2(qv[r]);
+      const float2 kf = __half22float2(kv[r]);
+      const float ks0 = kf.x * __expf(-b0), ks1 = kf.y * __expf(-b1);
+      bad |= !(fabsf(ks0) <= 65504.f) || !(fabsf(ks1) <= 65504.f);
+      const size_t idx = (static_cast<size_t>(b) * P.rows + t0 + r0 + r) * ldk + ch;
+      *reinterpret_cast<__half2*>(P.qs + idx) = __floats2half2_rn(qf.x * __expf(b0), qf.y * __expf(b1));
+      *reinterpret_cast<__half2*>(P.ks + idx) = __floats2half2_rn(ks0, ks1);
+    }
+  }
+  if (grp == 0) {
+    float* gm = P.gamma + (static_cast<size_t>(b) * P.n_chunks + c) * ldk + ch;
+    gm[0] = __expf(all0);
+    gm[1] = __expf(all1);
+  }
   if (bad) atomicCAS(p.err, 0, kDevRange);
+}
+
+template <int RP, int R>
+cudaError_t launch_gate_t(const GateParams& p, cudaStream_t st) {
+  const int groups = kChunk / R;
+  const int smem = (kChunk * RP + p.dkp * RP + groups * p.dkp) * static_cast<int>(sizeof(float));
+  cudaError_t e = cudaFuncSetAttribute(gate_kernel<RP, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  gate_kernel<RP, R><<<p.total_blocks, kGateThreads, smem, st>>>(p);
+  return cudaGetLastError();
 }
 
 // one thread per 8 output columns of one row; flat grid over B*L*(d/8)
@@ -232,23 +404,35 @@ __global__ void bf16_copy_rows_kernel(const __nv_bfloat16* src, int src_ld, int 
 
 }  // namespace
 
+template <int P>
+cudaError_t launch_pool_rows(const PoolParams& p, cudaStream_t st) {
+  const int smem = p.n_scales * p.d * static_cast<int>(sizeof(float));
+  cudaError_t e = cudaFuncSetAttribute(pool_fuse_rows_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const size_t warps = static_cast<size_t>(p.B) * ((p.L + P - 1) / P);
+  pool_fuse_rows_kernel<P><<<static_cast<unsigned>((warps + 7) / 8), 256, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st) {
   if (p.B * p.L == 0) return cudaSuccess;
-  dim3 grid((p.L + p.block_rows - 1) / p.block_rows, p.B);
-  pool_fuse_kernel<<<grid, kPoolThreads, 0, st>>>(p);
+  // block_rows carries the least common multiple of the coarse scales (1 if none)
+  if (p.block_rows <= 4 && p.n_scales * p.d * 4 <= 160 * 1024) return launch_pool_rows<4>(p, st);
+  if (p.block_rows == 8 && p.n_scales * p.d * 4 <= 160 * 1024) return launch_pool_rows<8>(p, st);
+  PoolParams q = p;
+  q.block_rows = p.block_rows;
+  while (q.block_rows < 32) q.block_rows *= 2;
+  dim3 grid((p.L + q.block_rows - 1) / q.block_rows, p.B);
+  pool_fuse_kernel<<<grid, kPoolThreads, 0, st>>>(q);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gate(const GateParams& p, cudaStream_t st) {
-  if (p.B * p.rows == 0) return cudaSuccess;
-  const int smem = (kGateRows + p.dkp) * p.rp * static_cast<int>(sizeof(float));
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-  }
-  dim3 grid(p.n_chunks, p.heads, p.B);
-  gate_kernel<<<grid, p.dkp / 2, smem, st>>>(p);
-  return cudaGetLastError();
+  if (p.total_blocks <= 0) return cudaSuccess;
+  // 512 threads = (dkp/2) channel pairs x groups; rows per group R = 64 / groups
+  if (p.dkp == 256) return p.rp == 16 ? launch_gate_t<16, 16>(p, st) : launch_gate_t<32, 16>(p, st);
+  if (p.dkp == 128) return p.rp == 16 ? launch_gate_t<16, 8>(p, st) : launch_gate_t<32, 8>(p, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_hold_fuse(const HoldFuseParams& p, cudaStream_t st) {

@@ -15,7 +15,8 @@
 // 64 rows are ignored.
 //
 // One CTA = (batch, branch, head, 128-column value tile), looping over chunks:
-//   warp 0        TMA loads of Qs, Ks (64 x dkp) and V (64 x 128) per chunk
+//   warp 0        TMA loads of Qs, Ks (64 x dkp, double-buffered: chunk c+1 is
+//                 fetched while chunk c computes) and V (64 x 128) per chunk
 //   warp 1        TMEM allocation (512 columns) + tcgen05.mma issue
 //   warps 4..7    score epilogue (mask, fp16 into shared memory) and the o store
 //   warps 8..15   state epilogue: S <- gamma * S in TMEM, fp16 copy of S for the
@@ -30,18 +31,24 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kAtom = 64 * 128;  // one 64-row x 128-byte swizzle block (8 KB)
-// shared memory map (bytes from the 1024-aligned base)
-constexpr int kOffQ = 0;                      // Qs: up to 4 atoms (d_k <= 256)
-constexpr int kOffK = kOffQ + 4 * kAtom;      // Ks: up to 4 atoms
-constexpr int kOffV = kOffK + 4 * kAtom;      // V: 2 atoms (128 value columns)
+// shared memory map (bytes from the 1024-aligned base). The score MMA reads 128
+// rows of Ks, i.e. up to 8 KB past a stage's last atom: that lands in the next
+// buffer, never outside the allocation.
+constexpr int kStageQK = 8 * kAtom;           // Qs (4 atoms) + Ks (4 atoms), d_k <= 256
+constexpr int kOffQK = 0;                     // 2 stages
+constexpr int kOffV = kOffQK + 2 * kStageQK;  // V: 2 atoms (128 value columns)
 constexpr int kOffS = kOffV + 2 * kAtom;      // S^T fp16: 2 MN blocks x 256 rows x 128 B
 constexpr int kOffA = kOffS + 2 * 256 * 128;  // A^T fp16: 64 rows x 128 B
 constexpr int kOffBar = kOffA + kAtom;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 constexpr uint32_t kColS = 0, kColO = 256, kColA = 320;
 
-enum { B_IN_FULL = 0, B_IN_EMPTY, B_A_FULL, B_A_SMEM, B_O_FULL, B_O_EMPTY, B_S_FULL, B_S_DONE, B_COUNT };
+enum {
+  B_QK_FULL0 = 0, B_QK_FULL1, B_QK_EMPTY0, B_QK_EMPTY1, B_V_FULL, B_V_EMPTY,
+  B_A_FULL, B_A_SMEM, B_O_FULL, B_O_EMPTY, B_S_FULL, B_S_DONE, B_COUNT
+};
 
 __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_constant__ GlaParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -65,8 +72,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
-    mbar_init(&bar[B_IN_FULL], 1);
-    mbar_init(&bar[B_IN_EMPTY], 1);
+    mbar_init(&bar[B_QK_FULL0], 1);
+    mbar_init(&bar[B_QK_FULL1], 1);
+    mbar_init(&bar[B_QK_EMPTY0], 1);
+    mbar_init(&bar[B_QK_EMPTY1], 1);
+    mbar_init(&bar[B_V_FULL], 1);
+    mbar_init(&bar[B_V_EMPTY], 1);
     mbar_init(&bar[B_A_FULL], 1);
     mbar_init(&bar[B_A_SMEM], 128);
     mbar_init(&bar[B_O_FULL], 1);
@@ -88,44 +99,56 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer
+      // ---------------- TMA producer: Qs/Ks of chunk c into stage c&1, V of chunk c
       prefetch_tmap(&T.tmQ);
       prefetch_tmap(&T.tmK);
       prefetch_tmap(&T.tmV);
-      const uint32_t bytes = static_cast<uint32_t>((2 * (dkp / 64) + 2) * kAtom);
+      const uint32_t qk_bytes = static_cast<uint32_t>(2 * (dkp / 64) * kAtom);
       for (int c = 0; c < nch; ++c) {
-        if (c > 0 && !mbar_wait(&bar[B_IN_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(&bar[B_IN_FULL], bytes);
+        const int st = c & 1;
+        if (c >= 2 && !mbar_wait(&bar[B_QK_EMPTY0 + st], ((c >> 1) - 1) & 1, abort_flag, p.err)) break;
+        uint8_t* sq = smem + kOffQK + st * kStageQK;
+        mbar_arrive_expect_tx(&bar[B_QK_FULL0 + st], qk_bytes);
         for (int ka = 0; ka < dkp / 64; ++ka) {
-          tma_load_3d(&T.tmQ, &bar[B_IN_FULL], smem + kOffQ + ka * kAtom, head * dkp + ka * 64, c * kChunk, b);
-          tma_load_3d(&T.tmK, &bar[B_IN_FULL], smem + kOffK + ka * kAtom, head * dkp + ka * 64, c * kChunk, b);
+          tma_load_3d(&T.tmQ, &bar[B_QK_FULL0 + st], sq + ka * kAtom, head * dkp + ka * 64, c * kChunk, b);
+          tma_load_3d(&T.tmK, &bar[B_QK_FULL0 + st], sq + (4 + ka) * kAtom, head * dkp + ka * 64, c * kChunk, b);
         }
+        if (c >= 1 && !mbar_wait(&bar[B_V_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
+        mbar_arrive_expect_tx(&bar[B_V_FULL], 2 * kAtom);
         for (int mb = 0; mb < 2; ++mb)
-          tma_load_3d(&T.tmV, &bar[B_IN_FULL], smem + kOffV + mb * kAtom,
-                      head * T.dvp + vt * kGlaTile + mb * 64, c * kChunk, b);
+          tma_load_3d(&T.tmV, &bar[B_V_FULL], smem + kOffV + mb * kAtom, head * T.dvp + vt * kGlaTile + mb * 64,
+                      c * kChunk, b);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer
+      // ---------------- MMA issuer. Per chunk: o^T(c), S update(c), scores(c+1).
       const uint32_t id_at = idesc_f16(128, 64, 0, 0, 0);   // Ks (K-major) x Qs (K-major)
       const uint32_t id_os = idesc_f16(128, 64, 0, 1, 0);   // S^T (MN-major) x Qs (K-major)
       const uint32_t id_ov = idesc_f16(128, 64, 0, 1, 1);   // V^T (MN-major) x A^T rows (MN-major)
       const uint32_t id_ds = idesc_f16(128, 128, 0, 1, 1);  // Ks^T (MN-major) x V (MN-major)
-      const uint32_t sQ = sbase + kOffQ, sK = sbase + kOffK, sV = sbase + kOffV;
-      const uint32_t sS = sbase + kOffS, sA = sbase + kOffA;
+      const uint32_t sV = sbase + kOffV, sS = sbase + kOffS, sA = sbase + kOffA;
       const uint32_t lbo_s = static_cast<uint32_t>(dkp) * 128;
-      for (int c = 0; c < nch; ++c) {
-        if (!mbar_wait(&bar[B_IN_FULL], c & 1, abort_flag, p.err)) break;
-        tc_fence_after();
+      auto scores = [&](int c) {
         // A^T[j][i] = sum_a Ks[j][a] Qs[i][a]
+        const uint32_t sQ = sbase + kOffQK + (c & 1) * kStageQK, sK = sQ + 4 * kAtom;
         for (int ka = 0; ka < dkp / 64; ++ka)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_f16(tmem + kColA, sdesc_sw128(sK + ka * kAtom + kk * 32, 16, 1024),
                      sdesc_sw128(sQ + ka * kAtom + kk * 32, 16, 1024), id_at, (ka | kk) != 0);
         umma_commit(&bar[B_A_FULL]);
+      };
+      bool ok = mbar_wait(&bar[B_QK_FULL0], 0, abort_flag, p.err);
+      if (ok) {
+        tc_fence_after();
+        scores(0);
+      }
+      for (int c = 0; c < nch && ok; ++c) {
+        const int st = c & 1;
+        const uint32_t sQ = sbase + kOffQK + st * kStageQK, sK = sQ + 4 * kAtom;
         if (!mbar_wait(&bar[B_A_SMEM], c & 1, abort_flag, p.err)) break;
+        if (!mbar_wait(&bar[B_V_FULL], c & 1, abort_flag, p.err)) break;
         if (c > 0) {
           if (!mbar_wait(&bar[B_S_DONE], (c - 1) & 1, abort_flag, p.err)) break;
           if (!mbar_wait(&bar[B_O_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
@@ -155,7 +178,13 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
             umma_f16(tmem + kColS + h * 128, sdesc_sw128(sK + 2 * h * kAtom + ks * 2048, kAtom, 1024),
                      sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_ds, (c > 0 || ks > 0) ? 1u : 0u);
         umma_commit(&bar[B_S_FULL]);
-        umma_commit(&bar[B_IN_EMPTY]);
+        umma_commit(&bar[B_V_EMPTY]);
+        umma_commit(&bar[B_QK_EMPTY0 + st]);
+        if (c + 1 < nch) {
+          if (!mbar_wait(&bar[B_QK_FULL0 + ((c + 1) & 1)], ((c + 1) >> 1) & 1, abort_flag, p.err)) break;
+          tc_fence_after();
+          scores(c + 1);
+        }
       }
     }
   } else if (warp >= 4 && warp < 8) {
@@ -200,9 +229,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
       const int col = head * T.dvp + vt * kGlaTile + j;
       const int t0 = c * kChunk;
       __half* dst = T.o + (static_cast<size_t>(b) * T.rows + t0) * ld_o + col;
+      const int nvalid = min(kChunk, T.rows - t0);
 #pragma unroll
       for (int i = 0; i < kChunk; ++i) {
-        if (t0 + i < T.rows) {
+        if (i < nvalid) {
           const float x = __uint_as_float(i < 32 ? r0[i & 31] : r1[i & 31]);
           dst[static_cast<size_t>(i) * ld_o] = __float2half_rn(p.qk_scale * x);
         }
@@ -216,35 +246,43 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
       const int a = g * 128 + quad * 32 + lane;  // d_k row
       uint8_t* sS = smem + kOffS;
       const size_t ld_g = static_cast<size_t>(T.heads) * dkp;
+      const float* gp = T.gamma + static_cast<size_t>(b) * nch * ld_g + head * dkp + a;
+      float gam = __ldg(gp);
       for (int c = 0; c < nch; ++c) {
-        const float gam = __ldg(T.gamma + (static_cast<size_t>(b) * nch + c) * ld_g + head * dkp + a);
+        const float gam_next = (c + 1 < nch) ? __ldg(gp + (c + 1) * ld_g) : 0.f;
         if (!mbar_wait(&bar[B_S_FULL], c & 1, abort_flag, p.err)) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t r[32];
-          const uint32_t ta = tmem_addr(tmem, quad * 32, kColS + g * 128 + q4 * 32);
-          tmem_ld32(ta, r);
+        for (int q2 = 0; q2 < 2; ++q2) {
+          uint32_t ra[32], rb[32];
+          const uint32_t ta = tmem_addr(tmem, quad * 32, kColS + g * 128 + q2 * 64);
+          tmem_ld32(ta, ra);
+          tmem_ld32(ta + 32, rb);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(gam * __uint_as_float(r[e]));
-          tmem_st32(ta, r);
-          // value columns q4*32 .. q4*32+31 -> MN block q4/2, 16-byte chunks (q4%2)*4 .. +3
-          const int mb = q4 >> 1;
+          for (int e = 0; e < 32; ++e) {
+            ra[e] = __float_as_uint(gam * __uint_as_float(ra[e]));
+            rb[e] = __float_as_uint(gam * __uint_as_float(rb[e]));
+          }
+          tmem_st32(ta, ra);
+          tmem_st32(ta + 32, rb);
+          // value columns q2*64 .. q2*64+63 -> MN block q2, 16-byte chunks 0..7
+          uint8_t* row = sS + q2 * dkp * 128 + a * 128;
 #pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            const int cc = (q4 & 1) * 4 + e4;
-            const uint32_t addr = smem_u32(sS + mb * dkp * 128 + a * 128 + ((cc ^ (a & 7)) << 4));
-            st_shared_v4(addr, pack_half2(__uint_as_float(r[8 * e4 + 0]), __uint_as_float(r[8 * e4 + 1])),
-                         pack_half2(__uint_as_float(r[8 * e4 + 2]), __uint_as_float(r[8 * e4 + 3])),
-                         pack_half2(__uint_as_float(r[8 * e4 + 4]), __uint_as_float(r[8 * e4 + 5])),
-                         pack_half2(__uint_as_float(r[8 * e4 + 6]), __uint_as_float(r[8 * e4 + 7])));
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const uint32_t* r = e4 < 4 ? ra + 8 * e4 : rb + 8 * (e4 - 4);
+            st_shared_v4(smem_u32(row + ((e4 ^ (a & 7)) << 4)),
+                         pack_half2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                         pack_half2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                         pack_half2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                         pack_half2(__uint_as_float(r[6]), __uint_as_float(r[7])));
           }
         }
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bar[B_S_DONE]);
+        gam = gam_next;
       }
     }
   }

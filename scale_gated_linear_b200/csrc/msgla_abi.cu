@@ -285,8 +285,26 @@ int create_impl(msgla_handle* h, const msgla_weights* w) {
   return MSGLA_OK;
 }
 
+// Optional per-launch event recording (msgla_forward_profiled).
+struct Recorder {
+  void* const* events = nullptr;
+  int max_events = 0;
+  int n = 0;
+  cudaError_t mark(cudaStream_t st) {
+    if (!events) return cudaSuccess;
+    if (n + 1 >= max_events) return cudaErrorInvalidValue;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[++n]), st);
+  }
+};
+
 int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* wsp, size_t ws_bytes,
-                 cudaStream_t st) {
+                 cudaStream_t st, Recorder* rec = nullptr) {
+  Recorder none;
+  if (!rec) rec = &none;
+  if (rec->events) {
+    if (rec->max_events < 1) return fail(MSGLA_ERR_INVALID_ARG, "max_events < 1");
+    CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(rec->events[0]), st));
+  }
   const msgla_config& c = h->cfg;
   const int d = c.d;
   const Workspace ws = layout(h, B, L);
@@ -314,6 +332,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   pp.block_rows = h->pool_rows;
   pp.err = h->d_err;
   CUDA_TRY(launch_pool_fuse(pp, st));
+  CUDA_TRY(rec->mark(st));
 
   // 2. projections (grouped over branches)
   static thread_local GemmParams gp;
@@ -348,29 +367,38 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   gp.n_tasks = ns;
   gp.total_tiles = tiles;
   CUDA_TRY(launch_gemm(gp, 256, st));
+  CUDA_TRY(rec->mark(st));
 
-  // 3. gates
-  for (int j = 0; j < ns; ++j) {
-    const Branch& b = h->br[j];
-    const BranchWs& bw = ws.br[j];
+  // 3. gates (one launch over all branches)
+  {
     GateParams g{};
-    g.q = static_cast<const __half*>(at(bw.q));
-    g.k = static_cast<const __half*>(at(bw.k));
-    g.g = static_cast<const float*>(at(bw.g));
-    g.Wg2 = b.Wg2p;
-    g.bg = b.bgp;
-    g.qs = static_cast<__half*>(at(bw.qs));
-    g.ks = static_cast<__half*>(at(bw.ks));
-    g.gamma = static_cast<float*>(at(bw.gamma));
-    g.B = B;
-    g.rows = bw.rows;
-    g.heads = b.heads;
+    int blocks = 0;
+    for (int j = 0; j < ns; ++j) {
+      const Branch& b = h->br[j];
+      const BranchWs& bw = ws.br[j];
+      GateBranch& q = g.br[j];
+      q.q = static_cast<const __half*>(at(bw.q));
+      q.k = static_cast<const __half*>(at(bw.k));
+      q.g = static_cast<const float*>(at(bw.g));
+      q.Wg2 = b.Wg2p;
+      q.bg = b.bgp;
+      q.qs = static_cast<__half*>(at(bw.qs));
+      q.ks = static_cast<__half*>(at(bw.ks));
+      q.gamma = static_cast<float*>(at(bw.gamma));
+      q.rows = bw.rows;
+      q.heads = b.heads;
+      q.n_chunks = bw.n_chunks;
+      q.block_begin = blocks;
+      blocks += B * b.heads * bw.n_chunks;
+    }
+    g.n_branches = ns;
+    g.total_blocks = blocks;
     g.dkp = h->dkp;
     g.rp = h->rp;
-    g.n_chunks = bw.n_chunks;
     g.inv_normalizer = 1.f / c.gate_normalizer;
     g.err = h->d_err;
     CUDA_TRY(launch_gate(g, st));
+    CUDA_TRY(rec->mark(st));
   }
 
   // 4. chunkwise GLA (grouped over branches; longest sequences first)
@@ -401,6 +429,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   lp.n_tasks = ns;
   lp.total_ctas = ctas;
   CUDA_TRY(launch_gla(lp, st));
+  CUDA_TRY(rec->mark(st));
 
   // 5. coarse branches: Y^(s) = o W_o^T (fp16)
   memset(&gp, 0, sizeof(gp));
@@ -430,6 +459,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     gp.n_tasks = nt;
     gp.total_tiles = tiles;
     CUDA_TRY(launch_gemm(gp, 256, st));
+    CUDA_TRY(rec->mark(st));
   }
 
   // 6. scale-1 branch fused with hold + fusion, or the stand-alone hold + fusion
@@ -468,6 +498,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     gp.n_tasks = 1;
     gp.total_tiles = B * t.m_tiles * t.n_tiles;
     CUDA_TRY(launch_gemm(gp, 256, st));
+    CUDA_TRY(rec->mark(st));
   } else {
     HoldFuseParams hp{};
     for (int j = 0; j < ns; ++j) {
@@ -482,6 +513,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     hp.d = d;
     hp.n_scales = ns;
     CUDA_TRY(launch_hold_fuse(hp, st));
+    CUDA_TRY(rec->mark(st));
   }
   return MSGLA_OK;
 }
@@ -539,8 +571,7 @@ int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weight
     if (cfg->scales[j] == 1) h->main_index = j;
     else lcm = lcm / gcd(lcm, cfg->scales[j]) * cfg->scales[j];
   }
-  h->pool_rows = lcm;
-  while (h->pool_rows < 32) h->pool_rows *= 2;
+  h->pool_rows = lcm;  // least common multiple of the coarse scales
   st = create_impl(h, w);
   if (st) {
     const std::string msg = g_last_error;
@@ -589,6 +620,27 @@ int msgla_forward(msgla_handle* h, const void* X, int B, int L, void* O, void* w
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
   return forward_impl(h, X, B, L, O, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int msgla_forward_profiled(msgla_handle* h, const void* X, int B, int L, void* O, void* workspace,
+                           size_t workspace_bytes, void* stream, void* const* events, int max_events,
+                           int* n_launches) {
+  if (!events || !n_launches) return fail(MSGLA_ERR_INVALID_ARG, "events or n_launches is NULL");
+  *n_launches = 0;
+  int st = check_forward_args(h, B, L);
+  if (st) return st;
+  if (B == 0 || L == 0) return MSGLA_OK;
+  if (!X || !O) return fail(MSGLA_ERR_INVALID_ARG, "X or O is NULL");
+  if (reinterpret_cast<uintptr_t>(X) % 16 || reinterpret_cast<uintptr_t>(O) % 16)
+    return fail(MSGLA_ERR_INVALID_ARG, "X and O must be 16-byte aligned");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
+  Recorder rec;
+  rec.events = events;
+  rec.max_events = max_events;
+  st = forward_impl(h, X, B, L, O, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), &rec);
+  *n_launches = rec.n;
+  return st;
 }
 
 int msgla_forward_host(msgla_handle* h, const void* X_host, int B, int L, void* O_host, void* workspace,

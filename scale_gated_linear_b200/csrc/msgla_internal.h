@@ -86,13 +86,13 @@ struct PoolParams {
   const __nv_bfloat16* Wfuse;  // [n_scales, d]
   const float* bfuse;          // [n_scales]
   float* w;                    // [B, L, n_scales]
-  int block_rows;              // rows per CTA (multiple of every scale > 1)
+  int block_rows;              // least common multiple of the scales > 1 (1 if none)
   int* err;
 };
 cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st);
 
 // gates: log alpha, chunk-local cumulative sums, scaled q/k and chunk decays
-struct GateParams {
+struct GateBranch {
   const __half* q;   // [B, n_s, h*dkp]
   const __half* k;
   const float* g;    // [B, n_s, rp]
@@ -101,7 +101,11 @@ struct GateParams {
   __half* qs;        // q * exp(b)
   __half* ks;        // k * exp(-b)
   float* gamma;      // [B, n_chunks, h*dkp] = exp(b at the chunk's last row)
-  int B, rows, heads, dkp, rp, n_chunks;
+  int rows, heads, n_chunks, block_begin;
+};
+struct GateParams {
+  GateBranch br[kMaxScales];
+  int n_branches, total_blocks, dkp, rp;
   float inv_normalizer;
   int* err;
 };

@@ -1,0 +1,276 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bar (bf16 inputs/outputs, fp32 accumulation): max|gpu - oracle| / max|oracle|
+<= 1e-2 and mean|gpu - oracle| / mean|oracle| <= 2e-3 on the layer output.
+Intermediate stages are checked against the oracle's own intermediates with a
+bar of 2e-3 (max) for the fp16 projections and 4e-3 for the GLA output.
+"""
+import numpy as np
+import pytest
+
+from helpers import MAX_REL, MEAN_REL, gpu_inputs, oracle_forward, rel_errors
+from scale_gated_linear_b200 import workloads as wl
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+needs_gpu = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+
+def _layer(w, inp, **kw):
+    from scale_gated_linear_b200 import MSGLA
+    return MSGLA.from_workload(w, inp, device=0, **kw)
+
+
+def run_gpu(w, inp, **kw):
+    layer = _layer(w, inp, **kw)
+    X = inp["X"].cuda()
+    B, L, _ = X.shape
+    ws = layer.alloc_workspace(B, L)
+    O = layer.forward(X, workspace=ws)
+    torch.cuda.synchronize()
+    layer.check_status()
+    return O.float().cpu().numpy(), layer, ws
+
+
+def assert_parity(got, ref, max_rel=MAX_REL, mean_rel=MEAN_REL):
+    mx, mn = rel_errors(got, ref)
+    assert np.isfinite(got).all()
+    assert mx <= max_rel and mn <= mean_rel, f"max_rel={mx:.3e} mean_rel={mn:.3e}"
+
+
+SMALL = wl.WORKLOADS["tiny"].replace(name="small", B=2, L=200, d=128, d_k=64, d_v=128, chunk=64)
+
+
+@needs_gpu
+def test_tiny_workload():
+    w = wl.WORKLOADS["tiny"]
+    inp = gpu_inputs(w)
+    got, layer, _ = run_gpu(w, inp)
+    assert_parity(got, oracle_forward(w, inp))
+    layer.close()
+
+
+@needs_gpu
+def test_intermediate_stages():
+    """Pooled rows, q/k/v, the low-rank gate, the GLA output and the fusion
+    weights each match the oracle's intermediates (several chunks, ragged tail)."""
+    from scale_gated_linear_b200 import WS_FUSION, WS_GATE, WS_O, WS_POOLED, WS_Q, WS_K, WS_V
+    w = wl.WORKLOADS["msgla_340m"].replace(name="mid")
+    B, L = 2, 300
+    inp = gpu_inputs(w, B=B, L=L)
+    got, layer, ws = run_gpu(w, inp)
+    ref, inter = oracle_forward(w, inp, intermediates=True)
+    assert_parity(got, ref)
+    f = wl.to_float64(inp)
+
+    def close(name, a, b, tol):
+        d = np.abs(a - b).max() / np.abs(b).max()
+        assert d <= tol, f"{name}: {d:.3e}"
+
+    close("w", layer.workspace_tensor(ws, B, L, 0, WS_FUSION).cpu().numpy(), inter["w"], 1e-5)
+    for j, (s, h) in enumerate(zip(w.scales, w.heads)):
+        bi = inter["branches"][j]
+        if s > 1:
+            close(f"pooled s={s}", layer.workspace_tensor(ws, B, L, j, WS_POOLED).float().cpu().numpy(), bi["Xp"],
+                  1e-3)
+        for name, which, width, ref_t, tol in (("q", WS_Q, w.d_k, bi["q"], 2e-3), ("k", WS_K, w.d_k, bi["k"], 2e-3),
+                                               ("v", WS_V, w.d_v, bi["v"], 2e-3), ("o", WS_O, w.d_v, bi["o"], 4e-3)):
+            t = layer.workspace_tensor(ws, B, L, j, which).float().cpu().numpy()
+            pad = t.shape[2] // h
+            t = np.concatenate([t[:, :, x * pad:x * pad + width] for x in range(h)], axis=2)
+            close(f"{name} s={s}", t, ref_t, tol)
+        g = layer.workspace_tensor(ws, B, L, j, WS_GATE).cpu().numpy()[:, :, :w.gate_rank]
+        close(f"g s={s}", g, bi["Xp"] @ f["branches"][j]["Wg1"].T, 2e-3)
+    layer.close()
+
+
+@needs_gpu
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 63, 64, 65, 127, 129, 200])
+def test_ragged_lengths(L):
+    """L below a pooling factor, at and around chunk (64) and GEMM tile (128) edges."""
+    inp = gpu_inputs(SMALL, L=L)
+    got, layer, _ = run_gpu(SMALL, inp)
+    assert_parity(got, oracle_forward(SMALL, inp))
+    layer.close()
+
+
+@needs_gpu
+def test_single_scale_plain_gla():
+    w = wl.WORKLOADS["gla_340m"].replace(name="gla_small", B=2, d=256)
+    inp = gpu_inputs(w, L=333)
+    got, layer, _ = run_gpu(w, inp)
+    assert_parity(got, oracle_forward(w, inp))
+    layer.close()
+
+
+@needs_gpu
+def test_no_fine_branch():
+    """{2,4} without the scale-1 branch takes the materialised hold + fusion path."""
+    w = wl.WORKLOADS["wide_8k_no_fine"].replace(name="nofine_small", d=256)
+    inp = gpu_inputs(w, B=2, L=150)
+    got, layer, _ = run_gpu(w, inp)
+    assert_parity(got, oracle_forward(w, inp))
+    layer.close()
+
+
+@needs_gpu
+def test_wide_scale_set_small():
+    w = wl.WORKLOADS["wide_8k"].replace(name="wide_small", d=256)
+    inp = gpu_inputs(w, B=2, L=260)
+    got, layer, _ = run_gpu(w, inp)
+    assert_parity(got, oracle_forward(w, inp))
+    layer.close()
+
+
+@needs_gpu
+@pytest.mark.parametrize("dk,dv", [(16, 16), (100, 200), (128, 384)])
+def test_padded_head_widths(dk, dv):
+    w = SMALL.replace(name=f"pad{dk}x{dv}", d_k=dk, d_v=dv)
+    inp = gpu_inputs(w, B=1, L=150)
+    got, layer, _ = run_gpu(w, inp)
+    assert_parity(got, oracle_forward(w, inp))
+    layer.close()
+
+
+@needs_gpu
+def test_qk_scale_and_long_memory_gates():
+    w = SMALL.replace(name="qk", gate_bias=3.0, gate_fan_in_init=True)
+    inp = gpu_inputs(w, B=1, L=300)
+    from scale_gated_linear_b200 import MSGLA
+    import oracle
+    layer = MSGLA.from_workload(w, inp, device=0, qk_scale=0.125)
+    O = layer(inp["X"].cuda())
+    torch.cuda.synchronize()
+    layer.check_status()
+    f = wl.to_float64(inp)
+    ref = oracle.layer_forward(f["X"], f, w.scales, w.heads, w.d_k, w.d_v, qk_scale=0.125)
+    assert_parity(O.float().cpu().numpy(), ref)
+    layer.close()
+
+
+@needs_gpu
+def test_empty_inputs_launch_nothing():
+    inp = gpu_inputs(SMALL, L=8)
+    layer = _layer(SMALL, inp)
+    assert layer.workspace_size(0, 100) == 0 and layer.workspace_size(3, 0) == 0
+    for B, L in ((0, 100), (3, 0)):
+        X = torch.zeros(B, L, SMALL.d, dtype=torch.bfloat16, device="cuda")
+        O = layer.forward(X, workspace=torch.empty(1, dtype=torch.uint8, device="cuda"))
+        assert O.shape == (B, L, SMALL.d)
+    assert layer.sync_status() == 0
+    layer.close()
+
+
+@needs_gpu
+def test_deterministic_and_batch_independent():
+    inp = gpu_inputs(SMALL, B=3, L=190)
+    layer = _layer(SMALL, inp)
+    X = inp["X"].cuda()
+    O1 = layer(X).clone()
+    O2 = layer(X).clone()
+    assert torch.equal(O1, O2)
+    for b in range(3):
+        Ob = layer(X[b:b + 1].contiguous())
+        assert torch.equal(Ob[0], O1[b])
+    layer.check_status()
+    layer.close()
+
+
+@needs_gpu
+def test_chunk_argument():
+    inp = gpu_inputs(SMALL, L=130)
+    a = _layer(SMALL, inp, chunk=0)
+    b = _layer(SMALL, inp, chunk=64)
+    X = inp["X"].cuda()
+    assert torch.equal(a(X), b(X))
+    a.close(), b.close()
+
+
+@needs_gpu
+def test_host_buffer_forward_matches_device_forward():
+    inp = gpu_inputs(SMALL, B=2, L=150)
+    layer = _layer(SMALL, inp)
+    Od = layer(inp["X"].cuda())
+    Xh = inp["X"].pin_memory()
+    Oh = torch.empty_like(Xh).pin_memory()
+    ws = layer.alloc_workspace(2, 150, host_staging=True)
+    layer.forward_host(Xh, Oh, ws)
+    assert torch.equal(Oh, Od.cpu())
+    layer.close()
+
+
+@needs_gpu
+def test_fp16_range_overflow_is_reported():
+    """Rows far outside the fp16 range make the pooled fp16 operand overflow: the
+    kernel latches MSGLA_ERR_RANGE (no fault) and the handle stays usable."""
+    from scale_gated_linear_b200 import MSGLAError
+    inp = gpu_inputs(SMALL, L=16)
+    layer = _layer(SMALL, inp)
+    X = (inp["X"].float() * 1e6).to(torch.bfloat16).cuda()
+    layer(X)
+    assert layer.sync_status() == -5
+    assert layer.sync_status() == 0  # cleared
+    O = layer(inp["X"].cuda())
+    layer.check_status()
+    assert torch.isfinite(O.float()).all()
+    layer.close()
+
+
+@needs_gpu
+def test_forward_profiled_records_every_launch():
+    inp = gpu_inputs(SMALL, L=100)
+    layer = _layer(SMALL, inp)
+    X = inp["X"].cuda()
+    ws = layer.alloc_workspace(*X.shape[:2])
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(layer.launch_names()) + 1)]
+    n = layer.forward_profiled(X, torch.empty_like(X), ws, ev)
+    torch.cuda.synchronize()
+    assert n == len(layer.launch_names())
+    assert all(ev[i].elapsed_time(ev[i + 1]) >= 0 for i in range(n))
+    layer.close()
+
+
+# ----------------------------------------------------------------- full sizes
+@needs_gpu
+def test_340m_layer_full_size_sampled_rows():
+    """The measured configuration (B=8, L=2048, d=1024) in the launch the bench
+    times; batch rows 0 and 7 are compared with the oracle in full."""
+    w = wl.WORKLOADS["msgla_340m"]
+    inp = gpu_inputs(w)
+    got, layer, _ = run_gpu(w, inp)
+    for b in (0, 7):
+        assert_parity(got[b:b + 1], oracle_forward(w, inp, batch=slice(b, b + 1)))
+    layer.close()
+
+
+@needs_gpu
+def test_gla_340m_full_size_sampled_row():
+    w = wl.WORKLOADS["gla_340m"]
+    inp = gpu_inputs(w)
+    got, layer, _ = run_gpu(w, inp)
+    assert_parity(got[3:4], oracle_forward(w, inp, batch=slice(3, 4)))
+    layer.close()
+
+
+@needs_gpu
+def test_long_32k_full_launch_prefix():
+    """L = 32768 in one launch; by causality its first 4096 outputs equal the
+    oracle run on the 4096-position prefix."""
+    w = wl.WORKLOADS["long_32k"]
+    inp = gpu_inputs(w)
+    got, layer, _ = run_gpu(w, inp)
+    assert_parity(got[:, :4096], oracle_forward(w, inp, rows=4096))
+    assert np.isfinite(got).all()
+    layer.close()
+
+
+@needs_gpu
+@pytest.mark.parametrize("name", ["wide_8k", "wide_8k_no_fine"])
+def test_wide_8k_full_launch_prefix(name):
+    w = wl.WORKLOADS[name]
+    inp = gpu_inputs(w)
+    got, layer, _ = run_gpu(w, inp)
+    assert_parity(got[0:1, :1024], oracle_forward(w, inp, rows=1024, batch=slice(0, 1)))
+    assert np.isfinite(got).all()
+    layer.close()
