@@ -113,6 +113,28 @@ int msgla_workspace_size(const msgla_handle* h, int B, int L, size_t* bytes);
 int msgla_forward(msgla_handle* h, const void* X, int B, int L, void* O,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* msgla_forward without a caller workspace and without any device allocation:
+ * for callers that cannot call cudaMalloc (or their framework's allocator) at the
+ * point where they run the layer -- for instance code inside a fixed memory arena
+ * or a runtime that forbids allocation after start-up. The pages describe no such
+ * entry point; it has no counterpart in the paper.
+ *   X, O, stream  as for msgla_forward (device bf16 [B, L, d], 16-byte aligned).
+ * The intermediates live in one fixed scratch array of 32 MiB inside the library's
+ * device image, which every GPU that loads the library holds until the process
+ * exits. Sizes whose workspace (msgla_workspace_size) exceeds 32 MiB are rejected
+ * with MSGLA_ERR_WORKSPACE; for the 340M-shaped layer (d = 1024, scales {1,2,4},
+ * d_k = 256, d_v = 512) that admits one sequence of up to about 2300 tokens.
+ * The first call on a device looks up the array's device address (a one-time
+ * set-up); make that first call before any stream capture. All calls share the
+ * array and it keeps the previous call's contents (every value a forward reads is
+ * written earlier in the same forward, so nothing needs clearing). Calls that can
+ * overlap on the GPU -- on different streams, or from different handles or
+ * threads -- race on the array and must be serialised by the caller.
+ * Asynchronous on `stream` like msgla_forward; device-side errors are reported by
+ * msgla_sync_status. */
+int msgla_forward_noalloc(msgla_handle* h, const void* X, int B, int L, void* O,
+                          void* stream);
+
 /* msgla_forward that also records CUDA events around its kernels, for timing each
  * kernel on `stream` with events. `events` holds caller-created cudaEvent_t
  * handles: events[0] is recorded before the first kernel and events[i+1] after

@@ -531,6 +531,36 @@ int check_forward_args(const msgla_handle* h, int B, int L) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- fixed scratch
+// Scratch of msgla_forward_noalloc: a file-scope device array. It is part of the
+// library's device image, so every GPU that loads the library holds these bytes
+// until the process exits. Host code must not pass `g_noalloc_scratch` itself to
+// a kernel (in host code the name is only a stand-in for the device symbol); the
+// device address comes from cudaGetSymbolAddress, once per device.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (set-up on first use).
+int noalloc_scratch(int device, void** out) {
+  if (device < 0 || device >= kMaxDevices) return fail(MSGLA_ERR_UNSUPPORTED, "device index %d", device);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[device]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(MSGLA_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+    g_noalloc_addr[device] = p;
+  }
+  *out = g_noalloc_addr[device];
+  return MSGLA_OK;
+}
+}  // namespace
+
 // ---------------------------------------------------------------- C ABI
 extern "C" {
 
@@ -620,6 +650,33 @@ int msgla_forward(msgla_handle* h, const void* X, int B, int L, void* O, void* w
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
   return forward_impl(h, X, B, L, O, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int msgla_forward_noalloc(msgla_handle* h, const void* X, int B, int L, void* O, void* stream) {
+  int st = check_forward_args(h, B, L);
+  if (st) return st;
+  if (B == 0 || L == 0) return MSGLA_OK;
+  if (!X || !O) return fail(MSGLA_ERR_INVALID_ARG, "X or O is NULL");
+  if (reinterpret_cast<uintptr_t>(X) % 16 || reinterpret_cast<uintptr_t>(O) % 16)
+    return fail(MSGLA_ERR_INVALID_ARG, "X and O must be 16-byte aligned");
+  const size_t nbytes = static_cast<size_t>(B) * L * h->cfg.d * 2;
+  const uint8_t* x0 = static_cast<const uint8_t*>(X);
+  const uint8_t* o0 = static_cast<const uint8_t*>(O);
+  if (x0 < o0 + nbytes && o0 < x0 + nbytes) return fail(MSGLA_ERR_INVALID_ARG, "O overlaps X");
+  const size_t need = layout(h, B, L).total;
+  if (need > kNoAllocScratchBytes)
+    return fail(MSGLA_ERR_WORKSPACE,
+                "B=%d, L=%d needs %zu bytes of scratch; the fixed scratch of msgla_forward_noalloc holds %zu "
+                "(use msgla_forward with a workspace)",
+                B, L, need, kNoAllocScratchBytes);
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
+  void* scratch = nullptr;
+  st = noalloc_scratch(h->device, &scratch);
+  if (st) return st;
+  // Every intermediate the kernels read is written earlier in the same forward, so
+  // the scratch needs no clearing between calls.
+  return forward_impl(h, X, B, L, O, scratch, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }
 
 int msgla_forward_profiled(msgla_handle* h, const void* X, int B, int L, void* O, void* workspace,
