@@ -75,7 +75,7 @@ def algorithmic_counts(w, B: int, L: int) -> dict:
     chunkwise GLA count 4 d_k d_v + C (d_k + d_v) per head and pooled step, the
     output projection at pooled length); bytes count each kernel's compulsory
     global-memory traffic."""
-    C = 64
+    C = 128
     r = w.gate_rank
     out = {}
     rows = {s: B * math.ceil(L / s) for s in w.scales}
@@ -94,7 +94,7 @@ def algorithmic_counts(w, B: int, L: int) -> dict:
     out["pool_fuse"] = {"bytes": B * L * w.d * 2 + sum(rows[s] * w.d * 2 for s in w.scales if s > 1)
                         + B * L * len(w.scales) * 4}
     out["gate"] = {"bytes": sum(rows[s] * (h * w.d_k * 2 * 2 * 2 + r * 4)
-                                + math.ceil(rows[s] / B / C) * B * h * w.d_k * 4
+                                + 2 * math.ceil(rows[s] / B / C) * B * h * w.d_k * 4
                                 for s, h in zip(w.scales, w.heads))}
     total_flops = sum(v.get("flops", 0) for v in out.values())
     weights = sum(h * (2 * w.d_k + w.d_v) * w.d * 2 + r * w.d * 2 + h * w.d_k * r * 4 + w.d * h * w.d_v * 2
@@ -362,7 +362,7 @@ def run_ours(args) -> int:
         "vs_baseline": None, "dtype": "f16/bf16 tensor-core operands, f32 accumulate; bf16 in/out",
         "data": "synthetic (seeded N(0,1) rows RMS-normalised, weights N(0,0.02))",
         "config": {"workload": f"{w.name}: B={w.B} per GPU, L={w.L}, d={w.d}, scales {list(w.scales)} heads "
-                               f"{list(w.heads)}, d_k={w.d_k}, d_v={w.d_v}, gate rank {w.gate_rank}, chunk 64",
+                               f"{list(w.heads)}, d_k={w.d_k}, d_v={w.d_v}, gate rank {w.gate_rank}, chunk 128",
                    "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"sequence-sharded x{world}",
                    "l2": "flushed between timed steps (256 MiB write)"},
         "roofline": roof,

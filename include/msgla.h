@@ -55,7 +55,7 @@ typedef struct msgla_config {
   int d_k;                       /* key width per head, 1..256                            */
   int d_v;                       /* value width per head, 1..1024                         */
   int gate_rank;                 /* rank r of the gate projection, 1..32                  */
-  int chunk;                     /* chunk length of the chunkwise GLA kernel: 0 or 64.
+  int chunk;                     /* chunk length of the chunkwise GLA kernel: 0 or 128.
                                     A compute parameter with no effect on the result
                                     beyond rounding (Sec. 3.4 of the notes).             */
   float gate_normalizer;         /* log alpha = logsigmoid(.) / gate_normalizer (> 0)     */

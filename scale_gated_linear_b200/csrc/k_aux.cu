@@ -5,8 +5,9 @@
 //                     unpooled rows (Sec. 3.3, Eq. (10)).
 //   gate_kernel       log alpha = logsigmoid(g W_g2^T + b_g) / normalizer (the
 //                     low-rank gate of Sec. 2.1), its cumulative sum b inside
-//                     each 64-row chunk, Qs = q e^{b}, Ks = k e^{-b} and the
-//                     chunk decay gamma = e^{b_last} used by the GLA kernel.
+//                     each 128-row GLA chunk referenced to the chunk's 64th
+//                     row (m): Qs = q e^{b - m}, Ks = k e^{m - b}, and per chunk
+//                     gamma = e^{b_last - m}, mid = e^{m}.
 //   hold_fuse_kernel  O_t = sum_s w_{t,s} Y^(s)_{floor((t+1)/s)-1} (Sec. 3.3,
 //                     Eq. (11)) when no branch has scale 1.
 //   weight converters used once by msgla_create.
@@ -231,11 +232,13 @@ __global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p)
 
 constexpr int kGateThreads = 512;
 
-// One CTA per (branch, batch, head, chunk); 512 threads = (dkp/2 channel pairs) x
-// (row groups of 64/groups rows). Every thread issues all of its q/k loads first,
-// computes log alpha for its rows, a local cumulative sum, then adds the totals of
-// the preceding row groups (through shared memory) to get b, and writes
-// Qs = q e^{b}, Ks = k e^{-b}; gamma = e^{b at the chunk's last row}.
+// One CTA per (branch, batch, head, 64-row half of a 128-row GLA chunk); 512
+// threads = (dkp/2 channel pairs) x (row groups of 64/groups rows). Every thread
+// issues all of its q/k loads first, computes log alpha for its rows and a local
+// cumulative sum, then adds the totals of the preceding row groups (through
+// shared memory). With b_loc the cumulative sum from the half's first row and T
+// its total: in the first half b - m = b_loc - T, in the second half b - m = b_loc
+// (m is the first half's total), so each half needs only its own rows.
 template <int RP, int R>
 __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constant__ GateParams p) {
   extern __shared__ float gsm[];
@@ -251,10 +254,12 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
     if (static_cast<int>(blockIdx.x) >= p.br[j].block_begin) bi = j;
   const GateBranch& P = p.br[bi];
   const int local = blockIdx.x - P.block_begin;
-  const int c = local % P.n_chunks;
-  const int head = (local / P.n_chunks) % P.heads;
-  const int b = local / (P.n_chunks * P.heads);
-  const int t0 = c * kChunk;
+  const int hc = local % P.n_halves;
+  const int head = (local / P.n_halves) % P.heads;
+  const int b = local / (P.n_halves * P.heads);
+  const int c = hc >> 1, second = hc & 1;
+  const int n_chunks = (P.n_halves + 1) >> 1;
+  const int t0 = hc * kChunk;
   const int nrows = min(kChunk, P.rows - t0);
   const int ldk = P.heads * dkp;
 
@@ -316,24 +321,37 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
     all0 += x0;
     all1 += x1;
   }
+  // reference: b - m = b_loc - T in the first half, b_loc in the second
+  const float ref0 = second ? 0.f : all0, ref1 = second ? 0.f : all1;
   bool bad = false;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     if (r0 + r < nrows) {
-      const float b0 = pre0 + c0[r], b1 = pre1 + c1[r];
+      const float b0 = pre0 + c0[r] - ref0, b1 = pre1 + c1[r] - ref1;
       const float2 qf = __half22float2(qv[r]);
       const float2 kf = __half22float2(kv[r]);
       const float ks0 = kf.x * __expf(-b0), ks1 = kf.y * __expf(-b1);
-      bad |= !(fabsf(ks0) <= 65504.f) || !(fabsf(ks1) <= 65504.f);
+      const float qs0 = qf.x * __expf(b0), qs1 = qf.y * __expf(b1);
+      bad |= !(fabsf(ks0) <= 65504.f) || !(fabsf(ks1) <= 65504.f) || !(fabsf(qs0) <= 65504.f) ||
+             !(fabsf(qs1) <= 65504.f);
       const size_t idx = (static_cast<size_t>(b) * P.rows + t0 + r0 + r) * ldk + ch;
-      *reinterpret_cast<__half2*>(P.qs + idx) = __floats2half2_rn(qf.x * __expf(b0), qf.y * __expf(b1));
+      *reinterpret_cast<__half2*>(P.qs + idx) = __floats2half2_rn(qs0, qs1);
       *reinterpret_cast<__half2*>(P.ks + idx) = __floats2half2_rn(ks0, ks1);
     }
   }
   if (grp == 0) {
-    float* gm = P.gamma + (static_cast<size_t>(b) * P.n_chunks + c) * ldk + ch;
-    gm[0] = __expf(all0);
-    gm[1] = __expf(all1);
+    const size_t gi = (static_cast<size_t>(b) * n_chunks + c) * ldk + ch;
+    if (second) {
+      P.gamma[gi] = __expf(all0);
+      P.gamma[gi + 1] = __expf(all1);
+    } else {
+      P.mid[gi] = __expf(all0);
+      P.mid[gi + 1] = __expf(all1);
+      if (hc + 1 >= P.n_halves) {  // chunk without a second half: b_last = m
+        P.gamma[gi] = 1.f;
+        P.gamma[gi + 1] = 1.f;
+      }
+    }
   }
   if (bad) atomicCAS(p.err, 0, kDevRange);
 }

@@ -4,25 +4,28 @@
 // reading notes, Sec. 2.1:  S_t = Diag(alpha_t) S_{t-1} + k_t^T v_t,
 // o_t = qk_scale * q_t S_t,  in its chunkwise form (Sec. 3.4: each branch is a
 // contiguous pooled sequence, so GLA's chunk algorithm applies unchanged).
-// With b_i the cumulative log forget gate inside a chunk (from its first row),
-// the gate kernel supplies Qs = q e^{b}, Ks = k e^{-b} and gamma = e^{b_last};
-// then for chunk c with state S (entering the chunk):
-//   A^T   = Ks Qs^T, masked to j <= i                 (intra-chunk scores)
-//   o^T   = S^T Qs^T + V^T A^T                        (inter + intra output)
-//   S    <- Diag(gamma) (S + Ks^T V)                  (state carried in TMEM)
-// Orientation: o is produced transposed (value column on the TMEM lane) so that
-// every MMA has M = 128; the 64-row score matrix uses an M = 128 MMA whose upper
-// 64 rows are ignored.
+//
+// Chunks hold C = 128 rows. With b_i the cumulative log forget gate from the
+// chunk's first row and m = b at its 64th row (the reference point), the gate
+// kernel supplies Qs = q e^{b - m}, Ks = k e^{m - b}, gamma = e^{b_last - m} and
+// mid = e^{m} per chunk and key channel. TMEM holds the scaled state
+// S' = Diag(e^{m_c}) S_{c-1} on entry to chunk c; per chunk:
+//   A     = Qs Ks^T, masked to j <= i            (scores, fp32 in TMEM)
+//   o     = Qs S' + A V                          (S' in shared memory as fp16,
+//                                                 A converted to fp16 in TMEM)
+//   S'   += Ks^T V
+//   S'   <- Diag(gamma_c mid_{c+1}) S'           (epilogue, in TMEM)
+// so every exponent stays within half a chunk's decay and every MMA is
+// M = 128, N = 128.
 //
 // One CTA = (batch, branch, head, 128-column value tile), looping over chunks:
-//   warp 0        TMA loads of Qs, Ks (64 x dkp, double-buffered: chunk c+1 is
-//                 fetched while chunk c computes) and V (64 x 128) per chunk
+//   warp 0        TMA loads of Qs, Ks (128 x dkp) and V (128 x 128)
 //   warp 1        TMEM allocation (512 columns) + tcgen05.mma issue
-//   warps 4..7    score epilogue (mask, fp16 into shared memory) and the o store
-//   warps 8..15   state epilogue: S <- gamma * S in TMEM, fp16 copy of S for the
-//                 next chunk's S^T Qs^T product (rows 0..127 / 128..255 of d_k)
-// TMEM columns: [0,256) state (two 128-lane halves of d_k), [256,320) o^T,
-// [320,384) A^T.
+//   warps 4..7    score epilogue (mask, fp16 back into TMEM) and the o store
+//   warps 8..15   state epilogue: S' <- factor * S' in TMEM and its fp16 copy
+//                 for the next chunk's Qs S' product (d_k rows 0..127 / 128..255)
+// TMEM columns: [0,256) S' (two 128-lane halves of d_k), [256,384) o,
+// [384,512) A (fp32; its fp16 form occupies [384,448)).
 #include "msgla_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -30,25 +33,33 @@ namespace msgla {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kAtom = 64 * 128;  // one 64-row x 128-byte swizzle block (8 KB)
-// shared memory map (bytes from the 1024-aligned base). The score MMA reads 128
-// rows of Ks, i.e. up to 8 KB past a stage's last atom: that lands in the next
-// buffer, never outside the allocation.
-constexpr int kStageQK = 8 * kAtom;           // Qs (4 atoms) + Ks (4 atoms), d_k <= 256
-constexpr int kOffQK = 0;                     // 2 stages
-constexpr int kOffV = kOffQK + 2 * kStageQK;  // V: 2 atoms (128 value columns)
-constexpr int kOffS = kOffV + 2 * kAtom;      // S^T fp16: 2 MN blocks x 256 rows x 128 B
-constexpr int kOffA = kOffS + 2 * 256 * 128;  // A^T fp16: 64 rows x 128 B
-constexpr int kOffBar = kOffA + kAtom;
+constexpr int kC = kGlaChunk;                 // 128 rows per chunk
+constexpr int kAtom = kC * 128;               // 128 rows x 128 bytes = 16 KB (64 16-bit columns)
+constexpr int kOffQ = 0;                      // Qs: up to 4 atoms (d_k <= 256)
+constexpr int kOffK = kOffQ + 4 * kAtom;      // Ks: up to 4 atoms
+constexpr int kOffV = kOffK + 4 * kAtom;      // V: 2 atoms (128 value columns)
+constexpr int kOffS = kOffV + 2 * kAtom;      // S' fp16: 2 MN blocks x 256 rows x 128 B
+constexpr int kOffBar = kOffS + 2 * 256 * 128;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-constexpr uint32_t kColS = 0, kColO = 256, kColA = 320;
+constexpr uint32_t kColS = 0, kColO = 256, kColA = 384;
 
 enum {
-  B_QK_FULL0 = 0, B_QK_FULL1, B_QK_EMPTY0, B_QK_EMPTY1, B_V_FULL, B_V_EMPTY,
-  B_A_FULL, B_A_SMEM, B_O_FULL, B_O_EMPTY, B_S_FULL, B_S_DONE, B_COUNT
+  B_Q_FULL = 0, B_Q_EMPTY, B_K_FULL, B_K_EMPTY, B_V_FULL, B_V_EMPTY,
+  B_A_FULL, B_A_READY, B_O_FULL, B_O_EMPTY, B_S_FULL, B_S_DONE, B_COUNT
 };
+
+// D[tmem] (+)= A[tmem] * B[smem]^T (A K-major in TMEM, 16-bit pairs per column)
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_constant__ GlaParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -72,17 +83,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
-    mbar_init(&bar[B_QK_FULL0], 1);
-    mbar_init(&bar[B_QK_FULL1], 1);
-    mbar_init(&bar[B_QK_EMPTY0], 1);
-    mbar_init(&bar[B_QK_EMPTY1], 1);
-    mbar_init(&bar[B_V_FULL], 1);
-    mbar_init(&bar[B_V_EMPTY], 1);
-    mbar_init(&bar[B_A_FULL], 1);
-    mbar_init(&bar[B_A_SMEM], 128);
-    mbar_init(&bar[B_O_FULL], 1);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], 1);
+    mbar_init(&bar[B_A_READY], 128);
     mbar_init(&bar[B_O_EMPTY], 128);
-    mbar_init(&bar[B_S_FULL], 1);
     mbar_init(&bar[B_S_DONE], 128 * n_half);
     *abort_flag = 0;
     fence_mbar_init();
@@ -99,147 +102,138 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer: Qs/Ks of chunk c into stage c&1, V of chunk c
+      // ---------------- TMA producer; each buffer is refilled once the MMAs of the
+      // previous chunk that read it have completed.
       prefetch_tmap(&T.tmQ);
       prefetch_tmap(&T.tmK);
       prefetch_tmap(&T.tmV);
-      const uint32_t qk_bytes = static_cast<uint32_t>(2 * (dkp / 64) * kAtom);
+      const uint32_t qk_bytes = static_cast<uint32_t>((dkp / 64) * kAtom);
       for (int c = 0; c < nch; ++c) {
-        const int st = c & 1;
-        if (c >= 2 && !mbar_wait(&bar[B_QK_EMPTY0 + st], ((c >> 1) - 1) & 1, abort_flag, p.err)) break;
-        uint8_t* sq = smem + kOffQK + st * kStageQK;
-        mbar_arrive_expect_tx(&bar[B_QK_FULL0 + st], qk_bytes);
-        for (int ka = 0; ka < dkp / 64; ++ka) {
-          tma_load_3d(&T.tmQ, &bar[B_QK_FULL0 + st], sq + ka * kAtom, head * dkp + ka * 64, c * kChunk, b);
-          tma_load_3d(&T.tmK, &bar[B_QK_FULL0 + st], sq + (4 + ka) * kAtom, head * dkp + ka * 64, c * kChunk, b);
-        }
-        if (c >= 1 && !mbar_wait(&bar[B_V_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
+        const int row = c * kC;
+        if (c > 0 && !mbar_wait(&bar[B_Q_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
+        mbar_arrive_expect_tx(&bar[B_Q_FULL], qk_bytes);
+        for (int ka = 0; ka < dkp / 64; ++ka)
+          tma_load_3d(&T.tmQ, &bar[B_Q_FULL], smem + kOffQ + ka * kAtom, head * dkp + ka * 64, row, b);
+        if (c > 0 && !mbar_wait(&bar[B_K_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
+        mbar_arrive_expect_tx(&bar[B_K_FULL], qk_bytes);
+        for (int ka = 0; ka < dkp / 64; ++ka)
+          tma_load_3d(&T.tmK, &bar[B_K_FULL], smem + kOffK + ka * kAtom, head * dkp + ka * 64, row, b);
+        if (c > 0 && !mbar_wait(&bar[B_V_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(&bar[B_V_FULL], 2 * kAtom);
         for (int mb = 0; mb < 2; ++mb)
-          tma_load_3d(&T.tmV, &bar[B_V_FULL], smem + kOffV + mb * kAtom, head * T.dvp + vt * kGlaTile + mb * 64,
-                      c * kChunk, b);
+          tma_load_3d(&T.tmV, &bar[B_V_FULL], smem + kOffV + mb * kAtom, head * T.dvp + vt * kGlaTile + mb * 64, row,
+                      b);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer. Per chunk: o^T(c), S update(c), scores(c+1).
-      const uint32_t id_at = idesc_f16(128, 64, 0, 0, 0);   // Ks (K-major) x Qs (K-major)
-      const uint32_t id_os = idesc_f16(128, 64, 0, 1, 0);   // S^T (MN-major) x Qs (K-major)
-      const uint32_t id_ov = idesc_f16(128, 64, 0, 1, 1);   // V^T (MN-major) x A^T rows (MN-major)
-      const uint32_t id_ds = idesc_f16(128, 128, 0, 1, 1);  // Ks^T (MN-major) x V (MN-major)
-      const uint32_t sV = sbase + kOffV, sS = sbase + kOffS, sA = sbase + kOffA;
+      // ---------------- MMA issuer. Per chunk: Qs S', scores, S' update, A V.
+      const uint32_t id_kk = idesc_f16(128, 128, 0, 0, 0);  // K-major x K-major
+      const uint32_t id_km = idesc_f16(128, 128, 0, 0, 1);  // K-major (smem or TMEM) x MN-major
+      const uint32_t id_mm = idesc_f16(128, 128, 0, 1, 1);  // MN-major x MN-major
+      const uint32_t sQ = sbase + kOffQ, sK = sbase + kOffK, sV = sbase + kOffV, sS = sbase + kOffS;
       const uint32_t lbo_s = static_cast<uint32_t>(dkp) * 128;
-      auto scores = [&](int c) {
-        // A^T[j][i] = sum_a Ks[j][a] Qs[i][a]
-        const uint32_t sQ = sbase + kOffQK + (c & 1) * kStageQK, sK = sQ + 4 * kAtom;
-        for (int ka = 0; ka < dkp / 64; ++ka)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_f16(tmem + kColA, sdesc_sw128(sK + ka * kAtom + kk * 32, 16, 1024),
-                     sdesc_sw128(sQ + ka * kAtom + kk * 32, 16, 1024), id_at, (ka | kk) != 0);
-        umma_commit(&bar[B_A_FULL]);
-      };
-      bool ok = mbar_wait(&bar[B_QK_FULL0], 0, abort_flag, p.err);
-      if (ok) {
-        tc_fence_after();
-        scores(0);
-      }
-      for (int c = 0; c < nch && ok; ++c) {
-        const int st = c & 1;
-        const uint32_t sQ = sbase + kOffQK + st * kStageQK, sK = sQ + 4 * kAtom;
-        if (!mbar_wait(&bar[B_A_SMEM], c & 1, abort_flag, p.err)) break;
-        if (!mbar_wait(&bar[B_V_FULL], c & 1, abort_flag, p.err)) break;
+      for (int c = 0; c < nch; ++c) {
+        const uint32_t ph = c & 1, pp = (c - 1) & 1;
+        if (!mbar_wait(&bar[B_Q_FULL], ph, abort_flag, p.err)) break;
         if (c > 0) {
-          if (!mbar_wait(&bar[B_S_DONE], (c - 1) & 1, abort_flag, p.err)) break;
-          if (!mbar_wait(&bar[B_O_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
-        }
-        tc_fence_after();
-        uint32_t acc = 0;
-        if (c > 0) {
-          // o^T += S^T Qs^T  (K = d_k)
-          for (int ks = 0; ks < dkp / 16; ++ks) {
-            umma_f16(tmem + kColO, sdesc_sw128(sS + ks * 2048, lbo_s, 1024),
-                     sdesc_sw128(sQ + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024), id_os, acc);
-            acc = 1;
-          }
-        }
-        // o^T += V^T A^T  (K = chunk rows j)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          umma_f16(tmem + kColO, sdesc_sw128(sV + ks * 2048, kAtom, 1024), sdesc_sw128(sA + ks * 2048, kAtom, 1024),
-                   id_ov, acc);
-          acc = 1;
-        }
-        umma_commit(&bar[B_O_FULL]);
-        // S += Ks^T V, per 128-row half of d_k
-        for (int h = 0; h < n_half; ++h)
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            umma_f16(tmem + kColS + h * 128, sdesc_sw128(sK + 2 * h * kAtom + ks * 2048, kAtom, 1024),
-                     sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_ds, (c > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(&bar[B_S_FULL]);
-        umma_commit(&bar[B_V_EMPTY]);
-        umma_commit(&bar[B_QK_EMPTY0 + st]);
-        if (c + 1 < nch) {
-          if (!mbar_wait(&bar[B_QK_FULL0 + ((c + 1) & 1)], ((c + 1) >> 1) & 1, abort_flag, p.err)) break;
+          if (!mbar_wait(&bar[B_S_DONE], pp, abort_flag, p.err)) break;
+          if (!mbar_wait(&bar[B_O_EMPTY], pp, abort_flag, p.err)) break;
           tc_fence_after();
-          scores(c + 1);
+          // o = Qs S'  (K = d_k)
+          for (int ks = 0; ks < dkp / 16; ++ks)
+            umma_f16(tmem + kColO, sdesc_sw128(sQ + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024),
+                     sdesc_sw128(sS + ks * 2048, lbo_s, 1024), id_km, ks > 0);
         }
+        if (!mbar_wait(&bar[B_K_FULL], ph, abort_flag, p.err)) break;
+        tc_fence_after();
+        // A = Qs Ks^T  (K = d_k)
+        for (int ks = 0; ks < dkp / 16; ++ks)
+          umma_f16(tmem + kColA, sdesc_sw128(sQ + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024),
+                   sdesc_sw128(sK + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024), id_kk, ks > 0);
+        umma_commit(&bar[B_A_FULL]);
+        umma_commit(&bar[B_Q_EMPTY]);
+        if (!mbar_wait(&bar[B_V_FULL], ph, abort_flag, p.err)) break;
+        tc_fence_after();
+        // S' += Ks^T V per 128-row half of d_k  (K = chunk rows j)
+        for (int h = 0; h < n_half; ++h)
+          for (int ks = 0; ks < kC / 16; ++ks)
+            umma_f16(tmem + kColS + h * 128, sdesc_sw128(sK + 2 * h * kAtom + ks * 2048, kAtom, 1024),
+                     sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_mm, (c > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(&bar[B_S_FULL]);
+        umma_commit(&bar[B_K_EMPTY]);
+        if (!mbar_wait(&bar[B_A_READY], ph, abort_flag, p.err)) break;
+        tc_fence_after();
+        // o += A V  (A fp16 in TMEM, 8 columns per 16 rows j)
+        for (int ks = 0; ks < kC / 16; ++ks)
+          umma_f16_ts(tmem + kColO, tmem + kColA + ks * 8, sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_km,
+                      (c > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(&bar[B_O_FULL]);
+        umma_commit(&bar[B_V_EMPTY]);
       }
     }
   } else if (warp >= 4 && warp < 8) {
-    // ---------------- scores (mask + fp16 into smem) and output store
+    // ---------------- scores -> fp16 in TMEM, then the output rows
     const int quad = warp & 3;
-    const int j = quad * 32 + lane;  // TMEM lane: chunk row j for A^T, value column for o^T
-    uint8_t* sA = smem + kOffA;
+    const int i = quad * 32 + lane;  // chunk row (TMEM lane)
     const size_t ld_o = static_cast<size_t>(T.heads) * T.dvp;
     for (int c = 0; c < nch; ++c) {
       if (!mbar_wait(&bar[B_A_FULL], c & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tmem_addr(tmem, quad * 32, kColA), r0);
-      tmem_ld32(tmem_addr(tmem, quad * 32, kColA + 32), r1);
-      tmem_wait_ld();
-      if (j < kChunk) {
-        // A^T[j][i] kept for i >= j (causal within the chunk)
+#pragma unroll 1
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t ra[32], rb[32], pk[32];
+        const uint32_t src = tmem_addr(tmem, quad * 32, kColA + h2 * 64);
+        tmem_ld32(src, ra);
+        tmem_ld32(src + 32, rb);
+        tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          float f[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int i = cc * 8 + e;
-            const float x = __uint_as_float(i < 32 ? r0[i & 31] : r1[i & 31]);
-            f[e] = (i >= j) ? x : 0.f;
-          }
-          st_shared_v4(smem_u32(sA + j * 128 + ((cc ^ (j & 7)) << 4)), pack_half2(f[0], f[1]),
-                       pack_half2(f[2], f[3]), pack_half2(f[4], f[5]), pack_half2(f[6], f[7]));
+        for (int e = 0; e < 16; ++e) {
+          const int j0 = h2 * 64 + 2 * e;
+          pk[e] = pack_half2(j0 <= i ? __uint_as_float(ra[2 * e]) : 0.f,
+                             j0 + 1 <= i ? __uint_as_float(ra[2 * e + 1]) : 0.f);
+          const int j1 = j0 + 32;
+          pk[16 + e] = pack_half2(j1 <= i ? __uint_as_float(rb[2 * e]) : 0.f,
+                                  j1 + 1 <= i ? __uint_as_float(rb[2 * e + 1]) : 0.f);
         }
+        tmem_st32(tmem_addr(tmem, quad * 32, kColA + h2 * 32), pk);
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar[B_A_SMEM]);
+      mbar_arrive(&bar[B_A_READY]);
 
       if (!mbar_wait(&bar[B_O_FULL], c & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      tmem_ld32(tmem_addr(tmem, quad * 32, kColO), r0);
-      tmem_ld32(tmem_addr(tmem, quad * 32, kColO + 32), r1);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bar[B_O_EMPTY]);
-      const int col = head * T.dvp + vt * kGlaTile + j;
-      const int t0 = c * kChunk;
-      __half* dst = T.o + (static_cast<size_t>(b) * T.rows + t0) * ld_o + col;
-      const int nvalid = min(kChunk, T.rows - t0);
+      const int t = c * kC + i;
+      __half* dst = T.o + (static_cast<size_t>(b) * T.rows + t) * ld_o + head * T.dvp + vt * kGlaTile;
+#pragma unroll 1
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t ra[32], rb[32];
+        const uint32_t src = tmem_addr(tmem, quad * 32, kColO + h2 * 64);
+        tmem_ld32(src, ra);
+        tmem_ld32(src + 32, rb);
+        tmem_wait_ld();
+        if (h2 == 1) {
+          tc_fence_before();
+          mbar_arrive(&bar[B_O_EMPTY]);
+        }
+        if (t < T.rows) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + h2 * 64);
 #pragma unroll
-      for (int i = 0; i < kChunk; ++i) {
-        if (i < nvalid) {
-          const float x = __uint_as_float(i < 32 ? r0[i & 31] : r1[i & 31]);
-          dst[static_cast<size_t>(i) * ld_o] = __float2half_rn(p.qk_scale * x);
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t* r = q < 4 ? ra + 8 * q : rb + 8 * (q - 4);
+            uint4 u;
+            u.x = pack_half2(p.qk_scale * __uint_as_float(r[0]), p.qk_scale * __uint_as_float(r[1]));
+            u.y = pack_half2(p.qk_scale * __uint_as_float(r[2]), p.qk_scale * __uint_as_float(r[3]));
+            u.z = pack_half2(p.qk_scale * __uint_as_float(r[4]), p.qk_scale * __uint_as_float(r[5]));
+            u.w = pack_half2(p.qk_scale * __uint_as_float(r[6]), p.qk_scale * __uint_as_float(r[7]));
+            d4[q] = u;
+          }
         }
       }
     }
   } else if (warp >= 8) {
-    // ---------------- state epilogue: S <- gamma * S, fp16 copy for the next chunk
+    // ---------------- state epilogue: S' <- gamma_c mid_{c+1} S', fp16 copy in smem
     const int g = (warp - 8) >> 2;  // d_k half
     const int quad = warp & 3;
     if (g < n_half) {
@@ -247,9 +241,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
       uint8_t* sS = smem + kOffS;
       const size_t ld_g = static_cast<size_t>(T.heads) * dkp;
       const float* gp = T.gamma + static_cast<size_t>(b) * nch * ld_g + head * dkp + a;
-      float gam = __ldg(gp);
+      const float* mp = T.mid + static_cast<size_t>(b) * nch * ld_g + head * dkp + a;
+      float f = __ldg(gp) * (nch > 1 ? __ldg(mp + ld_g) : 1.f);
       for (int c = 0; c < nch; ++c) {
-        const float gam_next = (c + 1 < nch) ? __ldg(gp + (c + 1) * ld_g) : 0.f;
+        const float f_next =
+            (c + 1 < nch) ? __ldg(gp + (c + 1) * ld_g) * ((c + 2 < nch) ? __ldg(mp + (c + 2) * ld_g) : 1.f) : 0.f;
         if (!mbar_wait(&bar[B_S_FULL], c & 1, abort_flag, p.err)) break;
         tc_fence_after();
 #pragma unroll 1
@@ -261,8 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            ra[e] = __float_as_uint(gam * __uint_as_float(ra[e]));
-            rb[e] = __float_as_uint(gam * __uint_as_float(rb[e]));
+            ra[e] = __float_as_uint(f * __uint_as_float(ra[e]));
+            rb[e] = __float_as_uint(f * __uint_as_float(rb[e]));
           }
           tmem_st32(ta, ra);
           tmem_st32(ta + 32, rb);
@@ -282,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bar[B_S_DONE]);
-        gam = gam_next;
+        f = f_next;
       }
     }
   }

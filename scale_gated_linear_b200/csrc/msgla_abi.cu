@@ -131,8 +131,8 @@ struct Region {
   size_t off = 0, bytes = 0;
 };
 struct BranchWs {
-  int rows, n_chunks;
-  Region Xp, q, k, qs, ks, v, g, gamma, o, Y;
+  int rows, n_chunks, n_halves;
+  Region Xp, q, k, qs, ks, v, g, gamma, mid, o, Y;
 };
 struct Workspace {
   BranchWs br[MSGLA_MAX_SCALES];
@@ -155,7 +155,8 @@ Workspace layout(const msgla_handle* h, int B, int L) {
     const Branch& b = h->br[j];
     BranchWs& w = ws.br[j];
     w.rows = ceil_div(L, b.scale);
-    w.n_chunks = ceil_div(w.rows, kChunk);
+    w.n_chunks = ceil_div(w.rows, kGlaChunk);
+    w.n_halves = ceil_div(w.rows, kChunk);
     const size_t n = BB * w.rows;
     if (b.scale > 1) add(w.Xp, cur, n * d * 2);
     add(w.q, cur, n * b.heads * h->dkp * 2);
@@ -165,6 +166,7 @@ Workspace layout(const msgla_handle* h, int B, int L) {
     add(w.v, cur, n * b.heads * h->dvp * 2);
     add(w.g, cur, n * h->rp * 4);
     add(w.gamma, cur, BB * w.n_chunks * b.heads * h->dkp * 4);
+    add(w.mid, cur, BB * w.n_chunks * b.heads * h->dkp * 4);
     add(w.o, cur, n * b.heads * h->dvp * 2);
     if (j != h->main_index) add(w.Y, cur, n * d * 2);
   }
@@ -193,8 +195,8 @@ int validate(const msgla_config* c) {
   if (c->d_v < 1 || c->d_v > 1024) return fail(MSGLA_ERR_UNSUPPORTED, "d_v=%d outside [1, 1024]", c->d_v);
   if (c->gate_rank < 1 || c->gate_rank > 32)
     return fail(MSGLA_ERR_UNSUPPORTED, "gate_rank=%d outside [1, 32]", c->gate_rank);
-  if (c->chunk != 0 && c->chunk != kChunk)
-    return fail(MSGLA_ERR_UNSUPPORTED, "chunk=%d: the GLA kernel runs 64-row chunks (pass 0 or 64)", c->chunk);
+  if (c->chunk != 0 && c->chunk != kGlaChunk)
+    return fail(MSGLA_ERR_UNSUPPORTED, "chunk=%d: the GLA kernel runs 128-row chunks (pass 0 or 128)", c->chunk);
   if (!(c->gate_normalizer > 0.f) || !std::isfinite(c->gate_normalizer))
     return fail(MSGLA_ERR_INVALID_ARG, "gate_normalizer must be finite and > 0");
   if (!std::isfinite(c->qk_scale)) return fail(MSGLA_ERR_INVALID_ARG, "qk_scale must be finite");
@@ -385,11 +387,12 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
       q.qs = static_cast<__half*>(at(bw.qs));
       q.ks = static_cast<__half*>(at(bw.ks));
       q.gamma = static_cast<float*>(at(bw.gamma));
+      q.mid = static_cast<float*>(at(bw.mid));
       q.rows = bw.rows;
       q.heads = b.heads;
-      q.n_chunks = bw.n_chunks;
+      q.n_halves = bw.n_halves;
       q.block_begin = blocks;
-      blocks += B * b.heads * bw.n_chunks;
+      blocks += B * b.heads * bw.n_halves;
     }
     g.n_branches = ns;
     g.total_blocks = blocks;
@@ -411,11 +414,12 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     const Branch& b = h->br[j];
     const BranchWs& bw = ws.br[j];
     GlaTask& t = lp.task[j];
-    if (!encode_3d(&t.tmQ, false, at(bw.qs), b.heads * h->dkp, bw.rows, B, kChunk) ||
-        !encode_3d(&t.tmK, false, at(bw.ks), b.heads * h->dkp, bw.rows, B, kChunk) ||
-        !encode_3d(&t.tmV, false, at(bw.v), b.heads * h->dvp, bw.rows, B, kChunk))
+    if (!encode_3d(&t.tmQ, false, at(bw.qs), b.heads * h->dkp, bw.rows, B, kGlaChunk) ||
+        !encode_3d(&t.tmK, false, at(bw.ks), b.heads * h->dkp, bw.rows, B, kGlaChunk) ||
+        !encode_3d(&t.tmV, false, at(bw.v), b.heads * h->dvp, bw.rows, B, kGlaChunk))
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (gla, scale %d)", b.scale);
     t.gamma = static_cast<const float*>(at(bw.gamma));
+    t.mid = static_cast<const float*>(at(bw.mid));
     t.o = static_cast<__half*>(at(bw.o));
     t.rows = bw.rows;
     t.n_chunks = bw.n_chunks;

@@ -13,7 +13,8 @@ namespace msgla {
 // Fixed tile constants.
 constexpr int kGemmBM = 128;     // GEMM rows per tile (tcgen05 M)
 constexpr int kGemmBK = 64;      // GEMM K per stage (one 128-byte swizzle atom of 16-bit data)
-constexpr int kChunk = 64;       // chunk length of the chunkwise GLA kernel
+constexpr int kChunk = 64;       // rows per gate block (half of a GLA chunk)
+constexpr int kGlaChunk = 128;   // chunk length of the chunkwise GLA kernel
 constexpr int kGlaTile = 128;    // value columns per GLA CTA (tcgen05 M of the output MMA)
 constexpr int kMaxTasks = 8;     // GEMM tasks per grouped launch
 constexpr int kMaxScales = 8;
@@ -59,7 +60,8 @@ struct alignas(64) GlaTask {
   CUtensorMap tmQ;  // 3D {h*dkp, n_s, B}, box {64, 64, 1}
   CUtensorMap tmK;  // same shape as tmQ
   CUtensorMap tmV;  // 3D {h*dvp, n_s, B}, box {64, 64, 1}
-  const float* gamma;  // [B, n_chunks, h*dkp]
+  const float* gamma;  // [B, n_chunks, h*dkp]: e^{b_last - m} per chunk
+  const float* mid;    // [B, n_chunks, h*dkp]: e^{m}, m = b at the chunk's 64th row
   __half* o;           // [B, n_s, h*dvp]
   int rows, n_chunks, heads, dkp, dvp, v_tiles, cta_begin, pad_;
 };
@@ -98,10 +100,11 @@ struct GateBranch {
   const float* g;    // [B, n_s, rp]
   const float* Wg2;  // [h*dkp, rp]
   const float* bg;   // [h*dkp]
-  __half* qs;        // q * exp(b)
-  __half* ks;        // k * exp(-b)
-  float* gamma;      // [B, n_chunks, h*dkp] = exp(b at the chunk's last row)
-  int rows, heads, n_chunks, block_begin;
+  __half* qs;        // q * exp(b - m)
+  __half* ks;        // k * exp(m - b)
+  float* gamma;      // [B, n_chunks, h*dkp] = exp(b_last - m)
+  float* mid;        // [B, n_chunks, h*dkp] = exp(m)
+  int rows, heads, n_halves, block_begin;
 };
 struct GateParams {
   GateBranch br[kMaxScales];

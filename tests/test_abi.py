@@ -58,7 +58,7 @@ def _cfg(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(d=100), -2), (dict(d=0), -2), (dict(n_scales=0), -1), (dict(n_scales=9), -1),
     (dict(scales=(1, 4, 2)), -1), (dict(scales=(0, 2, 4)), -1), (dict(heads=(2, 0, 1)), -1),
-    (dict(d_k=300), -2), (dict(d_v=0), -2), (dict(gate_rank=33), -2), (dict(chunk=16), -2),
+    (dict(d_k=300), -2), (dict(d_v=0), -2), (dict(gate_rank=33), -2), (dict(chunk=16), -2), (dict(chunk=64), -2),
     (dict(gate_normalizer=0.0), -1), (dict(gate_normalizer=float("nan")), -1),
     (dict(qk_scale=float("inf")), -1), (dict(scales=(1, 7, 11)), -2),
 ])

@@ -86,9 +86,10 @@ def test_intermediate_stages():
 
 
 @needs_gpu
-@pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 63, 64, 65, 127, 129, 200])
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 63, 64, 65, 127, 128, 129, 200, 255, 257, 520])
 def test_ragged_lengths(L):
-    """L below a pooling factor, at and around chunk (64) and GEMM tile (128) edges."""
+    """L below a pooling factor, at and around the gate block (64), GLA chunk and
+    GEMM tile (128) edges, for every branch's pooled length."""
     inp = gpu_inputs(SMALL, L=L)
     got, layer, _ = run_gpu(SMALL, inp)
     assert_parity(got, oracle_forward(SMALL, inp))
@@ -181,7 +182,7 @@ def test_deterministic_and_batch_independent():
 def test_chunk_argument():
     inp = gpu_inputs(SMALL, L=130)
     a = _layer(SMALL, inp, chunk=0)
-    b = _layer(SMALL, inp, chunk=64)
+    b = _layer(SMALL, inp, chunk=128)
     X = inp["X"].cuda()
     assert torch.equal(a(X), b(X))
     a.close(), b.close()
