@@ -139,7 +139,7 @@ int msgla_forward_noalloc(msgla_handle* h, const void* X, int B, int L, void* O,
  * kernel on `stream` with events. `events` holds caller-created cudaEvent_t
  * handles: events[0] is recorded before the first kernel and events[i+1] after
  * the i-th kernel. The kernels of one forward, in launch order, are:
- *   pool_fuse, proj_gemm, gate (all scales), gla,
+ *   pool_fuse (absent for a single scale-1 branch), proj_gemm, gate (all scales), gla,
  *   out_gemm_coarse (only when a scale-1 branch and a coarser branch exist),
  *   out_gemm_fused (scale-1 branch present) or, without a scale-1 branch,
  *   out_gemm_coarse for all branches followed by hold_fuse.

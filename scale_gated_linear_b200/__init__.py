@@ -109,7 +109,8 @@ class MSGLA:
 
     def launch_names(self):
         """Kernel names of one forward, in launch order (see msgla_forward_profiled)."""
-        names = ["pool_fuse", "proj_gemm", "gate", "gla"]
+        pool = any(s > 1 for s in self.scales) or 1 not in self.scales
+        names = (["pool_fuse"] if pool else []) + ["proj_gemm", "gate", "gla"]
         if 1 in self.scales:
             if len(self.scales) > 1:
                 names.append("out_gemm_coarse")

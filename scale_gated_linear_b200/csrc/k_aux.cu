@@ -130,11 +130,12 @@ __global__ void __launch_bounds__(kPoolThreads) pool_fuse_kernel(const PoolParam
 }
 
 // Streaming form for scale sets whose coarse scales all divide P (P <= 8): one
-// warp per block of P rows of one sequence. Each lane loads P x 16 bytes per
-// column group before using any of them (memory-level parallelism), forms the
-// pooled rows of every coarse scale and the partial fusion logits; the logits
-// are reduced across the warp once per row at the end.
-template <int P>
+// warp per block of P rows of one sequence. Per pass each lane first issues the
+// loads of GPL column groups (8 columns each) for all P rows (GPL * P * 16 bytes
+// in flight per lane), then forms the pooled rows of every coarse scale and the
+// partial fusion logits; the logits are reduced across the warp once per row at
+// the end. NS bounds the number of scales held in registers.
+template <int P, int GPL, int NS>
 __global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p) {
   extern __shared__ float wf_s[];  // [n_scales][d] fp32
   const int ns = p.n_scales;
@@ -148,69 +149,76 @@ __global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p)
   const int row0 = static_cast<int>(gw % blocks_per_seq) * P;
   const int nrows = min(P, p.L - row0);
   const __nv_bfloat16* Xb = p.X + (static_cast<size_t>(b) * p.L + row0) * p.d;
-  float part[P][kMaxScales];
+  float part[P][NS];
 #pragma unroll
   for (int r = 0; r < P; ++r)
 #pragma unroll
-    for (int j = 0; j < kMaxScales; ++j) part[r][j] = 0.f;
+    for (int j = 0; j < NS; ++j) part[r][j] = 0.f;
   const int groups = p.d / 8;
-  for (int cg = lane; cg < groups; cg += 32) {
-    float x[P][8];
+  for (int base = 0; base < groups; base += 32 * GPL) {
+    uint4 raw[GPL][P];
 #pragma unroll
-    for (int r = 0; r < P; ++r) {
-      if (r < nrows) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(Xb + static_cast<size_t>(r) * p.d) + cg);
-        bf16x8_to_f32(u, x[r]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[r][e] = 0.f;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kMaxScales; ++j) {
-      if (j >= ns) break;
-      const float4 wa = *reinterpret_cast<const float4*>(wf_s + j * p.d + cg * 8);
-      const float4 wb = *reinterpret_cast<const float4*>(wf_s + j * p.d + cg * 8 + 4);
+    for (int gi = 0; gi < GPL; ++gi) {
+      const int cg = base + gi * 32 + lane;
 #pragma unroll
       for (int r = 0; r < P; ++r)
-        part[r][j] += x[r][0] * wa.x + x[r][1] * wa.y + x[r][2] * wa.z + x[r][3] * wa.w + x[r][4] * wb.x +
-                      x[r][5] * wb.y + x[r][6] * wb.z + x[r][7] * wb.w;
-      const int s = p.scales[j];
-      if (s == 1) continue;
-      const int n_s = (p.L + s - 1) / s;
-      for (int i0 = 0; i0 < P; i0 += s) {
-        if (i0 >= nrows) break;
-        const int cnt = min(s, nrows - i0);
-        float m[8];
+        raw[gi][r] = (cg < groups && r < nrows)
+                         ? __ldg(reinterpret_cast<const uint4*>(Xb + static_cast<size_t>(r) * p.d) + cg)
+                         : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m[e] = 0.f;
+    for (int gi = 0; gi < GPL; ++gi) {
+      const int cg = base + gi * 32 + lane;
+      if (cg >= groups) continue;
+      float x[P][8];
+#pragma unroll
+      for (int r = 0; r < P; ++r) bf16x8_to_f32(raw[gi][r], x[r]);
+#pragma unroll
+      for (int j = 0; j < NS; ++j) {
+        if (j >= ns) break;
+        const float4 wa = *reinterpret_cast<const float4*>(wf_s + j * p.d + cg * 8);
+        const float4 wb = *reinterpret_cast<const float4*>(wf_s + j * p.d + cg * 8 + 4);
 #pragma unroll
         for (int r = 0; r < P; ++r)
-          if (r >= i0 && r < i0 + cnt)
+          part[r][j] += x[r][0] * wa.x + x[r][1] * wa.y + x[r][2] * wa.z + x[r][3] * wa.w + x[r][4] * wb.x +
+                        x[r][5] * wb.y + x[r][6] * wb.z + x[r][7] * wb.w;
+        const int s = p.scales[j];
+        if (s == 1) continue;
+        const int n_s = (p.L + s - 1) / s;
+        for (int i0 = 0; i0 < P; i0 += s) {
+          if (i0 >= nrows) break;
+          const int cnt = min(s, nrows - i0);
+          float m[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) m[e] += x[r][e];
-        const float inv = 1.f / static_cast<float>(cnt);
-        uint4 o;
-        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-        bool bad = false;
+          for (int e = 0; e < 8; ++e) m[e] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a0 = m[2 * e] * inv, a1 = m[2 * e + 1] * inv;
-          bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
-          ow[e] = pack_half2(a0, a1);
+          for (int r = 0; r < P; ++r)
+            if (r >= i0 && r < i0 + cnt)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) m[e] += x[r][e];
+          const float inv = 1.f / static_cast<float>(cnt);
+          uint4 o;
+          uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+          bool bad = false;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float a0 = m[2 * e] * inv, a1 = m[2 * e + 1] * inv;
+            bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
+            ow[e] = pack_half2(a0, a1);
+          }
+          if (bad) atomicCAS(p.err, 0, kDevRange);
+          const int i = (row0 + i0) / s;
+          reinterpret_cast<uint4*>(p.Xp[j] + (static_cast<size_t>(b) * n_s + i) * p.d)[cg] = o;
         }
-        if (bad) atomicCAS(p.err, 0, kDevRange);
-        const int i = (row0 + i0) / s;
-        reinterpret_cast<uint4*>(p.Xp[j] + (static_cast<size_t>(b) * n_s + i) * p.d)[cg] = o;
       }
     }
   }
 #pragma unroll
   for (int r = 0; r < P; ++r) {
-    float z[kMaxScales];
+    float z[NS];
     float zmax = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < kMaxScales; ++j) {
+    for (int j = 0; j < NS; ++j) {
       float v = part[r][j];
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -220,7 +228,7 @@ __global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p)
     if (lane == 0 && r < nrows) {
       float sum = 0.f;
 #pragma unroll
-      for (int j = 0; j < kMaxScales; ++j) {
+      for (int j = 0; j < NS; ++j) {
         z[j] = j < ns ? __expf(z[j] - zmax) : 0.f;
         sum += z[j];
       }
@@ -230,30 +238,86 @@ __global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p)
   }
 }
 
-constexpr int kGateThreads = 512;
+// Pooling only (the fusion logits come from the projection GEMM): one thread per
+// (sequence, block of P rows, 8 columns); all P row loads are issued together.
+template <int P>
+__global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
+  const int groups = p.d / 8;
+  const int nblk = (p.L + P - 1) / P;
+  const size_t gid = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (gid >= static_cast<size_t>(p.B) * nblk * groups) return;
+  const int cg = static_cast<int>(gid % groups);
+  const size_t rest = gid / groups;
+  const int blk = static_cast<int>(rest % nblk), b = static_cast<int>(rest / nblk);
+  const int row0 = blk * P;
+  const int nrows = min(P, p.L - row0);
+  const __nv_bfloat16* Xb = p.X + (static_cast<size_t>(b) * p.L + row0) * p.d;
+  uint4 raw[P];
+#pragma unroll
+  for (int r = 0; r < P; ++r)
+    raw[r] = r < nrows ? __ldg(reinterpret_cast<const uint4*>(Xb + static_cast<size_t>(r) * p.d) + cg)
+                       : make_uint4(0, 0, 0, 0);
+  float x[P][8];
+#pragma unroll
+  for (int r = 0; r < P; ++r) bf16x8_to_f32(raw[r], x[r]);
+  bool bad = false;
+  for (int j = 0; j < p.n_scales; ++j) {
+    const int s = p.scales[j];
+    if (s == 1) continue;
+    const int n_s = (p.L + s - 1) / s;
+    for (int i0 = 0; i0 < nrows; i0 += s) {
+      const int cnt = min(s, nrows - i0);
+      float m[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m[e] = 0.f;
+#pragma unroll
+      for (int r = 0; r < P; ++r)
+        if (r >= i0 && r < i0 + cnt)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m[e] += x[r][e];
+      const float inv = 1.f / static_cast<float>(cnt);
+      uint4 o;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a0 = m[2 * e] * inv, a1 = m[2 * e + 1] * inv;
+        bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
+        ow[e] = pack_half2(a0, a1);
+      }
+      reinterpret_cast<uint4*>(p.Xp[j] + (static_cast<size_t>(b) * n_s + (row0 + i0) / s) * p.d)[cg] = o;
+    }
+  }
+  if (bad) atomicCAS(p.err, 0, kDevRange);
+}
 
-// One CTA per (branch, batch, head, 64-row half of a 128-row GLA chunk); 512
-// threads = (dkp/2 channel pairs) x (row groups of 64/groups rows). Every thread
-// issues all of its q/k loads first, computes log alpha for its rows and a local
-// cumulative sum, then adds the totals of the preceding row groups (through
+constexpr int kGateThreads = 256;
+constexpr int kGateChannels = 128;  // key channels per CTA (64 pairs x 4 row groups of 16)
+
+// One CTA per (branch, batch, head, 64-row half of a 128-row GLA chunk, 128 key
+// channels); 256 threads = 64 channel pairs x 4 row groups of R = 16 rows. Every
+// thread issues all of its q/k loads first, computes log alpha for its rows and a
+// local cumulative sum, then adds the totals of the preceding row groups (through
 // shared memory). With b_loc the cumulative sum from the half's first row and T
 // its total: in the first half b - m = b_loc - T, in the second half b - m = b_loc
 // (m is the first half's total), so each half needs only its own rows.
 template <int RP, int R>
 __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constant__ GateParams p) {
-  extern __shared__ float gsm[];
+  __shared__ float g_s[kChunk * RP];                        // [64][RP]
+  __shared__ __align__(16) float w_s[RP * kGateChannels];   // [RP][128] (lanes read consecutive words)
+  __shared__ float tot[(kChunk / R) * kGateChannels];       // [groups][128]
   constexpr int kGroups = kChunk / R;
+  constexpr int kPairs = kGateChannels / 2;
+  static_assert(kPairs * kGroups == kGateThreads, "thread layout");
   const int dkp = p.dkp;
-  const int pairs = dkp / 2;  // == kGateThreads / kGroups
-  float* g_s = gsm;                  // [64][RP]
-  float* w_s = g_s + kChunk * RP;    // [dkp][RP]
-  float* tot = w_s + dkp * RP;       // [kGroups][dkp]
+  const int cblocks = dkp / kGateChannels;
   int bi = 0;
 #pragma unroll 1
   for (int j = 1; j < p.n_branches; ++j)
     if (static_cast<int>(blockIdx.x) >= p.br[j].block_begin) bi = j;
   const GateBranch& P = p.br[bi];
-  const int local = blockIdx.x - P.block_begin;
+  int local = blockIdx.x - P.block_begin;
+  const int cb = local % cblocks;
+  local /= cblocks;
   const int hc = local % P.n_halves;
   const int head = (local / P.n_halves) % P.heads;
   const int b = local / (P.n_halves * P.heads);
@@ -262,12 +326,12 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
   const int t0 = hc * kChunk;
   const int nrows = min(kChunk, P.rows - t0);
   const int ldk = P.heads * dkp;
+  const int cbase = head * dkp + cb * kGateChannels;  // first channel of this CTA
 
-  const int pair = threadIdx.x % pairs, grp = threadIdx.x / pairs;
-  const int a0 = 2 * pair;
-  const int ch = head * dkp + a0;
+  const int pair = threadIdx.x % kPairs, grp = threadIdx.x / kPairs;
+  const int a0 = 2 * pair;  // channel offset inside the CTA's 128
+  const int ch = cbase + a0;
   const int r0 = grp * R;
-  // issue the q/k loads of this thread's rows first
   __half2 qv[R], kv[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
@@ -279,14 +343,11 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
   }
   for (int i = threadIdx.x; i < nrows * RP; i += blockDim.x)
     g_s[i] = P.g[(static_cast<size_t>(b) * P.rows + t0) * RP + i];
-  for (int i = threadIdx.x; i < dkp * RP; i += blockDim.x) w_s[i] = P.Wg2[static_cast<size_t>(head) * dkp * RP + i];
-  __syncthreads();
-  float w0[RP], w1[RP];
-#pragma unroll
-  for (int r = 0; r < RP; ++r) {
-    w0[r] = w_s[a0 * RP + r];
-    w1[r] = w_s[(a0 + 1) * RP + r];
+  for (int i = threadIdx.x; i < kGateChannels * RP; i += blockDim.x) {
+    const int r = i / kGateChannels, a = i % kGateChannels;
+    w_s[i] = P.Wg2[static_cast<size_t>(cbase + a) * RP + r];
   }
+  __syncthreads();
   const float bias0 = P.bg[ch], bias1 = P.bg[ch + 1];
   float c0[R], c1[R];
   float run0 = 0.f, run1 = 0.f;
@@ -297,23 +358,24 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
       float z0 = bias0, z1 = bias1;
 #pragma unroll
       for (int u = 0; u < RP; ++u) {
-        z0 = fmaf(gi[u], w0[u], z0);
-        z1 = fmaf(gi[u], w1[u], z1);
+        const float2 wv = *reinterpret_cast<const float2*>(w_s + u * kGateChannels + a0);
+        z0 = fmaf(gi[u], wv.x, z0);
+        z1 = fmaf(gi[u], wv.y, z1);
       }
-      // logsigmoid(z) = min(z, 0) - log(1 + e^{-|z|})
-      run0 += (fminf(z0, 0.f) - log1pf(__expf(-fabsf(z0)))) * p.inv_normalizer;
-      run1 += (fminf(z1, 0.f) - log1pf(__expf(-fabsf(z1)))) * p.inv_normalizer;
+      // logsigmoid(z) = min(z, 0) - log(1 + e^{-|z|}); the log argument lies in (1, 2]
+      run0 += (fminf(z0, 0.f) - __logf(1.f + __expf(-fabsf(z0)))) * p.inv_normalizer;
+      run1 += (fminf(z1, 0.f) - __logf(1.f + __expf(-fabsf(z1)))) * p.inv_normalizer;
     }
     c0[r] = run0;
     c1[r] = run1;
   }
-  tot[grp * dkp + a0] = run0;
-  tot[grp * dkp + a0 + 1] = run1;
+  tot[grp * kGateChannels + a0] = run0;
+  tot[grp * kGateChannels + a0 + 1] = run1;
   __syncthreads();
   float pre0 = 0.f, pre1 = 0.f, all0 = 0.f, all1 = 0.f;
 #pragma unroll
   for (int g2 = 0; g2 < kGroups; ++g2) {
-    const float x0 = tot[g2 * dkp + a0], x1 = tot[g2 * dkp + a0 + 1];
+    const float x0 = tot[g2 * kGateChannels + a0], x1 = tot[g2 * kGateChannels + a0 + 1];
     if (g2 < grp) {
       pre0 += x0;
       pre1 += x1;
@@ -356,13 +418,9 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
   if (bad) atomicCAS(p.err, 0, kDevRange);
 }
 
-template <int RP, int R>
+template <int RP>
 cudaError_t launch_gate_t(const GateParams& p, cudaStream_t st) {
-  const int groups = kChunk / R;
-  const int smem = (kChunk * RP + p.dkp * RP + groups * p.dkp) * static_cast<int>(sizeof(float));
-  cudaError_t e = cudaFuncSetAttribute(gate_kernel<RP, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  gate_kernel<RP, R><<<p.total_blocks, kGateThreads, smem, st>>>(p);
+  gate_kernel<RP, 16><<<p.total_blocks, kGateThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -422,23 +480,39 @@ __global__ void bf16_copy_rows_kernel(const __nv_bfloat16* src, int src_ld, int 
 
 }  // namespace
 
-template <int P>
+template <int P, int GPL, int NS>
 cudaError_t launch_pool_rows(const PoolParams& p, cudaStream_t st) {
   const int smem = p.n_scales * p.d * static_cast<int>(sizeof(float));
-  cudaError_t e = cudaFuncSetAttribute(pool_fuse_rows_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(pool_fuse_rows_kernel<P, GPL, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const size_t warps = static_cast<size_t>(p.B) * ((p.L + P - 1) / P);
-  pool_fuse_rows_kernel<P><<<static_cast<unsigned>((warps + 7) / 8), 256, smem, st>>>(p);
+  pool_fuse_rows_kernel<P, GPL, NS><<<static_cast<unsigned>((warps + 7) / 8), 256, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int P>
+cudaError_t launch_pool_only(const PoolParams& p, cudaStream_t st) {
+  const size_t n = static_cast<size_t>(p.B) * ((p.L + P - 1) / P) * (p.d / 8);
+  pool_rows_kernel<P><<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st) {
   if (p.B * p.L == 0) return cudaSuccess;
+  if (!p.want_w) {
+    if (p.block_rows <= 2) return launch_pool_only<2>(p, st);
+    if (p.block_rows <= 4) return launch_pool_only<4>(p, st);
+    if (p.block_rows <= 8) return launch_pool_only<8>(p, st);
+  }
   // block_rows carries the least common multiple of the coarse scales (1 if none)
-  if (p.block_rows <= 4 && p.n_scales * p.d * 4 <= 160 * 1024) return launch_pool_rows<4>(p, st);
-  if (p.block_rows == 8 && p.n_scales * p.d * 4 <= 160 * 1024) return launch_pool_rows<8>(p, st);
+  if (p.n_scales * p.d * 4 <= 160 * 1024) {
+    if (p.block_rows <= 4)
+      return p.n_scales <= 4 ? launch_pool_rows<4, 4, 4>(p, st) : launch_pool_rows<4, 4, 8>(p, st);
+    if (p.block_rows == 8)
+      return p.n_scales <= 4 ? launch_pool_rows<8, 2, 4>(p, st) : launch_pool_rows<8, 2, 8>(p, st);
+  }
   PoolParams q = p;
-  q.block_rows = p.block_rows;
   while (q.block_rows < 32) q.block_rows *= 2;
   dim3 grid((p.L + q.block_rows - 1) / q.block_rows, p.B);
   pool_fuse_kernel<<<grid, kPoolThreads, 0, st>>>(q);
@@ -447,10 +521,8 @@ cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st) {
 
 cudaError_t launch_gate(const GateParams& p, cudaStream_t st) {
   if (p.total_blocks <= 0) return cudaSuccess;
-  // 512 threads = (dkp/2) channel pairs x groups; rows per group R = 64 / groups
-  if (p.dkp == 256) return p.rp == 16 ? launch_gate_t<16, 16>(p, st) : launch_gate_t<32, 16>(p, st);
-  if (p.dkp == 128) return p.rp == 16 ? launch_gate_t<16, 8>(p, st) : launch_gate_t<32, 8>(p, st);
-  return cudaErrorInvalidValue;
+  if (p.dkp % kGateChannels) return cudaErrorInvalidValue;
+  return p.rp == 16 ? launch_gate_t<16>(p, st) : launch_gate_t<32>(p, st);
 }
 
 cudaError_t launch_hold_fuse(const HoldFuseParams& p, cudaStream_t st) {

@@ -119,6 +119,7 @@ struct msgla_handle {
   msgla_config cfg;
   int device;
   int dkp, dvp, rp, n_scales, main_index, pool_rows;
+  int nzp, ldz;  // fusion-logit rows in the scale-1 packed weights (16) and z row stride
   Branch br[MSGLA_MAX_SCALES];
   __nv_bfloat16* Wfuse;
   float* bfuse;
@@ -136,7 +137,7 @@ struct BranchWs {
 };
 struct Workspace {
   BranchWs br[MSGLA_MAX_SCALES];
-  Region w;
+  Region w, z;
   size_t total = 0;
 };
 
@@ -171,6 +172,7 @@ Workspace layout(const msgla_handle* h, int B, int L) {
     if (j != h->main_index) add(w.Y, cur, n * d * 2);
   }
   add(ws.w, cur, BB * L * h->n_scales * 4);
+  if (h->main_index >= 0) add(ws.z, cur, BB * L * h->ldz * 4);
   ws.total = cur;
   return ws;
 }
@@ -273,6 +275,10 @@ int create_impl(msgla_handle* h, const msgla_weights* w) {
                                        0));
     }
     CUDA_TRY(put_rows(w->Wg1[j], 0, r, hh * (2 * h->dkp + h->dvp)));
+    if (j == h->main_index) {
+      if (!w->Wfuse) return fail(MSGLA_ERR_INVALID_ARG, "Wfuse is NULL");
+      CUDA_TRY(put_rows(w->Wfuse, 0, h->n_scales, hh * (2 * h->dkp + h->dvp) + h->rp));
+    }
   }
   if (!w->Wfuse) return fail(MSGLA_ERR_INVALID_ARG, "Wfuse is NULL");
   if ((st = dmalloc_zero(&h->Wfuse, static_cast<size_t>(h->n_scales) * d * 2))) return st;
@@ -332,9 +338,14 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   pp.bfuse = h->bfuse;
   pp.w = static_cast<float*>(at(ws.w));
   pp.block_rows = h->pool_rows;
+  pp.want_w = h->main_index < 0 ? 1 : 0;
   pp.err = h->d_err;
-  CUDA_TRY(launch_pool_fuse(pp, st));
-  CUDA_TRY(rec->mark(st));
+  // nothing to pool and no fusion weights to form: single-scale layer
+  const bool need_pool = pp.want_w || h->pool_rows > 1;
+  if (need_pool) {
+    CUDA_TRY(launch_pool_fuse(pp, st));
+    CUDA_TRY(rec->mark(st));
+  }
 
   // 2. projections (grouped over branches)
   static thread_local GemmParams gp;
@@ -360,6 +371,9 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.nq = t.nk = b.heads * h->dkp;
     t.nv = b.heads * h->dvp;
     t.ng = h->rp;
+    t.nz = (j == h->main_index) ? h->n_scales : 0;
+    t.ldz = h->ldz;
+    t.z = (j == h->main_index) ? static_cast<float*>(at(ws.z)) : nullptr;
     t.q = static_cast<__half*>(at(bw.q));
     t.k = static_cast<__half*>(at(bw.k));
     t.v = static_cast<__half*>(at(bw.v));
@@ -392,7 +406,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
       q.heads = b.heads;
       q.n_halves = bw.n_halves;
       q.block_begin = blocks;
-      blocks += B * b.heads * bw.n_halves;
+      blocks += B * b.heads * bw.n_halves * (h->dkp / 128);
     }
     g.n_branches = ns;
     g.total_blocks = blocks;
@@ -486,7 +500,10 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.ab_bf16 = 0;
     t.epi = kEpiFuse;
     t.out = static_cast<__nv_bfloat16*>(O);
-    t.w = static_cast<const float*>(at(ws.w));
+    t.zf = static_cast<const float*>(at(ws.z));
+    t.ldz = h->ldz;
+    t.bfuse = h->bfuse;
+    t.w = static_cast<float*>(at(ws.w));
     t.n_scales = ns;
     t.main_index = j;
     int nc = 0;
@@ -597,12 +614,17 @@ int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weight
   h->dvp = static_cast<int>(round_up(cfg->d_v, kGlaTile));
   h->rp = static_cast<int>(round_up(cfg->gate_rank, 16));
   h->main_index = -1;
+  h->nzp = 16;
+  h->ldz = cfg->n_scales <= 4 ? 4 : 8;
   int lcm = 1;
   for (int j = 0; j < h->n_scales; ++j) {
     h->br[j].scale = cfg->scales[j];
     h->br[j].heads = cfg->heads[j];
     h->br[j].np = cfg->heads[j] * (2 * h->dkp + h->dvp) + h->rp;
-    if (cfg->scales[j] == 1) h->main_index = j;
+    if (cfg->scales[j] == 1) {
+      h->main_index = j;
+      h->br[j].np += 16;  // fusion logits W_fuse x (n_scales <= 8 rows, zero padded)
+    }
     else lcm = lcm / gcd(lcm, cfg->scales[j]) * cfg->scales[j];
   }
   h->pool_rows = lcm;  // least common multiple of the coarse scales

@@ -30,17 +30,20 @@ struct alignas(64) GemmTask {
   CUtensorMap tmA;  // 3D {K, rows, B}, box {64, 128, 1}, 128B swizzle
   CUtensorMap tmB;  // 2D {K, N}, box {64, BN}, 128B swizzle
   int rows, m_tiles, n_tiles, N, K, tile_begin, ab_bf16, epi;
-  // kEpiProj
-  int nq, nk, nv, ng;
+  // kEpiProj (columns: q | k | v | g (ng) | fusion logits z (nz, scale-1 branch))
+  int nq, nk, nv, ng, nz, ldz;
   __half* q;
   __half* k;
   __half* v;
   float* g;
+  float* z;  // [B, rows, ldz] fp32
   // kEpiStoreF16
   __half* y;
   // kEpiFuse (rows == L, the branch with scale 1)
   __nv_bfloat16* out;
-  const float* w;   // [B, L, n_scales]
+  const float* zf;     // fusion logits [B, L, ldz] from the projection GEMM
+  const float* bfuse;  // [n_scales]
+  float* w;            // fusion weights [B, L, n_scales] (written by the n0 == 0 tiles)
   int n_scales, main_index, n_coarse, pad_;
   int coarse_scale[kMaxScales];
   int coarse_index[kMaxScales];
@@ -89,6 +92,7 @@ struct PoolParams {
   const float* bfuse;          // [n_scales]
   float* w;                    // [B, L, n_scales]
   int block_rows;              // least common multiple of the scales > 1 (1 if none)
+  int want_w;                  // 1: also the fusion weights (no scale-1 branch)
   int* err;
 };
 cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st);
