@@ -261,10 +261,47 @@ __global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
 #pragma unroll
   for (int r = 0; r < P; ++r) bf16x8_to_f32(raw[r], x[r]);
   bool bad = false;
+  auto put = [&](int j, int s, int i0, const float (&m)[8], float inv) {
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a0 = m[2 * e] * inv, a1 = m[2 * e + 1] * inv;
+      bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
+      ow[e] = pack_half2(a0, a1);
+    }
+    const int n_s = (p.L + s - 1) / s;
+    reinterpret_cast<uint4*>(p.Xp[j] + (static_cast<size_t>(b) * n_s + (row0 + i0) / s) * p.d)[cg] = o;
+  };
+  if (nrows == P) {
+    // complete block: sums over aligned groups of 2, 4, ... rows as a pairwise tree
+    float lv[P][8];
+#pragma unroll
+    for (int r = 0; r < P; ++r)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lv[r][e] = x[r][e];
+    int width = 1;
+#pragma unroll
+    for (int level = 0; (1 << level) < P; ++level) {
+      // lv[i] holds the sum of rows [i*width, (i+1)*width)
+      const int n = P >> level;
+#pragma unroll
+      for (int i = 0; i < P / 2; ++i)
+        if (i < n / 2)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) lv[i][e] = lv[2 * i][e] + lv[2 * i + 1][e];
+      width <<= 1;
+      for (int j = 0; j < p.n_scales; ++j) {
+        if (p.scales[j] != width) continue;
+#pragma unroll
+        for (int i = 0; i < P / 2; ++i)
+          if (i < n / 2) put(j, width, i * width, lv[i], 1.f / static_cast<float>(width));
+      }
+    }
+  }
   for (int j = 0; j < p.n_scales; ++j) {
     const int s = p.scales[j];
-    if (s == 1) continue;
-    const int n_s = (p.L + s - 1) / s;
+    if (s == 1 || (nrows == P && (s & (s - 1)) == 0)) continue;  // done above
     for (int i0 = 0; i0 < nrows; i0 += s) {
       const int cnt = min(s, nrows - i0);
       float m[8];
@@ -275,39 +312,53 @@ __global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
         if (r >= i0 && r < i0 + cnt)
 #pragma unroll
           for (int e = 0; e < 8; ++e) m[e] += x[r][e];
-      const float inv = 1.f / static_cast<float>(cnt);
-      uint4 o;
-      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float a0 = m[2 * e] * inv, a1 = m[2 * e + 1] * inv;
-        bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
-        ow[e] = pack_half2(a0, a1);
-      }
-      reinterpret_cast<uint4*>(p.Xp[j] + (static_cast<size_t>(b) * n_s + (row0 + i0) / s) * p.d)[cg] = o;
+      put(j, s, i0, m, 1.f / static_cast<float>(cnt));
     }
   }
   if (bad) atomicCAS(p.err, 0, kDevRange);
 }
 
 constexpr int kGateThreads = 256;
-constexpr int kGateChannels = 128;  // key channels per CTA (64 pairs x 4 row groups of 16)
+constexpr int kGateChannels = 128;  // key channels per CTA
+
+// tf32 split of an fp32 value: hi has the top 10 mantissa bits, lo the rest.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  uint32_t h;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+  float r = x - __uint_as_float(h);
+  uint32_t l;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(l) : "f"(r));
+  hi = h;
+  lo = l;
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
 
 // One CTA per (branch, batch, head, 64-row half of a 128-row GLA chunk, 128 key
-// channels); 256 threads = 64 channel pairs x 4 row groups of R = 16 rows. Every
-// thread issues all of its q/k loads first, computes log alpha for its rows and a
-// local cumulative sum, then adds the totals of the preceding row groups (through
-// shared memory). With b_loc the cumulative sum from the half's first row and T
-// its total: in the first half b - m = b_loc - T, in the second half b - m = b_loc
-// (m is the first half's total), so each half needs only its own rows.
-template <int RP, int R>
-__global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constant__ GateParams p) {
-  __shared__ float g_s[kChunk * RP];                        // [64][RP]
-  __shared__ __align__(16) float w_s[RP * kGateChannels];   // [RP][128] (lanes read consecutive words)
-  __shared__ float tot[(kChunk / R) * kGateChannels];       // [groups][128]
-  constexpr int kGroups = kChunk / R;
-  constexpr int kPairs = kGateChannels / 2;
+// channels), 256 threads.
+//  1. z = g W_g2^T for the 64 x 128 block on tensor cores (mma.sync m16n8k8 tf32;
+//     each operand split into tf32 hi + lo parts, three products, so z keeps
+//     fp32-level accuracy), then log alpha = logsigmoid(z + b_g) / normalizer in
+//     registers, stored to shared memory.
+//  2. 64 channel pairs x 4 row groups of 16 rows: each thread issues its q/k loads,
+//     forms the local cumulative sum of log alpha over its rows, adds the
+//     totals of the preceding row groups, and writes Qs = q e^{b - m},
+//     Ks = k e^{m - b}. With b_loc the cumulative sum from the half's first row
+//     and T its total: in the first half b - m = b_loc - T, in the second half
+//     b - m = b_loc (m is the first half's total), so each half needs only its
+//     own rows. Per chunk: gamma = e^{b_last - m}, mid = e^{m}.
+template <int RP>
+__global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_constant__ GateParams p) {
+  constexpr int R = 16, kGroups = kChunk / R, kPairs = kGateChannels / 2;
   static_assert(kPairs * kGroups == kGateThreads, "thread layout");
+  __shared__ float la_s[kChunk][kGateChannels + 4];  // log alpha (row, channel), padded rows
+  __shared__ float tot[kGroups][kGateChannels];
   const int dkp = p.dkp;
   const int cblocks = dkp / kGateChannels;
   int bi = 0;
@@ -327,55 +378,108 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
   const int nrows = min(kChunk, P.rows - t0);
   const int ldk = P.heads * dkp;
   const int cbase = head * dkp + cb * kGateChannels;  // first channel of this CTA
+  const size_t row_base = static_cast<size_t>(b) * P.rows + t0;
 
-  const int pair = threadIdx.x % kPairs, grp = threadIdx.x / kPairs;
-  const int a0 = 2 * pair;  // channel offset inside the CTA's 128
-  const int ch = cbase + a0;
-  const int r0 = grp * R;
-  __half2 qv[R], kv[R];
+
+  // ---- phase 1: z = g W^T on tensor cores. Warp w owns channels [16w, 16w+16)
+  // (two n8 tiles) for all 64 rows (four m16 tiles); K = RP in steps of 8.
+  {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gq = lane >> 2, tq = lane & 3;
+    float acc[4][2][4];
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    if (r0 + r < nrows) {
-      const size_t idx = (static_cast<size_t>(b) * P.rows + t0 + r0 + r) * ldk + ch;
-      qv[r] = *reinterpret_cast<const __half2*>(P.q + idx);
-      kv[r] = *reinterpret_cast<const __half2*>(P.k + idx);
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+    const float* gsrc = P.g + row_base * RP;
+#pragma unroll
+    for (int k8 = 0; k8 < RP / 8; ++k8) {
+      // B fragments: W[channel][k]; b0 = (k = tq, n = gq), b1 = (k = tq + 4, n = gq)
+      uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const float* wr = P.Wg2 + static_cast<size_t>(cbase + warp * 16 + nt * 8 + gq) * RP + k8 * 8;
+        split_tf32(__ldg(wr + tq), bh[nt][0], bl[nt][0]);
+        split_tf32(__ldg(wr + tq + 4), bh[nt][1], bl[nt][1]);
+      }
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        // A fragments: g[row][k]; a0 = (gq, tq), a1 = (gq + 8, tq), a2 = (gq, tq + 4), a3 = (gq + 8, tq + 4)
+        const int ra = mt * 16 + gq, rb = ra + 8;
+        const float* g0 = gsrc + static_cast<size_t>(ra) * RP + k8 * 8;
+        const float* g1 = gsrc + static_cast<size_t>(rb) * RP + k8 * 8;
+        const float x0 = ra < nrows ? __ldg(g0 + tq) : 0.f, x1 = rb < nrows ? __ldg(g1 + tq) : 0.f;
+        const float x2 = ra < nrows ? __ldg(g0 + tq + 4) : 0.f, x3 = rb < nrows ? __ldg(g1 + tq + 4) : 0.f;
+        uint32_t ah[4], al[4];
+        split_tf32(x0, ah[0], al[0]);
+        split_tf32(x1, ah[1], al[1]);
+        split_tf32(x2, ah[2], al[2]);
+        split_tf32(x3, ah[3], al[3]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          mma_tf32(acc[mt][nt], al, bh[nt]);
+          mma_tf32(acc[mt][nt], ah, bl[nt]);
+          mma_tf32(acc[mt][nt], ah, bh[nt]);
+        }
+      }
+    }
+    // log alpha into shared memory; D fragment: d0 = (gq, 2tq), d1 = (gq, 2tq+1),
+    // d2 = (gq+8, 2tq), d3 = (gq+8, 2tq+1)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int chl = warp * 16 + nt * 8 + 2 * tq;
+      const float bias0 = __ldg(P.bg + cbase + chl), bias1 = __ldg(P.bg + cbase + chl + 1);
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float z = acc[mt][nt][e] + ((e & 1) ? bias1 : bias0);
+          // logsigmoid(z) = min(z, 0) - log(1 + e^{-|z|}); the log argument lies in (1, 2]
+          const float la = (fminf(z, 0.f) - __logf(1.f + __expf(-fabsf(z)))) * p.inv_normalizer;
+          la_s[mt * 16 + gq + ((e & 2) ? 8 : 0)][chl + (e & 1)] = la;
+        }
+      }
     }
   }
-  for (int i = threadIdx.x; i < nrows * RP; i += blockDim.x)
-    g_s[i] = P.g[(static_cast<size_t>(b) * P.rows + t0) * RP + i];
-  for (int i = threadIdx.x; i < kGateChannels * RP; i += blockDim.x) {
-    const int r = i / kGateChannels, a = i % kGateChannels;
-    w_s[i] = P.Wg2[static_cast<size_t>(cbase + a) * RP + r];
-  }
   __syncthreads();
-  const float bias0 = P.bg[ch], bias1 = P.bg[ch + 1];
+
+  // ---- phase 2: cumulative sums along rows and the scaled operands
+  const int pair = threadIdx.x % kPairs, grp = threadIdx.x / kPairs;
+  const int a0 = 2 * pair;
+  const int r0 = grp * R;
+  __half2 qv[R], kv[R];
+  {
+    const __half* qrow = P.q + (row_base + r0) * ldk + cbase + a0;
+    const __half* krow = P.k + (row_base + r0) * ldk + cbase + a0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (r0 + r < nrows) {
+        qv[r] = *reinterpret_cast<const __half2*>(qrow + static_cast<size_t>(r) * ldk);
+        kv[r] = *reinterpret_cast<const __half2*>(krow + static_cast<size_t>(r) * ldk);
+      }
+    }
+  }
   float c0[R], c1[R];
   float run0 = 0.f, run1 = 0.f;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     if (r0 + r < nrows) {
-      const float* gi = g_s + (r0 + r) * RP;
-      float z0 = bias0, z1 = bias1;
-#pragma unroll
-      for (int u = 0; u < RP; ++u) {
-        const float2 wv = *reinterpret_cast<const float2*>(w_s + u * kGateChannels + a0);
-        z0 = fmaf(gi[u], wv.x, z0);
-        z1 = fmaf(gi[u], wv.y, z1);
-      }
-      // logsigmoid(z) = min(z, 0) - log(1 + e^{-|z|}); the log argument lies in (1, 2]
-      run0 += (fminf(z0, 0.f) - __logf(1.f + __expf(-fabsf(z0)))) * p.inv_normalizer;
-      run1 += (fminf(z1, 0.f) - __logf(1.f + __expf(-fabsf(z1)))) * p.inv_normalizer;
+      const float2 l2 = *reinterpret_cast<const float2*>(&la_s[r0 + r][a0]);
+      run0 += l2.x;
+      run1 += l2.y;
     }
     c0[r] = run0;
     c1[r] = run1;
   }
-  tot[grp * kGateChannels + a0] = run0;
-  tot[grp * kGateChannels + a0 + 1] = run1;
+  tot[grp][a0] = run0;
+  tot[grp][a0 + 1] = run1;
   __syncthreads();
   float pre0 = 0.f, pre1 = 0.f, all0 = 0.f, all1 = 0.f;
 #pragma unroll
   for (int g2 = 0; g2 < kGroups; ++g2) {
-    const float x0 = tot[g2 * kGateChannels + a0], x1 = tot[g2 * kGateChannels + a0 + 1];
+    const float x0 = tot[g2][a0], x1 = tot[g2][a0 + 1];
     if (g2 < grp) {
       pre0 += x0;
       pre1 += x1;
@@ -384,25 +488,26 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
     all1 += x1;
   }
   // reference: b - m = b_loc - T in the first half, b_loc in the second
-  const float ref0 = second ? 0.f : all0, ref1 = second ? 0.f : all1;
+  pre0 -= second ? 0.f : all0;
+  pre1 -= second ? 0.f : all1;
   bool bad = false;
+  __half* qrow = P.qs + (row_base + r0) * ldk + cbase + a0;
+  __half* krow = P.ks + (row_base + r0) * ldk + cbase + a0;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     if (r0 + r < nrows) {
-      const float b0 = pre0 + c0[r] - ref0, b1 = pre1 + c1[r] - ref1;
+      const float b0 = pre0 + c0[r], b1 = pre1 + c1[r];
       const float2 qf = __half22float2(qv[r]);
       const float2 kf = __half22float2(kv[r]);
       const float ks0 = kf.x * __expf(-b0), ks1 = kf.y * __expf(-b1);
       const float qs0 = qf.x * __expf(b0), qs1 = qf.y * __expf(b1);
-      bad |= !(fabsf(ks0) <= 65504.f) || !(fabsf(ks1) <= 65504.f) || !(fabsf(qs0) <= 65504.f) ||
-             !(fabsf(qs1) <= 65504.f);
-      const size_t idx = (static_cast<size_t>(b) * P.rows + t0 + r0 + r) * ldk + ch;
-      *reinterpret_cast<__half2*>(P.qs + idx) = __floats2half2_rn(qs0, qs1);
-      *reinterpret_cast<__half2*>(P.ks + idx) = __floats2half2_rn(ks0, ks1);
+      bad |= fmaxf(fmaxf(fabsf(ks0), fabsf(ks1)), fmaxf(fabsf(qs0), fabsf(qs1))) > 65504.f;
+      *reinterpret_cast<__half2*>(qrow + static_cast<size_t>(r) * ldk) = __floats2half2_rn(qs0, qs1);
+      *reinterpret_cast<__half2*>(krow + static_cast<size_t>(r) * ldk) = __floats2half2_rn(ks0, ks1);
     }
   }
   if (grp == 0) {
-    const size_t gi = (static_cast<size_t>(b) * n_chunks + c) * ldk + ch;
+    const size_t gi = (static_cast<size_t>(b) * n_chunks + c) * ldk + cbase + a0;
     if (second) {
       P.gamma[gi] = __expf(all0);
       P.gamma[gi + 1] = __expf(all1);
@@ -420,7 +525,7 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
 
 template <int RP>
 cudaError_t launch_gate_t(const GateParams& p, cudaStream_t st) {
-  gate_kernel<RP, 16><<<p.total_blocks, kGateThreads, 0, st>>>(p);
+  gate_kernel<RP><<<p.total_blocks, kGateThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
