@@ -321,6 +321,13 @@ __global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
 constexpr int kGateThreads = 256;
 constexpr int kGateChannels = 128;  // key channels per CTA
 
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // tf32 split of an fp32 value: hi has the top 10 mantissa bits, lo the rest.
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
   uint32_t h;
@@ -346,8 +353,8 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 //     each operand split into tf32 hi + lo parts, three products, so z keeps
 //     fp32-level accuracy), then log alpha = logsigmoid(z + b_g) / normalizer in
 //     registers, stored to shared memory.
-//  2. 64 channel pairs x 4 row groups of 16 rows: each thread issues its q/k loads,
-//     forms the local cumulative sum of log alpha over its rows, adds the
+//  2. 64 channel pairs x 4 row groups of 16 rows (q, k staged in shared memory by
+//     cp.async during phase 1): each thread forms the local cumulative sum of log alpha over its rows, adds the
 //     totals of the preceding row groups, and writes Qs = q e^{b - m},
 //     Ks = k e^{m - b}. With b_loc the cumulative sum from the half's first row
 //     and T its total: in the first half b - m = b_loc - T, in the second half
@@ -359,6 +366,7 @@ __global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_cons
   static_assert(kPairs * kGroups == kGateThreads, "thread layout");
   __shared__ float la_s[kChunk][kGateChannels + 4];  // log alpha (row, channel), padded rows
   __shared__ float tot[kGroups][kGateChannels];
+  extern __shared__ __align__(16) __half qk_s[];      // [2][64][128]: this CTA's q and k rows
   const int dkp = p.dkp;
   const int cblocks = dkp / kGateChannels;
   int bi = 0;
@@ -380,6 +388,14 @@ __global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_cons
   const int cbase = head * dkp + cb * kGateChannels;  // first channel of this CTA
   const size_t row_base = static_cast<size_t>(b) * P.rows + t0;
 
+  // ---- the q and k rows of this CTA go to shared memory asynchronously while
+  // phase 1 runs (16-byte copies: 16 per row and tensor)
+  for (int i = threadIdx.x; i < 2 * nrows * 16; i += blockDim.x) {
+    const int tsel = i / (nrows * 16), rem = i % (nrows * 16);
+    const int row = rem >> 4, seg = rem & 15;
+    const __half* src = (tsel ? P.k : P.q) + (row_base + row) * ldk + cbase + seg * 8;
+    cp_async16(qk_s + (tsel * kChunk + row) * kGateChannels + seg * 8, src);
+  }
 
   // ---- phase 1: z = g W^T on tensor cores. Warp w owns channels [16w, 16w+16)
   // (two n8 tiles) for all 64 rows (four m16 tiles); K = RP in steps of 8.
@@ -443,24 +459,13 @@ __global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_cons
       }
     }
   }
+  cp_async_wait_all();
   __syncthreads();
 
   // ---- phase 2: cumulative sums along rows and the scaled operands
   const int pair = threadIdx.x % kPairs, grp = threadIdx.x / kPairs;
   const int a0 = 2 * pair;
   const int r0 = grp * R;
-  __half2 qv[R], kv[R];
-  {
-    const __half* qrow = P.q + (row_base + r0) * ldk + cbase + a0;
-    const __half* krow = P.k + (row_base + r0) * ldk + cbase + a0;
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      if (r0 + r < nrows) {
-        qv[r] = *reinterpret_cast<const __half2*>(qrow + static_cast<size_t>(r) * ldk);
-        kv[r] = *reinterpret_cast<const __half2*>(krow + static_cast<size_t>(r) * ldk);
-      }
-    }
-  }
   float c0[R], c1[R];
   float run0 = 0.f, run1 = 0.f;
 #pragma unroll
@@ -497,8 +502,9 @@ __global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_cons
   for (int r = 0; r < R; ++r) {
     if (r0 + r < nrows) {
       const float b0 = pre0 + c0[r], b1 = pre1 + c1[r];
-      const float2 qf = __half22float2(qv[r]);
-      const float2 kf = __half22float2(kv[r]);
+      const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(qk_s + (r0 + r) * kGateChannels + a0));
+      const float2 kf =
+          __half22float2(*reinterpret_cast<const __half2*>(qk_s + (kChunk + r0 + r) * kGateChannels + a0));
       const float ks0 = kf.x * __expf(-b0), ks1 = kf.y * __expf(-b1);
       const float qs0 = qf.x * __expf(b0), qs1 = qf.y * __expf(b1);
       bad |= fmaxf(fmaxf(fabsf(ks0), fabsf(ks1)), fmaxf(fabsf(qs0), fabsf(qs1))) > 65504.f;
@@ -525,7 +531,10 @@ __global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_cons
 
 template <int RP>
 cudaError_t launch_gate_t(const GateParams& p, cudaStream_t st) {
-  gate_kernel<RP><<<p.total_blocks, kGateThreads, 0, st>>>(p);
+  const int smem = 2 * kChunk * kGateChannels * static_cast<int>(sizeof(__half));
+  cudaError_t e = cudaFuncSetAttribute(gate_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  gate_kernel<RP><<<p.total_blocks, kGateThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -358,7 +358,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     GemmTask& t = gp.task[j];
     const bool bf = (b.scale == 1);
     if (!encode_3d(&t.tmA, bf, bf ? X : at(bw.Xp), d, bw.rows, B, kGemmBM) ||
-        !encode_2d(&t.tmB, bf, b.Bproj, d, b.np, 256))
+        !encode_2d(&t.tmB, bf, b.Bproj, d, b.np, 128))
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (projection, scale %d)", b.scale);
     t.rows = bw.rows;
     t.m_tiles = ceil_div(bw.rows, kGemmBM);
@@ -460,7 +460,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     const BranchWs& bw = ws.br[j];
     GemmTask& t = gp.task[nt++];
     if (!encode_3d(&t.tmA, false, at(bw.o), b.heads * h->dvp, bw.rows, B, kGemmBM) ||
-        !encode_2d(&t.tmB, false, b.Wop, b.heads * h->dvp, d, 256))
+        !encode_2d(&t.tmB, false, b.Wop, b.heads * h->dvp, d, 128))
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (output, scale %d)", b.scale);
     t.rows = bw.rows;
     t.m_tiles = ceil_div(bw.rows, kGemmBM);
@@ -489,7 +489,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     const BranchWs& bw = ws.br[j];
     GemmTask& t = gp.task[0];
     if (!encode_3d(&t.tmA, false, at(bw.o), b.heads * h->dvp, bw.rows, B, kGemmBM) ||
-        !encode_2d(&t.tmB, false, b.Wop, b.heads * h->dvp, d, 256))
+        !encode_2d(&t.tmB, false, b.Wop, b.heads * h->dvp, d, 128))
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (output, scale 1)");
     t.rows = bw.rows;
     t.m_tiles = ceil_div(bw.rows, kGemmBM);

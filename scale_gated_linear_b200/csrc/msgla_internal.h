@@ -28,7 +28,7 @@ enum EpiKind : int {
 // One GEMM D[rows x N] = A[rows x K] * B[N x K]^T per batch, tiled 128 x BN.
 struct alignas(64) GemmTask {
   CUtensorMap tmA;  // 3D {K, rows, B}, box {64, 128, 1}, 128B swizzle
-  CUtensorMap tmB;  // 2D {K, N}, box {64, BN}, 128B swizzle
+  CUtensorMap tmB;  // 2D {K, N}, box {64, 128}, 128B swizzle
   int rows, m_tiles, n_tiles, N, K, tile_begin, ab_bf16, epi;
   // kEpiProj (columns: q | k | v | g (ng) | fusion logits z (nz, scale-1 branch))
   int nq, nk, nv, ng, nz, ldz;
