@@ -175,6 +175,15 @@ int msgla_sync_status(msgla_handle* h);
 int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index, int which,
                            size_t* offset, int dims[3]);
 
+/* Failure-detection testing: with enable != 0, the next forward on this handle
+ * runs its chunkwise-GLA kernel with one internal barrier arrival withheld in its
+ * first CTA. The warp waiting on it gives up after its bounded wait (about 2 s),
+ * the kernel exits normally and msgla_sync_status then returns
+ * MSGLA_ERR_DEVICE_TIMEOUT; the output of that forward is undefined. The switch
+ * resets itself after one forward; the handle stays usable. No counterpart in the
+ * pages (it exercises this library's own bounded waits). */
+int msgla_test_skip_arrival(msgla_handle* h, int enable);
+
 /* Static description of an error code. */
 const char* msgla_status_string(int status);
 

@@ -51,6 +51,7 @@ _SIGNATURES = {
     "msgla_forward_host": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "msgla_sync_status": (c_int, [c_void_p]),
     "msgla_workspace_tensor": (c_int, [c_void_p, c_int, c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_int)]),
+    "msgla_test_skip_arrival": (c_int, [c_void_p, c_int]),
     "msgla_status_string": (c_char_p, [c_int]),
     "msgla_last_error": (c_char_p, []),
 }

@@ -200,7 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar[B_A_READY]);
+      // failure-detection tests: CTA 0 may withhold its first arrival, so the MMA
+      // warp's bounded wait runs out and the launch reports a device timeout
+      if (!(p.skip_arrival && blockIdx.x == 0 && c == 0)) mbar_arrive(&bar[B_A_READY]);
 
       if (!mbar_wait(&bar[B_O_FULL], c & 1, abort_flag, p.err)) break;
       tc_fence_after();

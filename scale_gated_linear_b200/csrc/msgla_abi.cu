@@ -124,6 +124,7 @@ struct msgla_handle {
   __nv_bfloat16* Wfuse;
   float* bfuse;
   int* d_err;  // device error word
+  int test_skip_arrival;  // failure-detection tests (msgla_test_skip_arrival)
 };
 
 namespace {
@@ -423,6 +424,8 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   memset(&lp, 0, sizeof(lp));
   lp.err = h->d_err;
   lp.qk_scale = c.qk_scale;
+  lp.skip_arrival = h->test_skip_arrival;
+  h->test_skip_arrival = 0;
   int ctas = 0;
   for (int j = 0; j < ns; ++j) {
     const Branch& b = h->br[j];
@@ -607,6 +610,7 @@ int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weight
   h->Wfuse = nullptr;
   h->bfuse = nullptr;
   h->d_err = nullptr;
+  h->test_skip_arrival = 0;
   h->cfg = *cfg;
   h->device = device;
   h->n_scales = cfg->n_scales;
@@ -807,6 +811,12 @@ int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index,
   dims[0] = B;
   dims[1] = bw.rows;
   dims[2] = cols;
+  return MSGLA_OK;
+}
+
+int msgla_test_skip_arrival(msgla_handle* h, int enable) {
+  if (!h) return fail(MSGLA_ERR_INVALID_ARG, "handle is NULL");
+  h->test_skip_arrival = enable ? 1 : 0;
   return MSGLA_OK;
 }
 

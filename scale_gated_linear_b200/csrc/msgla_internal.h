@@ -74,6 +74,7 @@ struct GlaParams {
   int n_tasks;
   int total_ctas;
   float qk_scale;
+  int skip_arrival;  // failure-detection tests: CTA 0 omits one barrier arrival
   int* err;
 };
 
