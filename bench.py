@@ -286,7 +286,7 @@ def run_ours(args) -> int:
         ws = layer.alloc_workspace(wk.B, wk.L)
         flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
         flush = lambda: flush_buf.fill_(1)
-        names = layer.launch_names()
+        names = layer.launch_names(wk.B, wk.L)
         n_ev = len(names) + 1
         ev = time_layer(layer, X, O, ws, steps, warmup, flush, n_ev)
         torch.cuda.synchronize()

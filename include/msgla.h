@@ -138,11 +138,7 @@ int msgla_forward_noalloc(msgla_handle* h, const void* X, int B, int L, void* O,
 /* msgla_forward that also records CUDA events around its kernels, for timing each
  * kernel on `stream` with events. `events` holds caller-created cudaEvent_t
  * handles: events[0] is recorded before the first kernel and events[i+1] after
- * the i-th kernel. The kernels of one forward, in launch order, are:
- *   pool_fuse (absent for a single scale-1 branch), proj_gemm, gate (all scales), gla,
- *   out_gemm_coarse (only when a scale-1 branch and a coarser branch exist),
- *   out_gemm_fused (scale-1 branch present) or, without a scale-1 branch,
- *   out_gemm_coarse for all branches followed by hold_fuse.
+ * the i-th kernel; msgla_launch_plan lists the kernels in launch order.
  * `max_events` is the length of `events` (it must be at least n_launches + 1);
  * *n_launches receives the number of kernels launched. */
 int msgla_forward_profiled(msgla_handle* h, const void* X, int B, int L, void* O,
@@ -174,6 +170,14 @@ int msgla_sync_status(msgla_handle* h);
  * columns hold zeros. A tensor that does not exist gives MSGLA_ERR_INVALID_ARG. */
 int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index, int which,
                            size_t* offset, int dims[3]);
+
+/* Kernels that msgla_forward launches for a [B, L, d] input, in launch order, as a
+ * comma-separated list written to `names` (NUL-terminated, at most `len` bytes):
+ * pool_fuse, proj_gemm, gate, [gla_state, gla_scan], gla, [out_gemm_coarse],
+ * out_gemm_fused | out_gemm_coarse, hold_fuse. gla_state and gla_scan appear when
+ * long sequences are cut into segments (few sequences: the GLA kernel would fill
+ * less than half of the GPU). msgla_forward_profiled records one event per entry. */
+int msgla_launch_plan(const msgla_handle* h, int B, int L, char* names, size_t len);
 
 /* Failure-detection testing: with enable != 0, the next forward on this handle
  * runs its chunkwise-GLA kernel with one internal barrier arrival withheld in its

@@ -107,17 +107,11 @@ class MSGLA:
 
     __call__ = forward
 
-    def launch_names(self):
-        """Kernel names of one forward, in launch order (see msgla_forward_profiled)."""
-        pool = any(s > 1 for s in self.scales) or 1 not in self.scales
-        names = (["pool_fuse"] if pool else []) + ["proj_gemm", "gate", "gla"]
-        if 1 in self.scales:
-            if len(self.scales) > 1:
-                names.append("out_gemm_coarse")
-            names.append("out_gemm_fused")
-        else:
-            names += ["out_gemm_coarse", "hold_fuse"]
-        return names
+    def launch_names(self, B: int, L: int):
+        """Kernel names of one forward of a [B, L, d] input, in launch order."""
+        buf = ctypes.create_string_buffer(512)
+        _lib.check(self._lib.msgla_launch_plan(self._h, B, L, buf, len(buf)))
+        return buf.value.decode().split(",") if buf.value else []
 
     def forward_profiled(self, X, out, workspace, events, stream=None):
         """forward() recording events[0] before the first kernel and events[i+1]

@@ -52,6 +52,7 @@ _SIGNATURES = {
     "msgla_sync_status": (c_int, [c_void_p]),
     "msgla_workspace_tensor": (c_int, [c_void_p, c_int, c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_int)]),
     "msgla_test_skip_arrival": (c_int, [c_void_p, c_int]),
+    "msgla_launch_plan": (c_int, [c_void_p, c_int, c_int, c_char_p, c_size_t]),
     "msgla_status_string": (c_char_p, [c_int]),
     "msgla_last_error": (c_char_p, []),
 }

@@ -73,13 +73,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
   for (int t = 1; t < p.n_tasks; ++t)
     if (static_cast<int>(blockIdx.x) >= p.task[t].cta_begin) ti = t;
   const GlaTask& T = p.task[ti];
-  const int local = blockIdx.x - T.cta_begin;
+  const bool state_pass = p.mode == 1;
+  const int segs = state_pass ? T.n_segs - 1 : T.n_segs;  // segments launched per sequence
+  int local = blockIdx.x - T.cta_begin;
+  const int seg = local % segs;
+  local /= segs;
   const int vt = local % T.v_tiles;
   const int head = (local / T.v_tiles) % T.heads;
   const int b = local / (T.v_tiles * T.heads);
   const int dkp = T.dkp;
   const int n_half = dkp / 128;  // 1 or 2 state halves
-  const int nch = T.n_chunks;
+  const int nch_all = T.n_chunks;
+  const int c_begin = seg * T.seg_chunks;
+  const int nch = min(T.seg_chunks, nch_all - c_begin);  // chunks of this CTA
+  const bool has_init = !state_pass && seg > 0;          // starts from a carried state
+  const size_t seq_slot = ((static_cast<size_t>(b) * T.heads + head) * T.v_tiles + vt) * T.n_segs;
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
@@ -109,11 +117,13 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
       prefetch_tmap(&T.tmV);
       const uint32_t qk_bytes = static_cast<uint32_t>((dkp / 64) * kAtom);
       for (int c = 0; c < nch; ++c) {
-        const int row = c * kC;
-        if (c > 0 && !mbar_wait(&bar[B_Q_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(&bar[B_Q_FULL], qk_bytes);
-        for (int ka = 0; ka < dkp / 64; ++ka)
-          tma_load_3d(&T.tmQ, &bar[B_Q_FULL], smem + kOffQ + ka * kAtom, head * dkp + ka * 64, row, b);
+        const int row = (c_begin + c) * kC;
+        if (!state_pass) {  // the state pass reads only Ks and V
+          if (c > 0 && !mbar_wait(&bar[B_Q_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
+          mbar_arrive_expect_tx(&bar[B_Q_FULL], qk_bytes);
+          for (int ka = 0; ka < dkp / 64; ++ka)
+            tma_load_3d(&T.tmQ, &bar[B_Q_FULL], smem + kOffQ + ka * kAtom, head * dkp + ka * 64, row, b);
+        }
         if (c > 0 && !mbar_wait(&bar[B_K_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(&bar[B_K_FULL], qk_bytes);
         for (int ka = 0; ka < dkp / 64; ++ka)
@@ -133,12 +143,29 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
       const uint32_t id_mm = idesc_f16(128, 128, 0, 1, 1);  // MN-major x MN-major
       const uint32_t sQ = sbase + kOffQ, sK = sbase + kOffK, sV = sbase + kOffV, sS = sbase + kOffS;
       const uint32_t lbo_s = static_cast<uint32_t>(dkp) * 128;
-      for (int c = 0; c < nch; ++c) {
+      const uint32_t sd0 = has_init ? 1u : 0u;  // state-epilogue completions before chunk 0
+      for (int c = 0; c < nch && state_pass; ++c) {
+        // state pass: S' += Ks^T V and the state epilogue only
+        const uint32_t ph = c & 1;
+        if (!mbar_wait(&bar[B_K_FULL], ph, abort_flag, p.err)) break;
+        if (!mbar_wait(&bar[B_V_FULL], ph, abort_flag, p.err)) break;
+        if (c > 0 && !mbar_wait(&bar[B_S_DONE], (c - 1) & 1, abort_flag, p.err)) break;
+        tc_fence_after();
+        for (int h = 0; h < n_half; ++h)
+          for (int ks = 0; ks < kC / 16; ++ks)
+            umma_f16(tmem + kColS + h * 128, sdesc_sw128(sK + 2 * h * kAtom + ks * 2048, kAtom, 1024),
+                     sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_mm, (c > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(&bar[B_S_FULL]);
+        umma_commit(&bar[B_K_EMPTY]);
+        umma_commit(&bar[B_V_EMPTY]);
+      }
+      for (int c = 0; c < nch && !state_pass; ++c) {
         const uint32_t ph = c & 1, pp = (c - 1) & 1;
+        const bool carried = c > 0 || has_init;  // a state enters this chunk
         if (!mbar_wait(&bar[B_Q_FULL], ph, abort_flag, p.err)) break;
-        if (c > 0) {
-          if (!mbar_wait(&bar[B_S_DONE], pp, abort_flag, p.err)) break;
-          if (!mbar_wait(&bar[B_O_EMPTY], pp, abort_flag, p.err)) break;
+        if (carried) {
+          if (!mbar_wait(&bar[B_S_DONE], (c - 1 + sd0) & 1, abort_flag, p.err)) break;
+          if (c > 0 && !mbar_wait(&bar[B_O_EMPTY], pp, abort_flag, p.err)) break;
           tc_fence_after();
           // o = Qs S'  (K = d_k)
           for (int ks = 0; ks < dkp / 16; ++ks)
@@ -159,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
         for (int h = 0; h < n_half; ++h)
           for (int ks = 0; ks < kC / 16; ++ks)
             umma_f16(tmem + kColS + h * 128, sdesc_sw128(sK + 2 * h * kAtom + ks * 2048, kAtom, 1024),
-                     sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_mm, (c > 0 || ks > 0) ? 1u : 0u);
+                     sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_mm, (carried || ks > 0) ? 1u : 0u);
         umma_commit(&bar[B_S_FULL]);
         umma_commit(&bar[B_K_EMPTY]);
         if (!mbar_wait(&bar[B_A_READY], ph, abort_flag, p.err)) break;
@@ -167,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
         // o += A V  (A fp16 in TMEM, 8 columns per 16 rows j)
         for (int ks = 0; ks < kC / 16; ++ks)
           umma_f16_ts(tmem + kColO, tmem + kColA + ks * 8, sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_km,
-                      (c > 0 || ks > 0) ? 1u : 0u);
+                      (carried || ks > 0) ? 1u : 0u);
         umma_commit(&bar[B_O_FULL]);
         umma_commit(&bar[B_V_EMPTY]);
       }
@@ -177,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
     const int quad = warp & 3;
     const int i = quad * 32 + lane;  // chunk row (TMEM lane)
     const size_t ld_o = static_cast<size_t>(T.heads) * T.dvp;
-    for (int c = 0; c < nch; ++c) {
+    for (int c = 0; c < nch && !state_pass; ++c) {
       if (!mbar_wait(&bar[B_A_FULL], c & 1, abort_flag, p.err)) break;
       tc_fence_after();
 #pragma unroll 1
@@ -206,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
 
       if (!mbar_wait(&bar[B_O_FULL], c & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      const int t = c * kC + i;
+      const int t = (c_begin + c) * kC + i;
       __half* dst = T.o + (static_cast<size_t>(b) * T.rows + t) * ld_o + head * T.dvp + vt * kGlaTile;
 #pragma unroll 1
       for (int h2 = 0; h2 < 2; ++h2) {
@@ -242,14 +269,57 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
       const int a = g * 128 + quad * 32 + lane;  // d_k row
       uint8_t* sS = smem + kOffS;
       const size_t ld_g = static_cast<size_t>(T.heads) * dkp;
-      const float* gp = T.gamma + static_cast<size_t>(b) * nch * ld_g + head * dkp + a;
-      const float* mp = T.mid + static_cast<size_t>(b) * nch * ld_g + head * dkp + a;
-      float f = __ldg(gp) * (nch > 1 ? __ldg(mp + ld_g) : 1.f);
+      const float* gp = T.gamma + static_cast<size_t>(b) * nch_all * ld_g + head * dkp + a;
+      const float* mp = T.mid + static_cast<size_t>(b) * nch_all * ld_g + head * dkp + a;
+      // factor of global chunk cg: gamma_cg * mid_{cg+1} (1 past the sequence's end)
+      auto factor = [&](int cg) {
+        return __ldg(gp + static_cast<size_t>(cg) * ld_g) *
+               (cg + 1 < nch_all ? __ldg(mp + static_cast<size_t>(cg + 1) * ld_g) : 1.f);
+      };
+      // fp16 copy of 64 value columns (q2-th MN block) of row a for the o = Qs S' product
+      auto put_f16 = [&](int q2, const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
+        uint8_t* row = sS + q2 * dkp * 128 + a * 128;
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const uint32_t* r = e4 < 4 ? ra + 8 * e4 : rb + 8 * (e4 - 4);
+          st_shared_v4(smem_u32(row + ((e4 ^ (a & 7)) << 4)), pack_half2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                       pack_half2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                       pack_half2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                       pack_half2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+        }
+      };
+      if (has_init) {
+        // carried state of this segment (written by the scan) into TMEM and smem
+        const float4* src =
+            reinterpret_cast<const float4*>(T.seg_state + ((seq_slot + seg - 1) * dkp + a) * kGlaTile);
+#pragma unroll 1
+        for (int q2 = 0; q2 < 2; ++q2) {
+          uint32_t ra[32], rb[32];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 x = __ldg(src + q2 * 16 + e), y = __ldg(src + q2 * 16 + 8 + e);
+            ra[4 * e] = __float_as_uint(x.x), ra[4 * e + 1] = __float_as_uint(x.y);
+            ra[4 * e + 2] = __float_as_uint(x.z), ra[4 * e + 3] = __float_as_uint(x.w);
+            rb[4 * e] = __float_as_uint(y.x), rb[4 * e + 1] = __float_as_uint(y.y);
+            rb[4 * e + 2] = __float_as_uint(y.z), rb[4 * e + 3] = __float_as_uint(y.w);
+          }
+          const uint32_t ta = tmem_addr(tmem, quad * 32, kColS + g * 128 + q2 * 64);
+          tmem_st32(ta, ra);
+          tmem_st32(ta + 32, rb);
+          put_f16(q2, ra, rb);
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bar[B_S_DONE]);
+      }
+      float decay = 1.f;  // product of this segment's factors (state pass)
+      float f = factor(c_begin);
       for (int c = 0; c < nch; ++c) {
-        const float f_next =
-            (c + 1 < nch) ? __ldg(gp + (c + 1) * ld_g) * ((c + 2 < nch) ? __ldg(mp + (c + 2) * ld_g) : 1.f) : 0.f;
+        const float f_next = (c + 1 < nch) ? factor(c_begin + c + 1) : 0.f;
         if (!mbar_wait(&bar[B_S_FULL], c & 1, abort_flag, p.err)) break;
         tc_fence_after();
+        const bool last = c + 1 == nch;
 #pragma unroll 1
         for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t ra[32], rb[32];
@@ -264,24 +334,28 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
           }
           tmem_st32(ta, ra);
           tmem_st32(ta + 32, rb);
-          // value columns q2*64 .. q2*64+63 -> MN block q2, 16-byte chunks 0..7
-          uint8_t* row = sS + q2 * dkp * 128 + a * 128;
+          if (!state_pass) {
+            put_f16(q2, ra, rb);
+          } else if (last) {
+            // end state of this segment (from zero) for the scan
+            float4* dst = reinterpret_cast<float4*>(T.seg_state + ((seq_slot + seg) * dkp + a) * kGlaTile) + q2 * 16;
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const uint32_t* r = e4 < 4 ? ra + 8 * e4 : rb + 8 * (e4 - 4);
-            st_shared_v4(smem_u32(row + ((e4 ^ (a & 7)) << 4)),
-                         pack_half2(__uint_as_float(r[0]), __uint_as_float(r[1])),
-                         pack_half2(__uint_as_float(r[2]), __uint_as_float(r[3])),
-                         pack_half2(__uint_as_float(r[4]), __uint_as_float(r[5])),
-                         pack_half2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+            for (int e = 0; e < 8; ++e) {
+              dst[e] = make_float4(__uint_as_float(ra[4 * e]), __uint_as_float(ra[4 * e + 1]),
+                                   __uint_as_float(ra[4 * e + 2]), __uint_as_float(ra[4 * e + 3]));
+              dst[8 + e] = make_float4(__uint_as_float(rb[4 * e]), __uint_as_float(rb[4 * e + 1]),
+                                       __uint_as_float(rb[4 * e + 2]), __uint_as_float(rb[4 * e + 3]));
+            }
           }
         }
+        decay *= f;
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bar[B_S_DONE]);
         f = f_next;
       }
+      if (state_pass) T.seg_decay[(seq_slot + seg) * dkp + a] = decay;
     }
   }
   tc_fence_before();
@@ -292,7 +366,40 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
   }
 }
 
+// Initial state of every segment: S'_init(s+1) = G_s * S'_init(s) + A_s with
+// S'_init(0) = 0, written over A_s. One thread per state element of a sequence.
+__global__ void gla_scan_kernel(const __grid_constant__ GlaParams p, int B) {
+  size_t gid = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  for (int t = 0; t < p.n_tasks; ++t) {
+    const GlaTask& T = p.task[t];
+    const size_t per_seq = static_cast<size_t>(T.dkp) * kGlaTile;
+    const size_t n = static_cast<size_t>(B) * T.heads * T.v_tiles * per_seq;
+    if (gid >= n) {
+      gid -= n;
+      continue;
+    }
+    const size_t sq = gid / per_seq, e = gid % per_seq;
+    const int a = static_cast<int>(e / kGlaTile);
+    float x = 0.f;
+    for (int s = 0; s + 1 < T.n_segs; ++s) {
+      float* slot = T.seg_state + (sq * T.n_segs + s) * per_seq + e;
+      x = T.seg_decay[(sq * T.n_segs + s) * T.dkp + a] * x + *slot;
+      *slot = x;
+    }
+    return;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_gla_scan(const GlaParams& p, int B, cudaStream_t st) {
+  size_t n = 0;
+  for (int t = 0; t < p.n_tasks; ++t)
+    n += static_cast<size_t>(B) * p.task[t].heads * p.task[t].v_tiles * p.task[t].dkp * kGlaTile;
+  if (n == 0) return cudaSuccess;
+  gla_scan_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p, B);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gla(const GlaParams& p, cudaStream_t st) {
   if (p.total_ctas <= 0) return cudaSuccess;

@@ -119,6 +119,7 @@ struct msgla_handle {
   msgla_config cfg;
   int device;
   int dkp, dvp, rp, n_scales, main_index, pool_rows;
+  int sm_count;  // streaming multiprocessors of the device
   int nzp, ldz;  // fusion-logit rows in the scale-1 packed weights (16) and z row stride
   Branch br[MSGLA_MAX_SCALES];
   __nv_bfloat16* Wfuse;
@@ -133,7 +134,8 @@ struct Region {
   size_t off = 0, bytes = 0;
 };
 struct BranchWs {
-  int rows, n_chunks, n_halves;
+  int rows, n_chunks, n_halves, seg_chunks, n_segs;
+  Region seg_state, seg_decay;
   Region Xp, q, k, qs, ks, v, g, gamma, mid, o, Y;
 };
 struct Workspace {
@@ -148,9 +150,34 @@ void add(Region& r, size_t& cur, size_t bytes) {
   cur = round_up(cur + bytes, 256);
 }
 
+// Chunks per sequence segment of the GLA kernel. One CTA runs each (sequence, head,
+// value tile); when those CTAs fill less than half of the GPU, long sequences are
+// cut into segments (state pass + scan + full pass) using the shortest segment
+// length that still fits all segments of all branches in one wave.
+int plan_seg_chunks(const msgla_handle* h, int B, int L) {
+  const int vt = h->dvp / kGlaTile;
+  long long base = 0;
+  int max_nch = 0;
+  for (int j = 0; j < h->n_scales; ++j) {
+    base += static_cast<long long>(B) * h->br[j].heads * vt;
+    max_nch = std::max(max_nch, ceil_div(ceil_div(L, h->br[j].scale), kGlaChunk));
+  }
+  const int no_split = std::max(max_nch, 1);
+  if (2 * base > h->sm_count) return no_split;
+  for (int seg = 2; seg < max_nch; ++seg) {
+    long long ctas = 0;
+    for (int j = 0; j < h->n_scales; ++j)
+      ctas += static_cast<long long>(B) * h->br[j].heads * vt *
+              ceil_div(ceil_div(ceil_div(L, h->br[j].scale), kGlaChunk), seg);
+    if (ctas <= h->sm_count) return seg;
+  }
+  return no_split;
+}
+
 Workspace layout(const msgla_handle* h, int B, int L) {
   Workspace ws;
   size_t cur = 0;
+  const int seg_chunks = plan_seg_chunks(h, B, L);
   const size_t BB = static_cast<size_t>(B);
   const int d = h->cfg.d;
   for (int j = 0; j < h->n_scales; ++j) {
@@ -159,6 +186,8 @@ Workspace layout(const msgla_handle* h, int B, int L) {
     w.rows = ceil_div(L, b.scale);
     w.n_chunks = ceil_div(w.rows, kGlaChunk);
     w.n_halves = ceil_div(w.rows, kChunk);
+    w.seg_chunks = std::max(1, std::min(seg_chunks, w.n_chunks));
+    w.n_segs = std::max(1, ceil_div(w.n_chunks, w.seg_chunks));
     const size_t n = BB * w.rows;
     if (b.scale > 1) add(w.Xp, cur, n * d * 2);
     add(w.q, cur, n * b.heads * h->dkp * 2);
@@ -171,6 +200,11 @@ Workspace layout(const msgla_handle* h, int B, int L) {
     add(w.mid, cur, BB * w.n_chunks * b.heads * h->dkp * 4);
     add(w.o, cur, n * b.heads * h->dvp * 2);
     if (j != h->main_index) add(w.Y, cur, n * d * 2);
+    if (w.n_segs > 1) {
+      const size_t seqs = BB * b.heads * (h->dvp / kGlaTile) * w.n_segs;
+      add(w.seg_state, cur, seqs * h->dkp * kGlaTile * 4);
+      add(w.seg_decay, cur, seqs * h->dkp * 4);
+    }
   }
   add(ws.w, cur, BB * L * h->n_scales * 4);
   if (h->main_index >= 0) add(ws.z, cur, BB * L * h->ldz * 4);
@@ -419,14 +453,14 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     CUDA_TRY(rec->mark(st));
   }
 
-  // 4. chunkwise GLA (grouped over branches; longest sequences first)
+  // 4. chunkwise GLA (grouped over branches; longest sequences first). Long
+  // sequences with few CTAs run as segments: a state pass over all but the last
+  // segment, a scan for the segments' initial states, then the full pass.
   static thread_local GlaParams lp;
   memset(&lp, 0, sizeof(lp));
   lp.err = h->d_err;
   lp.qk_scale = c.qk_scale;
-  lp.skip_arrival = h->test_skip_arrival;
-  h->test_skip_arrival = 0;
-  int ctas = 0;
+  bool segmented = false;
   for (int j = 0; j < ns; ++j) {
     const Branch& b = h->br[j];
     const BranchWs& bw = ws.br[j];
@@ -444,11 +478,43 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.dkp = h->dkp;
     t.dvp = h->dvp;
     t.v_tiles = h->dvp / kGlaTile;
-    t.cta_begin = ctas;
-    ctas += B * b.heads * t.v_tiles;
+    t.seg_chunks = bw.seg_chunks;
+    t.n_segs = bw.n_segs;
+    if (bw.n_segs > 1) {
+      t.seg_state = static_cast<float*>(at(bw.seg_state));
+      t.seg_decay = static_cast<float*>(at(bw.seg_decay));
+      segmented = true;
+    }
   }
   lp.n_tasks = ns;
+  if (segmented) {
+    static thread_local GlaParams sp;
+    sp = lp;
+    sp.mode = 1;
+    int nt = 0, sctas = 0;
+    for (int j = 0; j < ns; ++j) {
+      if (lp.task[j].n_segs < 2) continue;
+      sp.task[nt] = lp.task[j];
+      sp.task[nt].cta_begin = sctas;
+      sctas += B * lp.task[j].heads * lp.task[j].v_tiles * (lp.task[j].n_segs - 1);
+      ++nt;
+    }
+    sp.n_tasks = nt;
+    sp.total_ctas = sctas;
+    CUDA_TRY(launch_gla(sp, st));
+    CUDA_TRY(rec->mark(st));
+    CUDA_TRY(launch_gla_scan(sp, B, st));
+    CUDA_TRY(rec->mark(st));
+  }
+  int ctas = 0;
+  for (int j = 0; j < ns; ++j) {
+    lp.task[j].cta_begin = ctas;
+    ctas += B * lp.task[j].heads * lp.task[j].v_tiles * lp.task[j].n_segs;
+  }
   lp.total_ctas = ctas;
+  lp.mode = 0;
+  lp.skip_arrival = h->test_skip_arrival;
+  h->test_skip_arrival = 0;
   CUDA_TRY(launch_gla(lp, st));
   CUDA_TRY(rec->mark(st));
 
@@ -618,6 +684,7 @@ int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weight
   h->dvp = static_cast<int>(round_up(cfg->d_v, kGlaTile));
   h->rp = static_cast<int>(round_up(cfg->gate_rank, 16));
   h->main_index = -1;
+  h->sm_count = prop.multiProcessorCount;
   h->nzp = 16;
   h->ldz = cfg->n_scales <= 4 ? 4 : 8;
   int lcm = 1;
@@ -811,6 +878,40 @@ int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index,
   dims[0] = B;
   dims[1] = bw.rows;
   dims[2] = cols;
+  return MSGLA_OK;
+}
+
+int msgla_launch_plan(const msgla_handle* h, int B, int L, char* names, size_t len) {
+  if (!h || !names || len == 0) return fail(MSGLA_ERR_INVALID_ARG, "NULL argument");
+  int st = check_forward_args(h, B, L);
+  if (st) return st;
+  std::string out;
+  auto add_name = [&](const char* n) {
+    if (!out.empty()) out += ",";
+    out += n;
+  };
+  if (B > 0 && L > 0) {
+    if (h->main_index < 0 || h->pool_rows > 1) add_name("pool_fuse");
+    add_name("proj_gemm");
+    add_name("gate");
+    const Workspace ws = layout(h, B, L);
+    bool segmented = false;
+    for (int j = 0; j < h->n_scales; ++j) segmented |= ws.br[j].n_segs > 1;
+    if (segmented) {
+      add_name("gla_state");
+      add_name("gla_scan");
+    }
+    add_name("gla");
+    if (h->main_index >= 0) {
+      if (h->n_scales > 1) add_name("out_gemm_coarse");
+      add_name("out_gemm_fused");
+    } else {
+      add_name("out_gemm_coarse");
+      add_name("hold_fuse");
+    }
+  }
+  if (out.size() + 1 > len) return fail(MSGLA_ERR_INVALID_ARG, "names buffer of %zu bytes is too small", len);
+  memcpy(names, out.c_str(), out.size() + 1);
   return MSGLA_OK;
 }
 

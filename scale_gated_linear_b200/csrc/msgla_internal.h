@@ -66,7 +66,10 @@ struct alignas(64) GlaTask {
   const float* gamma;  // [B, n_chunks, h*dkp]: e^{b_last - m} per chunk
   const float* mid;    // [B, n_chunks, h*dkp]: e^{m}, m = b at the chunk's 64th row
   __half* o;           // [B, n_s, h*dvp]
-  int rows, n_chunks, heads, dkp, dvp, v_tiles, cta_begin, pad_;
+  // sequence segments (long sequences): chunks [s*seg_chunks, (s+1)*seg_chunks)
+  float* seg_state;    // [B, h, v_tiles, n_segs, dkp, 128]: end states, then initial states
+  float* seg_decay;    // [B, h, v_tiles, n_segs, dkp]: product of the state factors
+  int rows, n_chunks, heads, dkp, dvp, v_tiles, cta_begin, seg_chunks, n_segs, pad_;
 };
 
 struct GlaParams {
@@ -74,6 +77,7 @@ struct GlaParams {
   int n_tasks;
   int total_ctas;
   float qk_scale;
+  int mode;          // 0: full pass; 1: state pass over segments 0..n_segs-2
   int skip_arrival;  // failure-detection tests: CTA 0 omits one barrier arrival
   int* err;
 };
@@ -82,6 +86,8 @@ struct GlaParams {
 // (each returns the cudaError_t of the launch)
 cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st);
 cudaError_t launch_gla(const GlaParams& p, cudaStream_t st);
+// initial state of every segment from the state pass's end states (sequential over segments)
+cudaError_t launch_gla_scan(const GlaParams& p, int B, cudaStream_t st);
 
 // pooled rows (fp16) for scales > 1 and fusion weights w = softmax(W_fuse x + b)
 struct PoolParams {

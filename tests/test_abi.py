@@ -83,16 +83,6 @@ def test_null_arguments():
     lib.msgla_destroy(None)
 
 
-def test_launch_names_follow_the_documented_order():
-    m = MSGLA.__new__(MSGLA)
-    m.scales = (1, 2, 4)
-    assert m.launch_names() == ["pool_fuse", "proj_gemm", "gate", "gla", "out_gemm_coarse", "out_gemm_fused"]
-    m.scales = (1,)
-    assert m.launch_names() == ["proj_gemm", "gate", "gla", "out_gemm_fused"]
-    m.scales = (2, 4)
-    assert m.launch_names()[-2:] == ["out_gemm_coarse", "hold_fuse"]
-
-
 def test_product_does_not_use_the_oracle():
     pkg = os.path.join(ROOT, "scale_gated_linear_b200")
     for dirpath, _, files in os.walk(pkg):

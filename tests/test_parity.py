@@ -224,10 +224,12 @@ def test_forward_profiled_records_every_launch():
     layer = _layer(SMALL, inp)
     X = inp["X"].cuda()
     ws = layer.alloc_workspace(*X.shape[:2])
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(layer.launch_names()) + 1)]
+    names = layer.launch_names(*X.shape[:2])
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
     n = layer.forward_profiled(X, torch.empty_like(X), ws, ev)
     torch.cuda.synchronize()
-    assert n == len(layer.launch_names())
+    assert n == len(names)
+    assert names == ["pool_fuse", "proj_gemm", "gate", "gla", "out_gemm_coarse", "out_gemm_fused"]
     assert all(ev[i].elapsed_time(ev[i + 1]) >= 0 for i in range(n))
     layer.close()
 
@@ -274,4 +276,28 @@ def test_wide_8k_full_launch_prefix(name):
     got, layer, _ = run_gpu(w, inp)
     assert_parity(got[0:1, :1024], oracle_forward(w, inp, rows=1024, batch=slice(0, 1)))
     assert np.isfinite(got).all()
+    layer.close()
+
+
+# ----------------------------------------------------------------- long sequences
+@needs_gpu
+def test_segment_plan():
+    w = wl.WORKLOADS["msgla_340m"]
+    inp = gpu_inputs(w, B=1, L=64)
+    layer = _layer(w, inp)
+    assert "gla_state" not in layer.launch_names(8, 2048)   # 128 CTAs: one pass
+    plan = layer.launch_names(1, 4096)                       # 16 CTAs: segmented
+    assert plan[plan.index("gla_state"):plan.index("gla") + 1] == ["gla_state", "gla_scan", "gla"]
+    layer.close()
+
+
+@needs_gpu
+def test_segmented_long_sequence_matches_oracle():
+    """One 4096-token sequence of the 340M-shaped layer: the GLA kernel cuts each
+    branch into segments (state pass, scan, full pass from carried states)."""
+    w = wl.WORKLOADS["msgla_340m"]
+    inp = gpu_inputs(w, B=1, L=4096)
+    got, layer, _ = run_gpu(w, inp)
+    assert "gla_state" in layer.launch_names(1, 4096)
+    assert_parity(got, oracle_forward(w, inp))
     layer.close()
