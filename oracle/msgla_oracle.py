@@ -14,8 +14,11 @@ summarised in the MS-GLA reading notes (arXiv 2609.35664v1):
   (0,1)^{d_k} comes from a low-rank projection of the hidden state followed by
   a sigmoid-type map.
 * Sec. 3.1, Eq. (8): non-overlapping mean pooling over s adjacent rows, pooled
-  length ceil(L/s), the incomplete tail block averaged over its valid rows
-  (no padding mask: every row inside L is valid).
+  length ceil(L/s), each block averaged over its valid rows (token mask M, 1 =
+  valid, 0 = padding; rows past L count as padding; the denominator is clamped
+  to at least 1, so an all-padding block pools to zero). Without a mask every
+  row inside L is valid. The formula is applied at every scale, s = 1 included,
+  where it zeroes padded rows.
 * Sec. 3.2, Eq. (9): the H heads are split over the scales (sum_s h_s = H);
   each branch has its own q/k/v/gate/output projections.
 * Sec. 3.3: causal hold -- each coarse output is repeated s times and shifted
@@ -33,7 +36,9 @@ notes of this repository):
 * o_t = qk_scale * q_t S_t with qk_scale = 1 by default (the notes' equation
   has no scale);
 * no per-branch normalisation and no output gate (the notes list a
-  per-branch "normalisation" without defining it).
+  per-branch "normalisation" without defining it);
+* the mask enters the pooling only: the fusion weights of Eq. (10) read the
+  unpooled row x_t whatever its mask.
 
 Every step is written token by token or row by row; numpy's matmul is used as
 a library primitive for the per-row projections only.
@@ -41,7 +46,8 @@ a library primitive for the per-row projections only.
 Parity pins (tests/test_oracle.py): brute-force quadratic form of the GLA
 recurrence, alpha = 1 reducing to causal (Q K^T) V, the single-scale layer
 reducing to plain GLA + W_o, the constant-input geometric closed form, the
-worked s = 4 hold table and pooling example of Sec. 3.1/3.3, causality,
+worked s = 4 hold table and pooling example of Sec. 3.1/3.3, a masked s = 4
+pooling example with an all-padding block, causality,
 half-life, the 11/16 update count and the simplex property of the fusion
 weights.
 """
@@ -51,24 +57,29 @@ import numpy as np
 
 
 # ---------------------------------------------------------------------------
-# Sec. 3.1, Eq. (8): non-overlapping mean pooling (mask M = 1 inside L)
+# Sec. 3.1, Eq. (8): non-overlapping mean pooling with the valid-token mask M
 # ---------------------------------------------------------------------------
-def pool(X: np.ndarray, s: int) -> np.ndarray:
-    """Mean of each block of s consecutive rows; X is [L, d] -> [ceil(L/s), d].
+def pool(X: np.ndarray, s: int, M: np.ndarray | None = None) -> np.ndarray:
+    """Eq. (8): block i of s consecutive rows of X [L, d] -> [ceil(L/s), d].
 
-    The incomplete tail block (L not divisible by s) is the mean of its valid
-    rows: Eq. (8) with M = 1 for rows inside L and 0 for the right padding,
-    denominator max(1, sum M).
+    X_i = sum_j X_{is+j} M_{is+j} / max(1, sum_j M_{is+j}) over the rows j of the
+    block that lie inside L (right padding past L counts as M = 0). Without a mask,
+    M = 1 for every row inside L: the incomplete tail block is the mean of its
+    valid rows.
     """
     L = X.shape[0]
+    if M is None:
+        M = np.ones(L)
     n = -(-L // s)
     out = np.zeros((n, X.shape[1]), dtype=np.float64)
     for i in range(n):
         rows = [i * s + j for j in range(s) if i * s + j < L]
         acc = np.zeros(X.shape[1], dtype=np.float64)
+        cnt = 0.0
         for r in rows:
-            acc += X[r]
-        out[i] = acc / max(1, len(rows))
+            acc += X[r] * M[r]
+            cnt += M[r]
+        out[i] = acc / max(1.0, cnt)
     return out
 
 
@@ -148,8 +159,12 @@ def fusion_weights(X: np.ndarray, Wfuse: np.ndarray, bfuse: np.ndarray) -> np.nd
 # ---------------------------------------------------------------------------
 def layer_forward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: int,
                   gate_normalizer: float = 16.0, qk_scale: float = 1.0,
-                  intermediates: bool = False, counter: list | None = None):
+                  intermediates: bool = False, counter: list | None = None,
+                  mask: np.ndarray | None = None):
     """MS-GLA layer forward for X [B, L, d] (float64).
+
+    ``mask`` [B, L] (1 = valid token, 0 = padding) enters only the pooling of
+    Eq. (8); without it every row inside L is valid.
 
     ``weights`` holds ``branches`` (per scale: Wq, Wk, Wv, Wg1, Wg2, bg, Wo)
     and ``Wfuse``, ``bfuse``. Returns O [B, L, d]; with ``intermediates`` also a
@@ -167,7 +182,7 @@ def layer_forward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: in
         inter["w"].append(w)
         for j, (s, h) in enumerate(zip(scales, heads)):
             br = weights["branches"][j]
-            Xp = pool(X[b], s)
+            Xp = pool(X[b], s, None if mask is None else np.asarray(mask[b], dtype=np.float64))
             q, k, v, la = branch_projections(Xp, br, gate_normalizer)
             o = np.zeros((Xp.shape[0], h * d_v), dtype=np.float64)
             for hh in range(h):

@@ -150,6 +150,54 @@ def test_pool_tail_block():
     check_pool_tail()
 
 
+def check_pool_mask():
+    tab = _read_table("pool_mask_s4.txt")
+    M = np.array([0, 1, 1, 0, 0, 0, 0, 0], dtype=float)
+    P = om.pool(np.eye(8), 4, M)
+    for row in tab:
+        np.testing.assert_allclose(P[int(row[0])], row[1:], rtol=0, atol=1e-15)
+
+
+def test_pool_mask_example():
+    check_pool_mask()
+
+
+def test_all_ones_mask_is_the_unmasked_layer():
+    rng = np.random.default_rng(11)
+    d, dk, dv, L = 6, 3, 2, 14
+    W = _rand_weights(rng, d, (1, 2, 4), (2, 1, 1), dk, dv)
+    X = rng.normal(size=(2, L, d))
+    np.testing.assert_array_equal(om.layer_forward(X, W, (1, 2, 4), (2, 1, 1), dk, dv, mask=np.ones((2, L))),
+                                  om.layer_forward(X, W, (1, 2, 4), (2, 1, 1), dk, dv))
+
+
+def test_masked_rows_do_not_reach_pooled_rows():
+    """Changing X at a masked position changes no pooled row (Eq. (8) weights it by 0)."""
+    rng = np.random.default_rng(12)
+    X = rng.normal(size=(12, 5))
+    M = np.ones(12); M[[0, 1, 5, 11]] = 0
+    X2 = X.copy(); X2[[0, 1, 5, 11]] += 7.0
+    for s in (1, 2, 4):
+        np.testing.assert_array_equal(om.pool(X, s, M), om.pool(X2, s, M))
+
+
+def test_mask_at_scale_one_zeroes_padded_rows():
+    """Eq. (8) at s = 1: x_t M_t / max(1, M_t) is x_t when valid and 0 when padded."""
+    rng = np.random.default_rng(14)
+    X = rng.normal(size=(6, 4))
+    M = np.array([1, 0, 1, 1, 0, 1], dtype=float)
+    np.testing.assert_array_equal(om.pool(X, 1, M), X * M[:, None])
+
+
+def test_left_padding_changes_only_mixed_blocks():
+    rng = np.random.default_rng(13)
+    X = rng.normal(size=(8, 3))
+    M = np.array([0, 0, 0, 1, 1, 1, 1, 1], dtype=float)
+    P = om.pool(X, 4, M)
+    np.testing.assert_allclose(P[0], X[3], rtol=1e-15)
+    np.testing.assert_allclose(P[1], X[4:8].mean(0), rtol=1e-15)
+
+
 def test_update_ratio_11_16():
     num, den = _read_table("update_ratio.txt")[0]
     L = 256
@@ -353,10 +401,20 @@ def _mutant_gla_decay_after_write(q, k, v, log_alpha, qk_scale=1.0, counter=None
     return o
 
 
-def _mutant_pool_divide_by_s(X, s):
+def _mutant_pool_divide_by_s(X, s, M=None):
     L = X.shape[0]; n = -(-L // s)
     Xp = np.zeros((n * s, X.shape[1])); Xp[:L] = X
     return Xp.reshape(n, s, -1).sum(1) / s
+
+
+def _mutant_pool_mask_divide_by_block(X, s, M=None):
+    L = X.shape[0]; n = -(-L // s)
+    M = np.ones(L) if M is None else M
+    out = np.zeros((n, X.shape[1]))
+    for i in range(n):
+        rows = [i * s + j for j in range(s) if i * s + j < L]
+        out[i] = sum(X[r] * M[r] for r in rows) / len(rows)   # ignores the mask in the denominator
+    return out
 
 
 def _mutant_softmax_wrong_axis(X, Wfuse, bfuse):
@@ -364,7 +422,7 @@ def _mutant_softmax_wrong_axis(X, Wfuse, bfuse):
     return np.exp(z) / np.exp(z).sum(axis=0, keepdims=True)
 
 
-PINS = [check_hold_table, check_pool_example, check_pool_tail, check_gla_bruteforce,
+PINS = [check_hold_table, check_pool_example, check_pool_tail, check_pool_mask, check_gla_bruteforce,
         check_layer_bruteforce, check_constant_input_closed_form]
 
 
@@ -374,6 +432,7 @@ PINS = [check_hold_table, check_pool_example, check_pool_tail, check_gla_brutefo
     ("gla_recurrent", _mutant_gla_read_before_write),
     ("gla_recurrent", _mutant_gla_decay_after_write),
     ("pool", _mutant_pool_divide_by_s),
+    ("pool", _mutant_pool_mask_divide_by_block),
     ("fusion_weights", _mutant_softmax_wrong_axis),
 ])
 def test_planted_mistake_is_caught(monkeypatch, name, mutant):
