@@ -113,6 +113,20 @@ int msgla_workspace_size(const msgla_handle* h, int B, int L, size_t* bytes);
 int msgla_forward(msgla_handle* h, const void* X, int B, int L, void* O,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* msgla_forward with a valid-token mask M in the pooling (Sec. 3.1, Eq. (8)):
+ *   Xbar^(s)_i = sum_j x_{is+j} M_{is+j} / max(1, sum_j M_{is+j}),
+ * the sums over the rows of block i that lie inside L. The formula applies at
+ * every scale, so at s = 1 a padded row enters its branch as a zero row; an
+ * all-padding block pools to zero. The fusion weights (Eq. (10)) read the
+ * unpooled x_t whatever its mask.
+ *   M  device uint8 [B, L], row-major; nonzero = valid token, 0 = padding; not
+ *      written. NULL gives msgla_forward's result.
+ *   X, O, workspace, stream and errors as for msgla_forward (same workspace size).
+ * Padding anywhere (left, right or interior) is accepted. Outputs at padded
+ * positions are computed like any other (they are not zeroed). */
+int msgla_forward_masked(msgla_handle* h, const void* X, const void* M, int B, int L,
+                         void* O, void* workspace, size_t workspace_bytes, void* stream);
+
 /* msgla_forward without a caller workspace and without any device allocation:
  * for callers that cannot call cudaMalloc (or their framework's allocator) at the
  * point where they run the layer -- for instance code inside a fixed memory arena

@@ -86,12 +86,17 @@ class MSGLA:
         return torch.empty(max(n, 1), dtype=torch.uint8, device=torch.device("cuda", self.device))
 
     # ------------------------------------------------------------- forward
-    def forward(self, X, out=None, workspace=None, stream=None):
+    def forward(self, X, out=None, workspace=None, stream=None, mask=None):
         """O = MS-GLA(X) for cuda bf16 X [B, L, d]; asynchronous on `stream`
-        (default: torch's current stream)."""
+        (default: torch's current stream). ``mask``: optional cuda [B, L] tensor
+        of valid tokens (bool or uint8, nonzero = valid) for the pooling of
+        Eq. (8)."""
         import torch
         B, L, d = X.shape
         assert d == self.d and X.dtype == torch.bfloat16 and X.is_cuda and X.is_contiguous()
+        if mask is not None:
+            assert mask.shape == (B, L) and mask.is_cuda and mask.is_contiguous()
+            assert mask.dtype in (torch.bool, torch.uint8)
         if out is None:
             out = torch.empty_like(X)
         if workspace is None:
@@ -101,8 +106,13 @@ class MSGLA:
             workspace = self._ws
         if stream is None:
             stream = torch.cuda.current_stream(X.device)
-        _lib.check(self._lib.msgla_forward(self._h, X.data_ptr(), B, L, out.data_ptr(), workspace.data_ptr(),
-                                           workspace.numel(), ctypes.c_void_p(stream.cuda_stream)))
+        if mask is None:
+            _lib.check(self._lib.msgla_forward(self._h, X.data_ptr(), B, L, out.data_ptr(), workspace.data_ptr(),
+                                               workspace.numel(), ctypes.c_void_p(stream.cuda_stream)))
+        else:
+            _lib.check(self._lib.msgla_forward_masked(self._h, X.data_ptr(), mask.data_ptr(), B, L, out.data_ptr(),
+                                                      workspace.data_ptr(), workspace.numel(),
+                                                      ctypes.c_void_p(stream.cuda_stream)))
         return out
 
     __call__ = forward

@@ -58,12 +58,16 @@ __global__ void __launch_bounds__(kPoolThreads) pool_fuse_kernel(const PoolParam
       }
     }
     float acc[kMaxScales][8];
+    int nvalid[kMaxScales];
 #pragma unroll
-    for (int j = 0; j < kMaxScales; ++j)
+    for (int j = 0; j < kMaxScales; ++j) {
+      nvalid[j] = 0;
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+    }
     for (int r = 0; r < nrows; ++r) {
       const int t = row0 + r;
+      const bool keep = !p.M || p.M[static_cast<size_t>(b) * p.L + t];
       float x[8];
       if (active) {
         uint4 u = __ldg(reinterpret_cast<const uint4*>(Xb + static_cast<size_t>(t) * p.d) + cg);
@@ -83,13 +87,16 @@ __global__ void __launch_bounds__(kPoolThreads) pool_fuse_kernel(const PoolParam
         if (lane == 0) atomicAdd(&logit[r * ns + j], part);
         const int s = p.scales[j];
         if (s > 1) {
+          if (keep) {
+            ++nvalid[j];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[j][e] += x[e];
+            for (int e = 0; e < 8; ++e) acc[j][e] += x[e];
+          }
           const bool block_end = ((t + 1) % s == 0) || (t == p.L - 1);
           if (block_end) {
             if (active) {
               const int i = t / s;
-              const float inv = 1.f / static_cast<float>(t - i * s + 1);
+              const float inv = 1.f / static_cast<float>(max(1, nvalid[j]));
               uint4 o;
               uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
               bool bad = false;
@@ -103,6 +110,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_fuse_kernel(const PoolParam
               const int ns_rows = (p.L + s - 1) / s;
               reinterpret_cast<uint4*>(p.Xp[j] + (static_cast<size_t>(b) * ns_rows + i) * p.d)[cg] = o;
             }
+            nvalid[j] = 0;
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
           }
@@ -149,6 +157,12 @@ __global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p)
   const int row0 = static_cast<int>(gw % blocks_per_seq) * P;
   const int nrows = min(P, p.L - row0);
   const __nv_bfloat16* Xb = p.X + (static_cast<size_t>(b) * p.L + row0) * p.d;
+  // rows of this block that enter the pooled means (bit r = row0 + r)
+  uint32_t vm = (1u << nrows) - 1u;
+  if (p.M)
+#pragma unroll
+    for (int r = 0; r < P; ++r)
+      if (r < nrows && !p.M[static_cast<size_t>(b) * p.L + row0 + r]) vm &= ~(1u << r);
   float part[P][NS];
 #pragma unroll
   for (int r = 0; r < P; ++r)
@@ -193,10 +207,10 @@ __global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p)
           for (int e = 0; e < 8; ++e) m[e] = 0.f;
 #pragma unroll
           for (int r = 0; r < P; ++r)
-            if (r >= i0 && r < i0 + cnt)
+            if (r >= i0 && r < i0 + cnt && ((vm >> r) & 1u))
 #pragma unroll
               for (int e = 0; e < 8; ++e) m[e] += x[r][e];
-          const float inv = 1.f / static_cast<float>(cnt);
+          const float inv = 1.f / static_cast<float>(max(1, __popc((vm >> i0) & ((1u << cnt) - 1u))));
           uint4 o;
           uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
           bool bad = false;
@@ -252,11 +266,17 @@ __global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
   const int row0 = blk * P;
   const int nrows = min(P, p.L - row0);
   const __nv_bfloat16* Xb = p.X + (static_cast<size_t>(b) * p.L + row0) * p.d;
+  // rows of this block that enter the means (bit r = row0 + r); padded rows are not read
+  uint32_t vm = (1u << nrows) - 1u;
+  if (p.M)
+#pragma unroll
+    for (int r = 0; r < P; ++r)
+      if (r < nrows && !p.M[static_cast<size_t>(b) * p.L + row0 + r]) vm &= ~(1u << r);
   uint4 raw[P];
 #pragma unroll
   for (int r = 0; r < P; ++r)
-    raw[r] = r < nrows ? __ldg(reinterpret_cast<const uint4*>(Xb + static_cast<size_t>(r) * p.d) + cg)
-                       : make_uint4(0, 0, 0, 0);
+    raw[r] = ((vm >> r) & 1u) ? __ldg(reinterpret_cast<const uint4*>(Xb + static_cast<size_t>(r) * p.d) + cg)
+                              : make_uint4(0, 0, 0, 0);
   float x[P][8];
 #pragma unroll
   for (int r = 0; r < P; ++r) bf16x8_to_f32(raw[r], x[r]);
@@ -295,7 +315,9 @@ __global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
         if (p.scales[j] != width) continue;
 #pragma unroll
         for (int i = 0; i < P / 2; ++i)
-          if (i < n / 2) put(j, width, i * width, lv[i], 1.f / static_cast<float>(width));
+          if (i < n / 2)
+            put(j, width, i * width, lv[i],
+                1.f / static_cast<float>(max(1, __popc((vm >> (i * width)) & ((1u << width) - 1u)))));
       }
     }
   }
@@ -312,7 +334,7 @@ __global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
         if (r >= i0 && r < i0 + cnt)
 #pragma unroll
           for (int e = 0; e < 8; ++e) m[e] += x[r][e];
-      put(j, s, i0, m, 1.f / static_cast<float>(cnt));
+      put(j, s, i0, m, 1.f / static_cast<float>(max(1, __popc((vm >> i0) & ((1u << cnt) - 1u)))));
     }
   }
   if (bad) atomicCAS(p.err, 0, kDevRange);
@@ -614,16 +636,21 @@ cudaError_t launch_pool_only(const PoolParams& p, cudaStream_t st) {
 
 cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st) {
   if (p.B * p.L == 0) return cudaSuccess;
+  // block_rows carries the least common multiple of the coarse scales (1 if none);
+  // the row-block kernels take P rows at a time, so every scale must divide P
+  const int lcm = p.block_rows;
   if (!p.want_w) {
-    if (p.block_rows <= 2) return launch_pool_only<2>(p, st);
-    if (p.block_rows <= 4) return launch_pool_only<4>(p, st);
-    if (p.block_rows <= 8) return launch_pool_only<8>(p, st);
+    if (2 % lcm == 0) return launch_pool_only<2>(p, st);
+    if (4 % lcm == 0) return launch_pool_only<4>(p, st);
+    if (6 % lcm == 0) return launch_pool_only<6>(p, st);
+    if (8 % lcm == 0) return launch_pool_only<8>(p, st);
   }
-  // block_rows carries the least common multiple of the coarse scales (1 if none)
   if (p.n_scales * p.d * 4 <= 160 * 1024) {
-    if (p.block_rows <= 4)
+    if (4 % lcm == 0)
       return p.n_scales <= 4 ? launch_pool_rows<4, 4, 4>(p, st) : launch_pool_rows<4, 4, 8>(p, st);
-    if (p.block_rows == 8)
+    if (6 % lcm == 0)
+      return p.n_scales <= 4 ? launch_pool_rows<6, 2, 4>(p, st) : launch_pool_rows<6, 2, 8>(p, st);
+    if (8 % lcm == 0)
       return p.n_scales <= 4 ? launch_pool_rows<8, 2, 4>(p, st) : launch_pool_rows<8, 2, 8>(p, st);
   }
   PoolParams q = p;

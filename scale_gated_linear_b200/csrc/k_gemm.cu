@@ -194,6 +194,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
     return;
   }
   const float wmain = (T.epi == kEpiFuse && valid) ? wts[T.main_index] : 0.f;
+  // Eq. (8) at scale 1 zeroes a padded row; the projections have no bias, so its
+  // q | k | v | g columns are zero (the fusion logits read x_t and are kept)
+  const bool padded = T.epi == kEpiProj && T.mask && valid && !T.mask[grow];
+  const int n_zeroed = T.nq + T.nk + T.nv + T.ng;
   for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
     uint32_t v[32];
     tmem_ld32(tmem_addr(tacc, quad * 32, c0), v);
@@ -201,6 +205,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
     if (!valid) continue;
     const int col = tc.n0 + c0;
     if (T.epi == kEpiProj) {
+      if (padded)
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col + j < n_zeroed) v[j] = 0u;
       if (col < T.nq) {
         cvt_store_f16x32(T.q + grow * T.nq + col, v);
       } else if (col < T.nq + T.nk) {

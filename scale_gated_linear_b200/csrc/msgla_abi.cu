@@ -341,7 +341,7 @@ struct Recorder {
 };
 
 int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* wsp, size_t ws_bytes,
-                 cudaStream_t st, Recorder* rec = nullptr) {
+                 cudaStream_t st, Recorder* rec = nullptr, const uint8_t* M = nullptr) {
   Recorder none;
   if (!rec) rec = &none;
   if (rec->events) {
@@ -361,6 +361,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   // 1. pooling + fusion weights
   PoolParams pp{};
   pp.X = static_cast<const __nv_bfloat16*>(X);
+  pp.M = M;
   pp.B = B;
   pp.L = L;
   pp.d = d;
@@ -413,6 +414,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.k = static_cast<__half*>(at(bw.k));
     t.v = static_cast<__half*>(at(bw.v));
     t.g = static_cast<float*>(at(bw.g));
+    t.mask = bf ? M : nullptr;
     tiles += B * t.m_tiles * t.n_tiles;
   }
   gp.n_tasks = ns;
@@ -747,6 +749,26 @@ int msgla_forward(msgla_handle* h, const void* X, int B, int L, void* O, void* w
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
   return forward_impl(h, X, B, L, O, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int msgla_forward_masked(msgla_handle* h, const void* X, const void* M, int B, int L, void* O, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  int st = check_forward_args(h, B, L);
+  if (st) return st;
+  if (B == 0 || L == 0) return MSGLA_OK;
+  if (!X || !O) return fail(MSGLA_ERR_INVALID_ARG, "X or O is NULL");
+  if (reinterpret_cast<uintptr_t>(X) % 16 || reinterpret_cast<uintptr_t>(O) % 16)
+    return fail(MSGLA_ERR_INVALID_ARG, "X and O must be 16-byte aligned");
+  const size_t nbytes = static_cast<size_t>(B) * L * h->cfg.d * 2;
+  const uint8_t* x0 = static_cast<const uint8_t*>(X);
+  const uint8_t* o0 = static_cast<const uint8_t*>(O);
+  if (x0 < o0 + nbytes && o0 < x0 + nbytes) return fail(MSGLA_ERR_INVALID_ARG, "O overlaps X");
+  const uint8_t* m0 = static_cast<const uint8_t*>(M);
+  if (m0 && m0 < o0 + nbytes && o0 < m0 + static_cast<size_t>(B) * L)
+    return fail(MSGLA_ERR_INVALID_ARG, "O overlaps M");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
+  return forward_impl(h, X, B, L, O, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), nullptr, m0);
 }
 
 int msgla_forward_noalloc(msgla_handle* h, const void* X, int B, int L, void* O, void* stream) {

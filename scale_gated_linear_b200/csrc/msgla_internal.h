@@ -37,6 +37,8 @@ struct alignas(64) GemmTask {
   __half* v;
   float* g;
   float* z;  // [B, rows, ldz] fp32
+  const uint8_t* mask;  // [B, rows] valid-token mask of the scale-1 branch or null: padded rows
+                        // get zero q | k | v | g (the logits z stay: Eq. (10) reads x_t)
   // kEpiStoreF16
   __half* y;
   // kEpiFuse (rows == L, the branch with scale 1)
@@ -92,6 +94,7 @@ cudaError_t launch_gla_scan(const GlaParams& p, int B, cudaStream_t st);
 // pooled rows (fp16) for scales > 1 and fusion weights w = softmax(W_fuse x + b)
 struct PoolParams {
   const __nv_bfloat16* X;  // [B, L, d]
+  const uint8_t* M;        // [B, L] valid-token mask (nonzero = valid) or null (all valid)
   int B, L, d, n_scales;
   int scales[kMaxScales];
   __half* Xp[kMaxScales];  // [B, n_s, d] or null (scale 1)

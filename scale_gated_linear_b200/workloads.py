@@ -20,6 +20,9 @@ Recipe (all draws from one ``torch.Generator`` seeded per workload):
   * the long-sequence workload skews the forget gates toward long memory:
     b_g = +3, W_g1 ~ N(0, 1/d), W_g2 ~ N(0, 1/r), so that the gate
     pre-activation is about N(3, 1) for RMS-normalised rows.
+  * valid-token masks (``make_mask``, uint8 [B, L], 1 = valid): left or right
+    padding of a per-sequence length drawn uniformly from [0, L/2] (a batch of
+    unequal-length prompts), independent Bernoulli(0.8) tokens, or all padding.
 """
 from __future__ import annotations
 
@@ -129,6 +132,26 @@ def make_inputs(w: Workload, B: Optional[int] = None, L: Optional[int] = None,
     if w.rms_norm_x:
         X = X / X.pow(2).mean(-1, keepdim=True).sqrt()
     return {"X": lo(X), "branches": branches, "Wfuse": Wfuse, "bfuse": bfuse}
+
+
+MASK_KINDS = ("left", "right", "random", "none", "all_padding")
+
+
+def make_mask(B: int, L: int, kind: str, seed: int = 0) -> torch.Tensor:
+    """Valid-token mask uint8 [B, L] (1 = valid, 0 = padding) of the given kind."""
+    g = torch.Generator().manual_seed(seed)
+    if kind == "none":
+        return torch.ones(B, L, dtype=torch.uint8)
+    if kind == "all_padding":
+        return torch.zeros(B, L, dtype=torch.uint8)
+    if kind == "random":
+        return (torch.rand(B, L, generator=g) < 0.8).to(torch.uint8)
+    if kind not in ("left", "right"):
+        raise ValueError(f"unknown mask kind {kind!r}")
+    pad = torch.randint(0, L // 2 + 1, (B,), generator=g)
+    pos = torch.arange(L)[None, :]
+    valid = pos >= pad[:, None] if kind == "left" else pos < (L - pad)[:, None]
+    return valid.to(torch.uint8)
 
 
 def to_float64(inp: dict) -> dict:

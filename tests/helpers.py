@@ -24,11 +24,13 @@ def gpu_inputs(w: wl.Workload, B=None, L=None, seed=None):
     return inp
 
 
-def oracle_forward(w: wl.Workload, inp: dict, rows=None, intermediates=False, batch=None):
+def oracle_forward(w: wl.Workload, inp: dict, rows=None, intermediates=False, batch=None, mask=None):
     import oracle
     f = wl.to_float64(inp)
     X = f["X"] if batch is None else f["X"][batch]
     if rows is not None:
         X = X[:, :rows]
+    if mask is not None:
+        mask = np.asarray(mask, dtype=np.float64)
     return oracle.layer_forward(X, f, w.scales, w.heads, w.d_k, w.d_v,
-                                gate_normalizer=w.gate_normalizer, intermediates=intermediates)
+                                gate_normalizer=w.gate_normalizer, intermediates=intermediates, mask=mask)

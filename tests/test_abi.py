@@ -78,6 +78,7 @@ def test_null_arguments():
     assert lib.msgla_create(None, ctypes.byref(_cfg()), None, 0) == -1
     assert lib.msgla_workspace_size(None, 1, 1, ctypes.byref(n)) == -1
     assert lib.msgla_forward(None, None, 1, 1, None, None, 0, None) == -1
+    assert lib.msgla_forward_masked(None, None, None, 1, 1, None, None, 0, None) == -1
     assert lib.msgla_forward_host(None, None, 1, 1, None, None, 0, None) == -1
     assert lib.msgla_sync_status(None) == -1
     lib.msgla_destroy(None)

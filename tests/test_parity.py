@@ -125,6 +125,19 @@ def test_wide_scale_set_small():
 
 
 @needs_gpu
+@pytest.mark.parametrize("scales,heads", [((1, 3), (2, 1)), ((2, 3), (1, 1)), ((1, 2, 6), (1, 1, 1)),
+                                          ((1, 5), (1, 1)), ((2, 5), (1, 1)), ((3,), (2,))])
+def test_scale_sets_beyond_powers_of_two(scales, heads):
+    """Scales that do not divide 4 or 8: the pooling picks 6-row blocks or its
+    generic kernel; the hold index floor((t+1)/s) - 1 at odd s."""
+    w = SMALL.replace(name="odd", scales=scales, heads=heads)
+    inp = gpu_inputs(w, B=2, L=211)
+    got, layer, _ = run_gpu(w, inp)
+    assert_parity(got, oracle_forward(w, inp))
+    layer.close()
+
+
+@needs_gpu
 @pytest.mark.parametrize("dk,dv", [(16, 16), (100, 200), (128, 384)])
 def test_padded_head_widths(dk, dv):
     w = SMALL.replace(name=f"pad{dk}x{dv}", d_k=dk, d_v=dv)
