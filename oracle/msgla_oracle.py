@@ -35,8 +35,10 @@ notes of this repository):
   is a row gather);
 * o_t = qk_scale * q_t S_t with qk_scale = 1 by default (the notes' equation
   has no scale);
-* no per-branch normalisation and no output gate (the notes list a
-  per-branch "normalisation" without defining it);
+* per-branch normalisation (Sec. 3.2 lists one per branch without defining
+  it): off by default; when asked for, an RMS normalisation of each head's GLA
+  output row before the output projection, o_h / sqrt(mean(o_h^2) + eps) times a
+  per-channel weight (``head_rmsnorm``). No output gate;
 * the mask enters the pooling only: the fusion weights of Eq. (10) read the
   unpooled row x_t whatever its mask.
 
@@ -47,7 +49,8 @@ Parity pins (tests/test_oracle.py): brute-force quadratic form of the GLA
 recurrence, alpha = 1 reducing to causal (Q K^T) V, the single-scale layer
 reducing to plain GLA + W_o, the constant-input geometric closed form, the
 worked s = 4 hold table and pooling example of Sec. 3.1/3.3, a masked s = 4
-pooling example with an all-padding block, causality,
+pooling example with an all-padding block, unit RMS per head and invariance to
+the value scale of the optional head normalisation, causality,
 half-life, the 11/16 update count and the simplex property of the fusion
 weights.
 """
@@ -126,6 +129,20 @@ def gla_recurrent(q: np.ndarray, k: np.ndarray, v: np.ndarray, log_alpha: np.nda
 
 
 # ---------------------------------------------------------------------------
+# Sec. 3.2: per-branch normalisation (optional, read as a per-head RMS norm)
+# ---------------------------------------------------------------------------
+def head_rmsnorm(o: np.ndarray, weight: np.ndarray, eps: float) -> np.ndarray:
+    """One head's output rows o [n, d_v]: each row divided by its root mean
+    square over the head's d_v channels (with eps inside the root), then
+    multiplied channel-wise by ``weight`` [d_v]."""
+    out = np.zeros_like(o)
+    for t in range(o.shape[0]):
+        ms = float(np.dot(o[t], o[t])) / o.shape[1]
+        out[t] = o[t] / np.sqrt(ms + eps) * weight
+    return out
+
+
+# ---------------------------------------------------------------------------
 # Sec. 3.3: causal hold (repeat s times, shift right by s-1, zero fill)
 # ---------------------------------------------------------------------------
 def hold_index(t: int, s: int) -> int:
@@ -160,11 +177,13 @@ def fusion_weights(X: np.ndarray, Wfuse: np.ndarray, bfuse: np.ndarray) -> np.nd
 def layer_forward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: int,
                   gate_normalizer: float = 16.0, qk_scale: float = 1.0,
                   intermediates: bool = False, counter: list | None = None,
-                  mask: np.ndarray | None = None):
+                  mask: np.ndarray | None = None, head_norm_eps: float | None = None):
     """MS-GLA layer forward for X [B, L, d] (float64).
 
     ``mask`` [B, L] (1 = valid token, 0 = padding) enters only the pooling of
-    Eq. (8); without it every row inside L is valid.
+    Eq. (8); without it every row inside L is valid. ``head_norm_eps`` (None =
+    off) turns on the per-head RMS normalisation of the GLA output with the
+    branch's ``norm_w`` [h*d_v] (all ones when absent).
 
     ``weights`` holds ``branches`` (per scale: Wq, Wk, Wv, Wg1, Wg2, bg, Wo)
     and ``Wfuse``, ``bfuse``. Returns O [B, L, d]; with ``intermediates`` also a
@@ -189,6 +208,10 @@ def layer_forward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: in
                 ck, cv = slice(hh * d_k, (hh + 1) * d_k), slice(hh * d_v, (hh + 1) * d_v)
                 o[:, cv] = gla_recurrent(q[:, ck], k[:, ck], v[:, cv], la[:, ck],
                                          qk_scale=qk_scale, counter=counter)
+                if head_norm_eps is not None:
+                    nw = br.get("norm_w")
+                    nw = np.ones(h * d_v) if nw is None else nw
+                    o[:, cv] = head_rmsnorm(o[:, cv], nw[cv], head_norm_eps)
             Y = o @ br["Wo"].T
             O[b] += w[:, j:j + 1] * hold(Y, s, L)
             if intermediates:

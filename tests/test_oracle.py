@@ -198,6 +198,68 @@ def test_left_padding_changes_only_mixed_blocks():
     np.testing.assert_allclose(P[1], X[4:8].mean(0), rtol=1e-15)
 
 
+# --------------------------------------------------------------------------
+# optional per-head RMS normalisation (Sec. 3.2 reading)
+# --------------------------------------------------------------------------
+def check_head_norm_unit_rms(seed=21):
+    """eps ~ 0, unit weight: every head's normalised output row has RMS 1."""
+    rng = np.random.default_rng(seed)
+    d, dk, dv, L = 8, 3, 5, 19
+    W = _rand_weights(rng, d, (1, 2), (2, 1), dk, dv)
+    X = rng.normal(size=(1, L, d))
+    _, inter = om.layer_forward(X, W, (1, 2), (2, 1), dk, dv, intermediates=True, head_norm_eps=1e-30)
+    for (s, h), br in zip(((1, 2), (2, 1)), inter["branches"]):
+        o = br["o"][0]
+        for hh in range(h):
+            rms = np.sqrt((o[:, hh * dv:(hh + 1) * dv] ** 2).mean(axis=1))
+            np.testing.assert_allclose(rms, 1.0, rtol=1e-12)
+
+
+def check_head_norm_constant_row():
+    """A constant row c of width n: c / sqrt(c^2 + eps) times the weight."""
+    c, eps = 0.3, 0.05
+    w = np.array([1.0, -2.0, 0.5, 3.0])
+    got = om.head_rmsnorm(np.full((2, 4), c), w, eps)
+    np.testing.assert_allclose(got, np.tile(c / math.sqrt(c * c + eps) * w, (2, 1)), rtol=1e-14)
+
+
+def test_head_norm_unit_rms():
+    check_head_norm_unit_rms()
+
+
+def test_head_norm_constant_row():
+    check_head_norm_constant_row()
+
+
+def test_head_norm_is_invariant_to_value_scale():
+    """eps = 0: o is linear in W_v, and the RMS norm is homogeneous of degree 0,
+    so scaling every W_v by c > 0 leaves the layer output unchanged."""
+    rng = np.random.default_rng(22)
+    d, dk, dv = 6, 3, 4
+    W = _rand_weights(rng, d, (1, 2, 4), (2, 1, 1), dk, dv)
+    for br in W["branches"]:
+        br["norm_w"] = rng.normal(1.0, 0.3, br["Wv"].shape[0])
+    X = rng.normal(size=(2, 17, d))
+    a = om.layer_forward(X, W, (1, 2, 4), (2, 1, 1), dk, dv, head_norm_eps=0.0)
+    for br in W["branches"]:
+        br["Wv"] = br["Wv"] * 3.7
+    b = om.layer_forward(X, W, (1, 2, 4), (2, 1, 1), dk, dv, head_norm_eps=0.0)
+    np.testing.assert_allclose(b, a, rtol=1e-10, atol=1e-12)
+    c = om.layer_forward(X, W, (1, 2, 4), (2, 1, 1), dk, dv)
+    assert np.abs(c).max() > 2 * np.abs(a).max() or not np.allclose(c, a)
+
+
+def test_head_norm_off_by_default():
+    rng = np.random.default_rng(23)
+    W = _rand_weights(rng, 5, (1, 2), (1, 1), 2, 3)
+    for br in W["branches"]:
+        br["norm_w"] = np.full(3, 2.0)
+    X = rng.normal(size=(1, 9, 5))
+    _, inter = om.layer_forward(X, W, (1, 2), (1, 1), 2, 3, intermediates=True)
+    q, k, v, la = om.branch_projections(inter["branches"][0]["Xp"][0], W["branches"][0], 16.0)
+    np.testing.assert_array_equal(inter["branches"][0]["o"][0], om.gla_recurrent(q, k, v, la))
+
+
 def test_update_ratio_11_16():
     num, den = _read_table("update_ratio.txt")[0]
     L = 256
@@ -417,13 +479,30 @@ def _mutant_pool_mask_divide_by_block(X, s, M=None):
     return out
 
 
+def _mutant_head_norm_no_sqrt(o, weight, eps):
+    return o / ((o * o).mean(axis=1, keepdims=True) + eps) * weight
+
+
+def _mutant_head_norm_sum_not_mean(o, weight, eps):
+    return o / np.sqrt((o * o).sum(axis=1, keepdims=True) + eps) * weight
+
+
+def _mutant_head_norm_eps_outside(o, weight, eps):
+    return o / (np.sqrt((o * o).mean(axis=1, keepdims=True)) + eps) * weight
+
+
+def _mutant_head_norm_no_weight(o, weight, eps):
+    return o / np.sqrt((o * o).mean(axis=1, keepdims=True) + eps)
+
+
 def _mutant_softmax_wrong_axis(X, Wfuse, bfuse):
     z = X @ Wfuse.T + bfuse
     return np.exp(z) / np.exp(z).sum(axis=0, keepdims=True)
 
 
 PINS = [check_hold_table, check_pool_example, check_pool_tail, check_pool_mask, check_gla_bruteforce,
-        check_layer_bruteforce, check_constant_input_closed_form]
+        check_layer_bruteforce, check_constant_input_closed_form, check_head_norm_unit_rms,
+        check_head_norm_constant_row]
 
 
 @pytest.mark.parametrize("name,mutant", [
@@ -434,6 +513,10 @@ PINS = [check_hold_table, check_pool_example, check_pool_tail, check_pool_mask, 
     ("pool", _mutant_pool_divide_by_s),
     ("pool", _mutant_pool_mask_divide_by_block),
     ("fusion_weights", _mutant_softmax_wrong_axis),
+    ("head_rmsnorm", _mutant_head_norm_no_sqrt),
+    ("head_rmsnorm", _mutant_head_norm_sum_not_mean),
+    ("head_rmsnorm", _mutant_head_norm_eps_outside),
+    ("head_rmsnorm", _mutant_head_norm_no_weight),
 ])
 def test_planted_mistake_is_caught(monkeypatch, name, mutant):
     monkeypatch.setattr(om, name, mutant)
