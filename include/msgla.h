@@ -60,6 +60,11 @@ typedef struct msgla_config {
                                     beyond rounding (Sec. 3.4 of the notes).             */
   float gate_normalizer;         /* log alpha = logsigmoid(.) / gate_normalizer (> 0)     */
   float qk_scale;                /* o_t = qk_scale * q_t S_t                              */
+  int head_norm;                 /* per-branch normalisation (Sec. 3.2 lists one per branch
+                                    without defining it): 0 = none (default), 1 = RMS norm
+                                    of each head's GLA output row before W_o:
+                                    o_h <- o_h / sqrt(mean_c o_hc^2 + eps) * norm_w        */
+  float head_norm_eps;           /* eps of the RMS norm; finite and > 0 when head_norm = 1 */
 } msgla_config;
 
 /* Weights: DEVICE pointers on the handle's device, read during msgla_create only
@@ -71,6 +76,8 @@ typedef struct msgla_config {
  * Heads are laid side by side: head h of scale j owns rows h*d_k..h*d_k+d_k-1 of
  * Wq/Wk/Wg2/bg, rows h*d_v.. of Wv and columns h*d_v.. of Wo.
  *   Wfuse  bf16 [n_scales, d]    bfuse f32 [n_scales] (NULL = zeros)
+ *   norm_w[j] f32 [h_j*d_v]  per-channel weight of the head RMS norm (read only when
+ *              msgla_config.head_norm = 1; NULL = ones)
  * bg[j] may be NULL (zeros). */
 typedef struct msgla_weights {
   const void*  Wq[MSGLA_MAX_SCALES];
@@ -82,6 +89,7 @@ typedef struct msgla_weights {
   const void*  Wo[MSGLA_MAX_SCALES];
   const void*  Wfuse;
   const float* bfuse;
+  const float* norm_w[MSGLA_MAX_SCALES];
 } msgla_weights;
 
 typedef struct msgla_handle msgla_handle;

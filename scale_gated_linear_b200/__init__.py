@@ -33,7 +33,8 @@ class MSGLA:
 
     def __init__(self, d: int, scales: Sequence[int], heads: Sequence[int], d_k: int, d_v: int,
                  weights: dict, gate_rank: int = 16, gate_normalizer: float = 16.0,
-                 qk_scale: float = 1.0, chunk: int = 0, device: int = 0):
+                 qk_scale: float = 1.0, chunk: int = 0, device: int = 0,
+                 head_norm_eps: Optional[float] = None):
         import torch
 
         lib = _lib.load()
@@ -45,6 +46,8 @@ class MSGLA:
             cfg.scales[j], cfg.heads[j] = s, h
         cfg.d_k, cfg.d_v, cfg.gate_rank, cfg.chunk = d_k, d_v, gate_rank, chunk
         cfg.gate_normalizer, cfg.qk_scale = gate_normalizer, qk_scale
+        if head_norm_eps is not None:  # per-head RMS norm of the GLA output (off by default)
+            cfg.head_norm, cfg.head_norm_eps = 1, head_norm_eps
         dev = torch.device("cuda", device)
 
         def on_dev(t, dtype):
@@ -56,6 +59,7 @@ class MSGLA:
             ts = {k: on_dev(br[k], torch.bfloat16) for k in ("Wq", "Wk", "Wv", "Wg1", "Wo")}
             ts["Wg2"] = on_dev(br["Wg2"], torch.float32)
             ts["bg"] = on_dev(br.get("bg"), torch.float32)
+            ts["norm_w"] = on_dev(br.get("norm_w"), torch.float32)
             keep.append(ts)
             for k, t in ts.items():
                 getattr(w, k)[j] = _ptr(t)
@@ -185,5 +189,7 @@ class MSGLA:
 
     @classmethod
     def from_workload(cls, w, weights: dict, device: int = 0, **kw) -> "MSGLA":
+        if getattr(w, "head_norm", False):
+            kw.setdefault("head_norm_eps", w.norm_eps)
         return cls(d=w.d, scales=w.scales, heads=w.heads, d_k=w.d_k, d_v=w.d_v, weights=weights,
                    gate_rank=w.gate_rank, gate_normalizer=w.gate_normalizer, device=device, **kw)

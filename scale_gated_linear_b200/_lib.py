@@ -24,13 +24,15 @@ WS_POOLED, WS_Q, WS_K, WS_V, WS_GATE, WS_O, WS_Y, WS_FUSION = range(8)
 class Config(ctypes.Structure):
     _fields_ = [("d", c_int), ("n_scales", c_int), ("scales", c_int * MAX_SCALES),
                 ("heads", c_int * MAX_SCALES), ("d_k", c_int), ("d_v", c_int), ("gate_rank", c_int),
-                ("chunk", c_int), ("gate_normalizer", c_float), ("qk_scale", c_float)]
+                ("chunk", c_int), ("gate_normalizer", c_float), ("qk_scale", c_float),
+                ("head_norm", c_int), ("head_norm_eps", c_float)]
 
 
 class Weights(ctypes.Structure):
     _fields_ = [("Wq", c_void_p * MAX_SCALES), ("Wk", c_void_p * MAX_SCALES), ("Wv", c_void_p * MAX_SCALES),
                 ("Wg1", c_void_p * MAX_SCALES), ("Wg2", c_void_p * MAX_SCALES), ("bg", c_void_p * MAX_SCALES),
-                ("Wo", c_void_p * MAX_SCALES), ("Wfuse", c_void_p), ("bfuse", c_void_p)]
+                ("Wo", c_void_p * MAX_SCALES), ("Wfuse", c_void_p), ("bfuse", c_void_p),
+                ("norm_w", c_void_p * MAX_SCALES)]
 
 
 class MSGLAError(RuntimeError):

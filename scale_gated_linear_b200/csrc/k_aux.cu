@@ -8,6 +8,8 @@
 //                     each 128-row GLA chunk referenced to the chunk's 64th
 //                     row (m): Qs = q e^{b - m}, Ks = k e^{m - b}, and per chunk
 //                     gamma = e^{b_last - m}, mid = e^{m}.
+//   head_norm_kernel  optional per-branch normalisation (Sec. 3.2), read as an
+//                     RMS norm of each head's GLA output row, in place.
 //   hold_fuse_kernel  O_t = sum_s w_{t,s} Y^(s)_{floor((t+1)/s)-1} (Sec. 3.3,
 //                     Eq. (11)) when no branch has scale 1.
 //   weight converters used once by msgla_create.
@@ -340,6 +342,61 @@ __global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
   if (bad) atomicCAS(p.err, 0, kDevRange);
 }
 
+// One warp per (row, head): the head's dvp fp16 values (dvp <= 1024, a multiple
+// of 128) are read once into registers, 8 per 16-byte load, and written back
+// scaled; the padding columns are zero and stay zero (their weight is zero).
+constexpr int kNormMaxLoads = 4;  // 16-byte loads per lane: 4 * 32 * 8 = 1024 values
+__global__ void __launch_bounds__(256) head_norm_kernel(const HeadNormParams p) {
+  const long long gw = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (gw >= p.total_warps) return;
+  int j = 0;
+  while (j + 1 < p.n_branches && gw >= p.br[j + 1].warp_begin) ++j;
+  const HeadNormBranch& br = p.br[j];
+  const long long local = gw - br.warp_begin;
+  const long long row = local / br.heads;
+  const int head = static_cast<int>(local % br.heads);
+  __half* o = br.o + (row * br.heads + head) * p.dvp;
+  const float* w = br.w + static_cast<size_t>(head) * p.dvp;
+  const int lane = threadIdx.x & 31;
+  uint4 u[kNormMaxLoads];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kNormMaxLoads; ++i) {
+    const int c = (i * 32 + lane) * 8;
+    u[i] = c < p.dvp ? *reinterpret_cast<const uint4*>(o + c) : make_uint4(0, 0, 0, 0);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&u[i]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(h2[e]);
+      ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  const float inv = rsqrtf(ss / static_cast<float>(p.dv) + p.eps);
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < kNormMaxLoads; ++i) {
+    const int c = (i * 32 + lane) * 8;
+    if (c >= p.dvp) break;
+    const __half2* h2 = reinterpret_cast<const __half2*>(&u[i]);
+    const float4 wa = *reinterpret_cast<const float4*>(w + c);
+    const float4 wb = *reinterpret_cast<const float4*>(w + c + 4);
+    const float ws[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+    uint4 out;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(h2[e]);
+      const float a0 = f.x * inv * ws[2 * e], a1 = f.y * inv * ws[2 * e + 1];
+      bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
+      ow[e] = pack_half2(a0, a1);
+    }
+    *reinterpret_cast<uint4*>(o + c) = out;
+  }
+  if (bad) atomicCAS(p.err, 0, kDevRange);
+}
+
 constexpr int kGateThreads = 256;
 constexpr int kGateChannels = 128;  // key channels per CTA
 
@@ -657,6 +714,13 @@ cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st) {
   while (q.block_rows < 32) q.block_rows *= 2;
   dim3 grid((p.L + q.block_rows - 1) / q.block_rows, p.B);
   pool_fuse_kernel<<<grid, kPoolThreads, 0, st>>>(q);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_head_norm(const HeadNormParams& p, cudaStream_t st) {
+  if (p.total_warps <= 0) return cudaSuccess;
+  if (p.dvp % 128 || p.dvp > kNormMaxLoads * 32 * 8) return cudaErrorInvalidValue;
+  head_norm_kernel<<<static_cast<unsigned>((p.total_warps + 7) / 8), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 

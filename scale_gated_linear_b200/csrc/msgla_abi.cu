@@ -113,6 +113,7 @@ struct Branch {
   float* Wg2p;        // [h dkp, rp]
   float* bgp;         // [h dkp]
   __half* Wop;        // [d, h dvp]
+  float* normw;       // [h dvp] head RMS-norm weight (zero padding), when enabled
 };
 
 struct msgla_handle {
@@ -237,6 +238,10 @@ int validate(const msgla_config* c) {
   if (!(c->gate_normalizer > 0.f) || !std::isfinite(c->gate_normalizer))
     return fail(MSGLA_ERR_INVALID_ARG, "gate_normalizer must be finite and > 0");
   if (!std::isfinite(c->qk_scale)) return fail(MSGLA_ERR_INVALID_ARG, "qk_scale must be finite");
+  if (c->head_norm != 0 && c->head_norm != 1)
+    return fail(MSGLA_ERR_INVALID_ARG, "head_norm=%d: 0 (none) or 1 (RMS norm)", c->head_norm);
+  if (c->head_norm && !(c->head_norm_eps > 0.f && std::isfinite(c->head_norm_eps)))
+    return fail(MSGLA_ERR_INVALID_ARG, "head_norm_eps must be finite and > 0");
   int lcm = 1;
   for (int j = 0; j < c->n_scales; ++j)
     if (c->scales[j] > 1) lcm = lcm / gcd(lcm, c->scales[j]) * c->scales[j];
@@ -252,6 +257,7 @@ void free_handle(msgla_handle* h) {
     cudaFree(h->br[j].Wg2p);
     cudaFree(h->br[j].bgp);
     cudaFree(h->br[j].Wop);
+    cudaFree(h->br[j].normw);
   }
   cudaFree(h->Wfuse);
   cudaFree(h->bfuse);
@@ -308,6 +314,17 @@ int create_impl(msgla_handle* h, const msgla_weights* w) {
       CUDA_TRY(launch_bf16_to_f16_rows(static_cast<const __nv_bfloat16*>(w->Wo[j]) + static_cast<size_t>(x) * dv,
                                        hh * dv, d, dv, b.Wop + static_cast<size_t>(x) * h->dvp, hh * h->dvp, d_over,
                                        0));
+    }
+    if (c.head_norm) {
+      if ((st = dmalloc_zero(&b.normw, static_cast<size_t>(hh) * h->dvp * 4))) return st;
+      if (w->norm_w[j]) {
+        CUDA_TRY(cudaMemcpy2D(b.normw, h->dvp * 4, w->norm_w[j], dv * 4, dv * 4, hh, cudaMemcpyDeviceToDevice));
+      } else {
+        std::vector<float> ones(static_cast<size_t>(hh) * h->dvp, 0.f);
+        for (int x = 0; x < hh; ++x)
+          for (int e = 0; e < dv; ++e) ones[static_cast<size_t>(x) * h->dvp + e] = 1.f;
+        CUDA_TRY(cudaMemcpy(b.normw, ones.data(), ones.size() * 4, cudaMemcpyHostToDevice));
+      }
     }
     CUDA_TRY(put_rows(w->Wg1[j], 0, r, hh * (2 * h->dkp + h->dvp)));
     if (j == h->main_index) {
@@ -519,6 +536,29 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   h->test_skip_arrival = 0;
   CUDA_TRY(launch_gla(lp, st));
   CUDA_TRY(rec->mark(st));
+
+  // 4b. optional per-head RMS norm of the GLA output (in place)
+  if (c.head_norm) {
+    HeadNormParams np{};
+    long long warps = 0;
+    for (int j = 0; j < ns; ++j) {
+      HeadNormBranch& q = np.br[j];
+      q.o = static_cast<__half*>(at(ws.br[j].o));
+      q.w = h->br[j].normw;
+      q.rows = static_cast<long long>(B) * ws.br[j].rows;
+      q.heads = h->br[j].heads;
+      q.warp_begin = warps;
+      warps += q.rows * q.heads;
+    }
+    np.n_branches = ns;
+    np.total_warps = warps;
+    np.dvp = h->dvp;
+    np.dv = c.d_v;
+    np.eps = c.head_norm_eps;
+    np.err = h->d_err;
+    CUDA_TRY(launch_head_norm(np, st));
+    CUDA_TRY(rec->mark(st));
+  }
 
   // 5. coarse branches: Y^(s) = o W_o^T (fp16)
   memset(&gp, 0, sizeof(gp));
@@ -924,6 +964,7 @@ int msgla_launch_plan(const msgla_handle* h, int B, int L, char* names, size_t l
       add_name("gla_scan");
     }
     add_name("gla");
+    if (h->cfg.head_norm) add_name("head_norm");
     if (h->main_index >= 0) {
       if (h->n_scales > 1) add_name("out_gemm_coarse");
       add_name("out_gemm_fused");

@@ -128,6 +128,24 @@ struct GateParams {
 };
 cudaError_t launch_gate(const GateParams& p, cudaStream_t st);
 
+// optional per-head RMS norm of the GLA output, in place:
+// o_h <- o_h / sqrt(sum_c o_hc^2 / dv + eps) * w_h (one warp per row and head)
+struct HeadNormBranch {
+  __half* o;            // [B * rows, heads * dvp]
+  const float* w;       // [heads * dvp], zero in the padding columns
+  long long rows;       // B * rows
+  long long warp_begin;
+  int heads;
+};
+struct HeadNormParams {
+  HeadNormBranch br[kMaxScales];
+  int n_branches, dvp, dv;
+  long long total_warps;
+  float eps;
+  int* err;
+};
+cudaError_t launch_head_norm(const HeadNormParams& p, cudaStream_t st);
+
 // hold + fuse from materialised branch outputs (used when no branch has scale 1)
 struct HoldFuseParams {
   const __half* Y[kMaxScales];  // [B, n_s, d]

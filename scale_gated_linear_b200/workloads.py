@@ -51,6 +51,8 @@ class Workload:
     rms_norm_x: bool = True
     gate_bias: float = 0.0
     gate_fan_in_init: bool = False  # W_g1 ~ N(0,1/d), W_g2 ~ N(0,1/r)
+    head_norm: bool = False         # per-head RMS norm of the GLA output (norm_w ~ N(1, 0.1^2))
+    norm_eps: float = 1e-5
     seed: int = 0
 
     @property
@@ -94,7 +96,8 @@ def make_inputs(w: Workload, B: Optional[int] = None, L: Optional[int] = None,
 
     Returns a dict with ``X`` [B, L, d] and ``branches`` (one dict per scale
     with Wq [h*d_k, d], Wk [h*d_k, d], Wv [h*d_v, d], Wg1 [r, d], Wg2 [h*d_k, r],
-    bg [h*d_k], Wo [d, h*d_v]) plus ``Wfuse`` [n_scales, d] and ``bfuse``
+    bg [h*d_k], Wo [d, h*d_v], and norm_w [h*d_v] fp32 for ``head_norm``
+    workloads) plus ``Wfuse`` [n_scales, d] and ``bfuse``
     [n_scales]. Tensors meant for bf16 storage are returned as bfloat16 when
     ``round_to_bf16`` (default: the workload's dtype is bf16); fp32 otherwise.
     Weights are drawn before X so that a different B or L keeps the weights.
@@ -125,6 +128,8 @@ def make_inputs(w: Workload, B: Optional[int] = None, L: Optional[int] = None,
             br["Wg2"] = _normal(g, (h * w.d_k, r), std_for(r))
         br["bg"] = torch.full((h * w.d_k,), float(w.gate_bias), dtype=torch.float32)
         br["Wo"] = lo(_normal(g, (d, h * w.d_v), std_for(h * w.d_v)))
+        if w.head_norm:
+            br["norm_w"] = 1.0 + _normal(g, (h * w.d_v,), 0.1)
         branches.append(br)
     Wfuse = lo(_normal(g, (len(w.scales), d), std_for(d)))
     bfuse = torch.zeros(len(w.scales), dtype=torch.float32)

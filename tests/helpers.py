@@ -33,4 +33,5 @@ def oracle_forward(w: wl.Workload, inp: dict, rows=None, intermediates=False, ba
     if mask is not None:
         mask = np.asarray(mask, dtype=np.float64)
     return oracle.layer_forward(X, f, w.scales, w.heads, w.d_k, w.d_v,
-                                gate_normalizer=w.gate_normalizer, intermediates=intermediates, mask=mask)
+                                gate_normalizer=w.gate_normalizer, intermediates=intermediates, mask=mask,
+                                head_norm_eps=w.norm_eps if w.head_norm else None)

@@ -61,6 +61,8 @@ def _cfg(**kw):
     (dict(d_k=300), -2), (dict(d_v=0), -2), (dict(gate_rank=33), -2), (dict(chunk=16), -2), (dict(chunk=64), -2),
     (dict(gate_normalizer=0.0), -1), (dict(gate_normalizer=float("nan")), -1),
     (dict(qk_scale=float("inf")), -1), (dict(scales=(1, 7, 11)), -2),
+    (dict(head_norm=2, head_norm_eps=1e-5), -1), (dict(head_norm=1, head_norm_eps=0.0), -1),
+    (dict(head_norm=1, head_norm_eps=float("nan")), -1),
 ])
 def test_create_rejects_bad_config(kw, code):
     lib = _lib.load()
