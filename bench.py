@@ -10,6 +10,11 @@ seeded synthetic inputs (see scale_gated_linear_b200/workloads.py). With N > 1
 of 8 sequences: batch sequences are independent, so the work is sharded by
 sequence with no collective on the data path ("scaling": "weak").
 
+Variants of the same step: --mask left|right|random times the masked forward
+(valid-token mask in the pooling, Eq. (8); e2e is then not measured: the host
+entry point takes no mask) and --head-norm enables the optional per-head RMS
+norm of the GLA output.
+
 Prints one JSON line on rank 0. Timing: W untimed warm-up steps, then K timed
 steps, each bracketed by CUDA events on the launching stream with a 256 MiB
 write between steps to flush the 126 MB L2; the per-kernel events of
@@ -96,6 +101,8 @@ def algorithmic_counts(w, B: int, L: int) -> dict:
     out["gate"] = {"bytes": sum(rows[s] * (h * w.d_k * 2 * 2 * 2 + r * 4)
                                 + 2 * math.ceil(rows[s] / B / C) * B * h * w.d_k * 4
                                 for s, h in zip(w.scales, w.heads))}
+    if getattr(w, "head_norm", False):  # read + write of the GLA output, in place
+        out["head_norm"] = {"bytes": sum(rows[s] * h * w.d_v * 2 * 2 for s, h in zip(w.scales, w.heads))}
     total_flops = sum(v.get("flops", 0) for v in out.values())
     weights = sum(h * (2 * w.d_k + w.d_v) * w.d * 2 + r * w.d * 2 + h * w.d_k * r * 4 + w.d * h * w.d_v * 2
                   for s, h in zip(w.scales, w.heads))
@@ -183,7 +190,7 @@ def numpy_threads() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample(w, inp, rows_budget_s: float, prefix: int | None = None):
+def oracle_sample(w, inp, rows_budget_s: float, prefix: int | None = None, mask=None):
     """Run the fp64 oracle on whole batch rows (or a prefix of them) until about
     `rows_budget_s` seconds have passed. Returns (tokens, seconds, description)."""
     import numpy as np
@@ -195,7 +202,9 @@ def oracle_sample(w, inp, rows_budget_s: float, prefix: int | None = None):
     done, t0 = 0, time.perf_counter()
     for b in range(f["X"].shape[0]):
         oracle.layer_forward(f["X"][b:b + 1, :L], f, w.scales, w.heads, w.d_k, w.d_v,
-                             gate_normalizer=w.gate_normalizer)
+                             gate_normalizer=w.gate_normalizer,
+                             mask=None if mask is None else mask[b:b + 1, :L].numpy(),
+                             head_norm_eps=w.norm_eps if w.head_norm else None)
         done += 1
         if time.perf_counter() - t0 >= rows_budget_s:
             break
@@ -237,14 +246,14 @@ def run_reference(args) -> int:
 
 
 # --------------------------------------------------------------------- our arm
-def time_layer(layer, X, O, ws, steps: int, warmup: int, flush, n_events: int):
+def time_layer(layer, X, O, ws, steps: int, warmup: int, flush, n_events: int, mask=None):
     import torch
     stream = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(steps)]
     wev = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
     for _ in range(warmup):
         flush()
-        layer.forward_profiled(X, O, ws, wev, stream)
+        layer.forward_profiled(X, O, ws, wev, stream, mask=mask)
     return ev
 
 
@@ -267,14 +276,17 @@ def run_ours(args) -> int:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     w = wl.WORKLOADS[args.workload]
+    if args.head_norm:
+        w = w.replace(head_norm=True)
     peaks, peak_kind = load_peaks()
     cpu_line = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp0 = wl.make_inputs(w, B=min(w.B, 4))
-        tok, dt, desc = oracle_sample(w, inp0, args.cpu_seconds)
+        m0 = None if args.mask == "none" else wl.make_mask(min(w.B, 4), w.L, args.mask, seed=w.seed)
+        tok, dt, desc = oracle_sample(w, inp0, args.cpu_seconds, mask=m0)
         cpu_line = {"value": tok / dt, "unit": UNIT, "cores": numpy_threads(), "kind": "oracle", "sample": desc}
 
-    def measure(wk, steps, warmup, e2e: bool):
+    def measure(wk, steps, warmup, e2e: bool, mask_kind: str = "none"):
         inp = wl.make_inputs(wk)
         if rank > 0:  # this rank's own batch of sequences (same weights)
             g = torch.Generator().manual_seed(wk.seed * 1000 + rank)
@@ -282,13 +294,14 @@ def run_ours(args) -> int:
             inp["X"] = (X / X.pow(2).mean(-1, keepdim=True).sqrt()).to(torch.bfloat16)
         layer = MSGLA.from_workload(wk, inp, device=local)
         X = inp["X"].to(dev)
+        M = None if mask_kind == "none" else wl.make_mask(wk.B, wk.L, mask_kind, seed=wk.seed + rank).to(dev)
         O = torch.empty_like(X)
         ws = layer.alloc_workspace(wk.B, wk.L)
         flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
         flush = lambda: flush_buf.fill_(1)
         names = layer.launch_names(wk.B, wk.L)
         n_ev = len(names) + 1
-        ev = time_layer(layer, X, O, ws, steps, warmup, flush, n_ev)
+        ev = time_layer(layer, X, O, ws, steps, warmup, flush, n_ev, mask=M)
         torch.cuda.synchronize()
         layer.check_status()
         if world > 1:
@@ -302,7 +315,7 @@ def run_ours(args) -> int:
         stream = torch.cuda.current_stream()
         for k in range(steps):
             flush()
-            launches += layer.forward_profiled(X, O, ws, ev[k], stream)
+            launches += layer.forward_profiled(X, O, ws, ev[k], stream, mask=M)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -336,7 +349,7 @@ def run_ours(args) -> int:
         torch.cuda.empty_cache()
         return res
 
-    r = measure(w, args.steps, args.warmup, e2e=not args.no_e2e)
+    r = measure(w, args.steps, args.warmup, e2e=not args.no_e2e and args.mask == "none", mask_kind=args.mask)
     tokens = r["tokens_per_step"] * args.steps * world
     value = tokens / (r["total_ms"] / 1e3)
     counts = algorithmic_counts(w, w.B, w.L)
@@ -362,7 +375,9 @@ def run_ours(args) -> int:
         "vs_baseline": None, "dtype": "f16/bf16 tensor-core operands, f32 accumulate; bf16 in/out",
         "data": "synthetic (seeded N(0,1) rows RMS-normalised, weights N(0,0.02))",
         "config": {"workload": f"{w.name}: B={w.B} per GPU, L={w.L}, d={w.d}, scales {list(w.scales)} heads "
-                               f"{list(w.heads)}, d_k={w.d_k}, d_v={w.d_v}, gate rank {w.gate_rank}, chunk 128",
+                               f"{list(w.heads)}, d_k={w.d_k}, d_v={w.d_v}, gate rank {w.gate_rank}, chunk 128"
+                               + (f", {args.mask}-padding mask" if args.mask != "none" else "")
+                               + (", head RMS norm" if w.head_norm else ""),
                    "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"sequence-sharded x{world}",
                    "l2": "flushed between timed steps (256 MiB write)"},
         "roofline": roof,
@@ -375,7 +390,9 @@ def run_ours(args) -> int:
     if "e2e_ms" in r:
         line["e2e"] = {"value": tokens / (r["e2e_ms"] / 1e3), "unit": UNIT,
                        "h2d_bytes_per_step": r["io_bytes"], "d2h_bytes_per_step": r["io_bytes"]}
-    if world == 1 and not args.no_gla_baseline:
+    elif args.mask != "none":
+        line["e2e"] = {"value": None, "unit": UNIT, "note": "not measured: the host-buffer entry point takes no mask"}
+    if world == 1 and not args.no_gla_baseline and args.mask == "none" and not w.head_norm:
         g = measure(wl.WORKLOADS[BASELINE_WORKLOAD], max(3, args.steps // 2), args.warmup, e2e=False)
         g_ms = g["total_ms"] / max(3, args.steps // 2)
         line["gla_baseline"] = {"workload": BASELINE_WORKLOAD, "value": g["tokens_per_step"] / (g_ms * 1e-3),
@@ -402,6 +419,9 @@ def main(argv=None) -> int:
     ap.add_argument("--no-gla-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the CPU oracle baseline")
     ap.add_argument("--ref-prefix", type=int, default=512, help="positions per reference-arm step")
+    ap.add_argument("--mask", choices=("none", "left", "right", "random"), default="none",
+                    help="time the masked forward with this valid-token mask")
+    ap.add_argument("--head-norm", action="store_true", help="enable the per-head RMS norm of the GLA output")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)

@@ -162,8 +162,9 @@ int msgla_forward_noalloc(msgla_handle* h, const void* X, int B, int L, void* O,
  * handles: events[0] is recorded before the first kernel and events[i+1] after
  * the i-th kernel; msgla_launch_plan lists the kernels in launch order.
  * `max_events` is the length of `events` (it must be at least n_launches + 1);
- * *n_launches receives the number of kernels launched. */
-int msgla_forward_profiled(msgla_handle* h, const void* X, int B, int L, void* O,
+ * *n_launches receives the number of kernels launched. `M` is the optional
+ * valid-token mask of msgla_forward_masked (NULL = every token valid). */
+int msgla_forward_profiled(msgla_handle* h, const void* X, const void* M, int B, int L, void* O,
                            void* workspace, size_t workspace_bytes, void* stream,
                            void* const* events, int max_events, int* n_launches);
 
@@ -195,10 +196,11 @@ int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index,
 
 /* Kernels that msgla_forward launches for a [B, L, d] input, in launch order, as a
  * comma-separated list written to `names` (NUL-terminated, at most `len` bytes):
- * pool_fuse, proj_gemm, gate, [gla_state, gla_scan], gla, [out_gemm_coarse],
- * out_gemm_fused | out_gemm_coarse, hold_fuse. gla_state and gla_scan appear when
- * long sequences are cut into segments (few sequences: the GLA kernel would fill
- * less than half of the GPU). msgla_forward_profiled records one event per entry. */
+ * pool_fuse, proj_gemm, gate, [gla_state, gla_scan], gla, [head_norm],
+ * [out_gemm_coarse], out_gemm_fused | out_gemm_coarse, hold_fuse. gla_state and
+ * gla_scan appear when long sequences are cut into segments (few sequences: the
+ * GLA kernel would fill less than half of the GPU); head_norm when the config
+ * enables the head RMS norm. msgla_forward_profiled records one event per entry. */
 int msgla_launch_plan(const msgla_handle* h, int B, int L, char* names, size_t len);
 
 /* Failure-detection testing: with enable != 0, the next forward on this handle

@@ -127,10 +127,10 @@ class MSGLA:
         _lib.check(self._lib.msgla_launch_plan(self._h, B, L, buf, len(buf)))
         return buf.value.decode().split(",") if buf.value else []
 
-    def forward_profiled(self, X, out, workspace, events, stream=None):
+    def forward_profiled(self, X, out, workspace, events, stream=None, mask=None):
         """forward() recording events[0] before the first kernel and events[i+1]
         after kernel i (torch.cuda.Event objects with timing enabled). Returns the
-        number of kernels launched."""
+        number of kernels launched. ``mask`` as for forward()."""
         import torch
         B, L, d = X.shape
         if stream is None:
@@ -140,7 +140,11 @@ class MSGLA:
                 e.record(stream)
         arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         n = ctypes.c_int()
-        _lib.check(self._lib.msgla_forward_profiled(self._h, X.data_ptr(), B, L, out.data_ptr(),
+        if mask is not None:
+            assert mask.shape == (B, L) and mask.is_cuda and mask.is_contiguous()
+            assert mask.dtype in (torch.bool, torch.uint8)
+        _lib.check(self._lib.msgla_forward_profiled(self._h, X.data_ptr(), None if mask is None else mask.data_ptr(),
+                                                    B, L, out.data_ptr(),
                                                     workspace.data_ptr(), workspace.numel(),
                                                     ctypes.c_void_p(stream.cuda_stream), arr, len(events),
                                                     ctypes.byref(n)))

@@ -49,8 +49,8 @@ _SIGNATURES = {
     "msgla_forward_masked": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_size_t,
                                      c_void_p]),
     "msgla_forward_noalloc": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p]),
-    "msgla_forward_profiled": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_size_t, c_void_p,
-                                       POINTER(c_void_p), c_int, POINTER(c_int)]),
+    "msgla_forward_profiled": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_size_t,
+                                       c_void_p, POINTER(c_void_p), c_int, POINTER(c_int)]),
     "msgla_workspace_size_host": (c_int, [c_void_p, c_int, c_int, POINTER(c_size_t)]),
     "msgla_forward_host": (c_int, [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "msgla_sync_status": (c_int, [c_void_p]),

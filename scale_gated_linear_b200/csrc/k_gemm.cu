@@ -161,11 +161,21 @@ __device__ __forceinline__ void epilogue_fuse_prefetch(const GemmTask& T, const 
   }
 }
 
+// Whether this thread's accumulator row is a padded token of a masked scale-1
+// projection. Read before the wait for the accumulator so that the load's latency
+// hides behind the MMAs.
+__device__ __forceinline__ bool row_is_padded(const GemmParams& p, const TileCoord& tc, int quad, int lane) {
+  const GemmTask& T = p.task[tc.task];
+  if (T.epi != kEpiProj || !T.mask) return false;
+  const int row = tc.m0 + quad * 32 + lane;
+  return row < T.rows && !__ldg(T.mask + static_cast<size_t>(tc.b) * T.rows + row);
+}
+
 // Columns [c_lo, c_hi) of the tile (multiples of 32 from 0) for the accumulator
 // rows of TMEM lane quadrant `quad`.
 template <int BN>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
-                                              int lane, int c_lo, int c_hi) {
+                                              int lane, int c_lo, int c_hi, bool padded) {
   const GemmTask& T = p.task[tc.task];
   const int r = quad * 32 + lane;
   const int row = tc.m0 + r;
@@ -196,7 +206,6 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
   const float wmain = (T.epi == kEpiFuse && valid) ? wts[T.main_index] : 0.f;
   // Eq. (8) at scale 1 zeroes a padded row; the projections have no bias, so its
   // q | k | v | g columns are zero (the fusion logits read x_t and are kept)
-  const bool padded = T.epi == kEpiProj && T.mask && valid && !T.mask[grow];
   const int n_zeroed = T.nq + T.nk + T.nv + T.ng;
   for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
     uint32_t v[32];
@@ -358,11 +367,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
       const TileCoord tc = decode_tile(p, tile, BN);
       const uint32_t buf = it & 1;
+      const bool padded = row_is_padded(p, tc, quad, lane);
       if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
       int lo, hi;
       epi_columns(warp, tc.n_eff, lo, hi);
-      epilogue_tile<BN>(p, tc, tmem + buf * BN, quad, lane, lo, hi);
+      epilogue_tile<BN>(p, tc, tmem + buf * BN, quad, lane, lo, hi, padded);
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
     }
@@ -491,11 +501,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       TileCoord tc = decode_tile(p, tile, kPairBN, kPairBM);
       tc.m0 += 128 * static_cast<int>(rank);
       const uint32_t buf = it & 1;
+      const bool padded = row_is_padded(p, tc, quad, lane);
       if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
       int lo, hi;
       epi_columns(warp, tc.n_eff, lo, hi);
-      epilogue_tile<kPairBN>(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi);
+      epilogue_tile<kPairBN>(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded);
       tc_fence_before();
       mbar_arrive_cluster(buf ? lead_empty1 : lead_empty0);
     }

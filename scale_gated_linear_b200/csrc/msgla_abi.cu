@@ -838,7 +838,7 @@ int msgla_forward_noalloc(msgla_handle* h, const void* X, int B, int L, void* O,
   return forward_impl(h, X, B, L, O, scratch, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }
 
-int msgla_forward_profiled(msgla_handle* h, const void* X, int B, int L, void* O, void* workspace,
+int msgla_forward_profiled(msgla_handle* h, const void* X, const void* M, int B, int L, void* O, void* workspace,
                            size_t workspace_bytes, void* stream, void* const* events, int max_events,
                            int* n_launches) {
   if (!events || !n_launches) return fail(MSGLA_ERR_INVALID_ARG, "events or n_launches is NULL");
@@ -854,7 +854,8 @@ int msgla_forward_profiled(msgla_handle* h, const void* X, int B, int L, void* O
   Recorder rec;
   rec.events = events;
   rec.max_events = max_events;
-  st = forward_impl(h, X, B, L, O, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), &rec);
+  st = forward_impl(h, X, B, L, O, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), &rec,
+                    static_cast<const uint8_t*>(M));
   *n_launches = rec.n;
   return st;
 }
