@@ -110,26 +110,35 @@ def algorithmic_counts(w, B: int, L: int) -> dict:
     return {"kernels": out, "total_flops": total_flops, "layer_bytes": layer_bytes}
 
 
-def kernel_source_hash() -> str:
+# source files that decide what each timed kernel does (its own file and the shared headers)
+KERNEL_SOURCES = {
+    "proj_gemm": "k_gemm.cu", "out_gemm_coarse": "k_gemm.cu", "out_gemm_fused": "k_gemm.cu",
+    "gla": "k_gla.cu", "gla_state": "k_gla.cu", "gla_scan": "k_gla.cu",
+    "gate": "k_aux.cu", "pool_fuse": "k_aux.cu", "head_norm": "k_aux.cu", "hold_fuse": "k_aux.cu",
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "scale_gated_linear_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in (KERNEL_SOURCES[kernel], "msgla_internal.h", "sm100_ptx.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel: str, workload: str):
-    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None if
-    there is none or the kernel sources changed since it was taken."""
+    """Per-launch DRAM bytes (read + write) of `kernel` from the committed ncu
+    summary, or None if there is none or the kernel's sources changed since."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
-    if t.get("source_hash") != kernel_source_hash():
+    e = t.get("kernels", {}).get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
-    return t.get("kernels", {}).get(workload, {}).get(kernel)
+    return e.get("dram_bytes")
 
 
 class ClockSampler:
@@ -276,6 +285,8 @@ def run_ours(args) -> int:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     w = wl.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.replace(B=args.batch)
     if args.head_norm:
         w = w.replace(head_norm=True)
     peaks, peak_kind = load_peaks()
@@ -365,7 +376,8 @@ def run_ours(args) -> int:
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
     roof.update({"kernel": dominant, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst)"
-                 if peak_kind == "measured" else "fallback", "traffic": traffic_for(dominant, w.name),
+                 if peak_kind == "measured" else "fallback", "traffic": traffic_for(dominant, f"{w.name}/B{w.B}/L{w.L}")
+                 if args.mask == "none" and not w.head_norm else None,
                  "kernel_ms": mean_k[dominant]})
     step_ms = r["total_ms"] / args.steps
     path_tf = counts["total_flops"] / (step_ms * 1e-3) / 1e12
@@ -422,6 +434,7 @@ def main(argv=None) -> int:
     ap.add_argument("--mask", choices=("none", "left", "right", "random"), default="none",
                     help="time the masked forward with this valid-token mask")
     ap.add_argument("--head-norm", action="store_true", help="enable the per-head RMS norm of the GLA output")
+    ap.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's)")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
