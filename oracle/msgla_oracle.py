@@ -26,6 +26,10 @@ summarised in the MS-GLA reading notes (arXiv 2609.35664v1):
   floor((t+1)/s) - 1, or zero when that index is negative.
 * Sec. 3.3, Eqs. (10)-(11): w_t = softmax(W_fuse x_t + b_fuse) from the
   unpooled row x_t, and O_t = sum_s w_{t,s} Yhat^(s)_t.
+* token-by-token inference (the notes' item on training and per-token
+  inference, after the authors' cache): each branch keeps its GLA state, the
+  tokens of its unfinished block and its latest output; a branch steps once
+  its block is full and otherwise repeats its latest output.
 
 Readings where the notes leave a step open (each is also listed in the design
 notes of this repository):
@@ -225,6 +229,60 @@ def layer_forward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: in
         for name in list(br):
             br[name] = np.stack(br[name]) if br[name] else None
     return O, inter
+
+
+# ---------------------------------------------------------------------------
+# token-by-token inference (reading notes, method part, item 7 "training and
+# token-by-token inference"): per-branch cache, one token at a time
+# ---------------------------------------------------------------------------
+def decode_init(B: int, d: int, scales, heads, d_k: int, d_v: int) -> dict:
+    """Empty cache for B sequences. Per branch: the GLA state of every head
+    (S [B, h, d_k, d_v]), the running sum of the tokens not yet forming a full
+    block (buf [B, d]) with their count, and the branch output most recently
+    produced (Y [B, d], zero before the first complete block). Its size does
+    not depend on how many tokens have been consumed."""
+    return {"branches": [dict(S=np.zeros((B, h, d_k, d_v)), buf=np.zeros((B, d)), n=0, Y=np.zeros((B, d)))
+                         for s, h in zip(scales, heads)]}
+
+
+def decode_step(cache: dict, x: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: int,
+                gate_normalizer: float = 16.0, qk_scale: float = 1.0,
+                head_norm_eps: float | None = None) -> np.ndarray:
+    """Consume one token x [B, d] of each sequence; return O_t [B, d].
+
+    Each branch adds x to its buffer; once it holds s tokens, their mean is the
+    next pooled row (Eq. (8)), which takes one GLA step per head (S = Diag(alpha)
+    S + k^T v, o = qk_scale * q S), goes through W_o, replaces the cached output
+    and empties the buffer. Otherwise the branch keeps its previous output. The
+    output fuses the cached branch outputs with w = softmax(W_fuse x + b_fuse)."""
+    x = np.asarray(x, dtype=np.float64)
+    B = x.shape[0]
+    w = fusion_weights(x, weights["Wfuse"], weights["bfuse"])
+    O = np.zeros_like(x)
+    for j, (s, h) in enumerate(zip(scales, heads)):
+        br, c = weights["branches"][j], cache["branches"][j]
+        c["buf"] = c["buf"] + x
+        c["n"] += 1
+        if c["n"] == s:
+            xbar = c["buf"] / s
+            q, k, v, la = branch_projections(xbar, br, gate_normalizer)
+            alpha = np.exp(la)
+            o = np.zeros((B, h * d_v))
+            for b in range(B):
+                for hh in range(h):
+                    ck, cv = slice(hh * d_k, (hh + 1) * d_k), slice(hh * d_v, (hh + 1) * d_v)
+                    S = alpha[b, ck][:, None] * c["S"][b, hh] + np.outer(k[b, ck], v[b, cv])
+                    c["S"][b, hh] = S
+                    o[b, cv] = qk_scale * (q[b, ck] @ S)
+                    if head_norm_eps is not None:
+                        nw = br.get("norm_w")
+                        nw = np.ones(h * d_v) if nw is None else nw
+                        o[b:b + 1, cv] = head_rmsnorm(o[b:b + 1, cv], nw[cv], head_norm_eps)
+            c["Y"] = o @ br["Wo"].T
+            c["buf"] = np.zeros_like(c["buf"])
+            c["n"] = 0
+        O += w[:, j:j + 1] * c["Y"]
+    return O
 
 
 def state_updates(L: int, scales, heads) -> int:

@@ -260,6 +260,56 @@ def test_head_norm_off_by_default():
     np.testing.assert_array_equal(inter["branches"][0]["o"][0], om.gla_recurrent(q, k, v, la))
 
 
+# --------------------------------------------------------------------------
+# token-by-token inference against the whole-sequence layer
+# --------------------------------------------------------------------------
+def _decode_all(X, W, scales, heads, dk, dv, **kw):
+    B, L, d = X.shape
+    cache = om.decode_init(B, d, scales, heads, dk, dv)
+    return np.stack([om.decode_step(cache, X[:, t], W, scales, heads, dk, dv, **kw) for t in range(L)], axis=1)
+
+
+def check_decode_matches_parallel(seed=31):
+    """Feeding a ragged sequence one token at a time gives, at every position,
+    the layer output of Sec. 3 (the causal hold reads the block that ended last),
+    for scale sets with and without the scale-1 branch."""
+    rng = np.random.default_rng(seed)
+    d, dk, dv, L = 7, 3, 4, 23
+    for scales, heads in (((1, 2, 4), (2, 1, 1)), ((2, 3), (1, 2)), ((1, 5), (1, 1))):
+        W = _rand_weights(rng, d, scales, heads, dk, dv, gate_bias=1.0)
+        X = rng.normal(size=(2, L, d))
+        np.testing.assert_allclose(_decode_all(X, W, scales, heads, dk, dv, qk_scale=0.7),
+                                   om.layer_forward(X, W, scales, heads, dk, dv, qk_scale=0.7),
+                                   rtol=1e-11, atol=1e-12)
+
+
+def test_decode_matches_parallel():
+    check_decode_matches_parallel()
+
+
+def test_decode_with_head_norm_matches_parallel():
+    rng = np.random.default_rng(32)
+    d, dk, dv, L = 6, 2, 3, 17
+    W = _rand_weights(rng, d, (1, 2, 4), (2, 1, 1), dk, dv)
+    for br in W["branches"]:
+        br["norm_w"] = rng.normal(1.0, 0.2, br["Wv"].shape[0])
+    X = rng.normal(size=(1, L, d))
+    np.testing.assert_allclose(_decode_all(X, W, (1, 2, 4), (2, 1, 1), dk, dv, head_norm_eps=1e-3),
+                               om.layer_forward(X, W, (1, 2, 4), (2, 1, 1), dk, dv, head_norm_eps=1e-3),
+                               rtol=1e-11, atol=1e-12)
+
+
+def test_decode_cache_does_not_grow():
+    rng = np.random.default_rng(33)
+    W = _rand_weights(rng, 5, (1, 4), (1, 1), 2, 2)
+    cache = om.decode_init(3, 5, (1, 4), (1, 1), 2, 2)
+    shapes = [[v.shape for v in (c["S"], c["buf"], c["Y"])] for c in cache["branches"]]
+    for t in range(41):
+        om.decode_step(cache, rng.normal(size=(3, 5)), W, (1, 4), (1, 1), 2, 2)
+    assert [[v.shape for v in (c["S"], c["buf"], c["Y"])] for c in cache["branches"]] == shapes
+    assert cache["branches"][1]["n"] == 41 % 4
+
+
 def test_update_ratio_11_16():
     num, den = _read_table("update_ratio.txt")[0]
     L = 256
@@ -495,6 +545,25 @@ def _mutant_head_norm_no_weight(o, weight, eps):
     return o / np.sqrt((o * o).mean(axis=1, keepdims=True) + eps)
 
 
+_real_decode_step = om.decode_step
+
+
+def _mutant_decode_one_step_late(cache, x, weights, scales, heads, d_k, d_v, **kw):
+    old = [c["Y"].copy() for c in cache["branches"]]
+    _real_decode_step(cache, x, weights, scales, heads, d_k, d_v, **kw)
+    w = om.fusion_weights(np.asarray(x, dtype=float), weights["Wfuse"], weights["bfuse"])
+    return sum(w[:, j:j + 1] * old[j] for j in range(len(scales)))
+
+
+def _mutant_decode_buffer_kept(cache, x, weights, scales, heads, d_k, d_v, **kw):
+    before = [c["buf"].copy() for c in cache["branches"]]
+    out = _real_decode_step(cache, x, weights, scales, heads, d_k, d_v, **kw)
+    for c, b in zip(cache["branches"], before):
+        if c["n"] == 0:          # the branch fired: keep the old tokens in its buffer
+            c["buf"] = b + x
+    return out
+
+
 def _mutant_softmax_wrong_axis(X, Wfuse, bfuse):
     z = X @ Wfuse.T + bfuse
     return np.exp(z) / np.exp(z).sum(axis=0, keepdims=True)
@@ -502,7 +571,7 @@ def _mutant_softmax_wrong_axis(X, Wfuse, bfuse):
 
 PINS = [check_hold_table, check_pool_example, check_pool_tail, check_pool_mask, check_gla_bruteforce,
         check_layer_bruteforce, check_constant_input_closed_form, check_head_norm_unit_rms,
-        check_head_norm_constant_row]
+        check_head_norm_constant_row, check_decode_matches_parallel]
 
 
 @pytest.mark.parametrize("name,mutant", [
@@ -517,6 +586,8 @@ PINS = [check_hold_table, check_pool_example, check_pool_tail, check_pool_mask, 
     ("head_rmsnorm", _mutant_head_norm_sum_not_mean),
     ("head_rmsnorm", _mutant_head_norm_eps_outside),
     ("head_rmsnorm", _mutant_head_norm_no_weight),
+    ("decode_step", _mutant_decode_one_step_late),
+    ("decode_step", _mutant_decode_buffer_kept),
 ])
 def test_planted_mistake_is_caught(monkeypatch, name, mutant):
     monkeypatch.setattr(om, name, mutant)
