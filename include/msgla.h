@@ -194,6 +194,40 @@ int msgla_sync_status(msgla_handle* h);
 int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index, int which,
                            size_t* offset, int dims[3]);
 
+/* ---- token-by-token inference (the notes' item on per-token inference, after the
+ * authors' cache): every branch keeps its GLA state, the sum of the tokens of its
+ * unfinished block and its latest output; a branch steps once its block of s
+ * tokens is complete (the block's mean is its next pooled row, Eq. (8)) and
+ * otherwise repeats its latest output, which is the causal hold of Sec. 3.3. The
+ * outputs equal those of msgla_forward position by position.
+ *
+ * Bytes of the decode cache of B sequences (B in [0, 65535]): per branch the state
+ * f32 [B, h, dkp, dvp] (dkp = 128 or 256, dvp = d_v rounded up to 128) and, for
+ * s > 1, the block sum f32 [B, d] and the latest output f16 [B, d]. The size does
+ * not depend on how many tokens have been consumed. */
+int msgla_cache_size(const msgla_handle* h, int B, size_t* bytes);
+
+/* Empty the cache (the state before the first token): an asynchronous memset of
+ * msgla_cache_size bytes on `stream`. `cache` is a device buffer owned by the
+ * caller, 256-byte aligned. */
+int msgla_cache_reset(msgla_handle* h, void* cache, int B, void* stream);
+
+/* Bytes of device workspace msgla_step needs for B sequences. */
+int msgla_step_workspace_size(const msgla_handle* h, int B, size_t* bytes);
+
+/* Consume token t of each of B sequences and write the layer output at t.
+ *   cache  device buffer of msgla_cache_size(h, B) bytes, 256-byte aligned; read
+ *          and updated. After msgla_cache_reset it must be fed t = 0, 1, 2, ... in
+ *          order: the position decides which branches step ((t + 1) % s == 0).
+ *   x      device bf16 [B, d], 16-byte aligned (token t of every sequence).
+ *   O      device bf16 [B, d], 16-byte aligned, not overlapping x.
+ *   workspace  device buffer of at least msgla_step_workspace_size bytes, 256-byte
+ *          aligned, owned by the caller.
+ * Asynchronous on `stream`; kernel-side errors are reported by msgla_sync_status.
+ * B = 0 launches nothing. A padding mask is not supported here. */
+int msgla_step(msgla_handle* h, void* cache, const void* x, int B, long long t, void* O,
+               void* workspace, size_t workspace_bytes, void* stream);
+
 /* Kernels that msgla_forward launches for a [B, L, d] input, in launch order, as a
  * comma-separated list written to `names` (NUL-terminated, at most `len` bytes):
  * pool_fuse, proj_gemm, gate, [gla_state, gla_scan], gla, [head_norm],

@@ -121,6 +121,51 @@ class MSGLA:
 
     __call__ = forward
 
+    # ------------------------------------------------------------- decode
+    def cache_size(self, B: int) -> int:
+        n = ctypes.c_size_t()
+        _lib.check(self._lib.msgla_cache_size(self._h, B, ctypes.byref(n)))
+        return n.value
+
+    def new_cache(self, B: int, stream=None):
+        """Device buffer holding the per-branch decode cache of B sequences,
+        emptied (the state before the first token)."""
+        import torch
+        cache = torch.empty(max(self.cache_size(B), 1), dtype=torch.uint8, device=torch.device("cuda", self.device))
+        self.reset_cache(cache, B, stream)
+        return cache
+
+    def reset_cache(self, cache, B: int, stream=None):
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream(cache.device)
+        _lib.check(self._lib.msgla_cache_reset(self._h, cache.data_ptr(), B, ctypes.c_void_p(stream.cuda_stream)))
+
+    def step_workspace_size(self, B: int) -> int:
+        n = ctypes.c_size_t()
+        _lib.check(self._lib.msgla_step_workspace_size(self._h, B, ctypes.byref(n)))
+        return n.value
+
+    def step(self, x, t: int, cache, out=None, workspace=None, stream=None):
+        """Layer output at position t for token x (cuda bf16 [B, d]) of every
+        sequence, updating ``cache`` (from new_cache); tokens must come in order
+        t = 0, 1, 2, ... after the cache was emptied."""
+        import torch
+        B, d = x.shape
+        assert d == self.d and x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous()
+        if out is None:
+            out = torch.empty_like(x)
+        if workspace is None:
+            need = self.step_workspace_size(B)
+            if getattr(self, "_step_ws", None) is None or self._step_ws.numel() < need:
+                self._step_ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+            workspace = self._step_ws
+        if stream is None:
+            stream = torch.cuda.current_stream(x.device)
+        _lib.check(self._lib.msgla_step(self._h, cache.data_ptr(), x.data_ptr(), B, t, out.data_ptr(),
+                                        workspace.data_ptr(), workspace.numel(), ctypes.c_void_p(stream.cuda_stream)))
+        return out
+
     def launch_names(self, B: int, L: int):
         """Kernel names of one forward of a [B, L, d] input, in launch order."""
         buf = ctypes.create_string_buffer(512)

@@ -8,7 +8,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from ctypes import POINTER, c_char_p, c_float, c_int, c_size_t, c_void_p
+from ctypes import POINTER, c_char_p, c_float, c_int, c_longlong, c_size_t, c_void_p
 
 MAX_SCALES = 8
 PKG = os.path.dirname(os.path.abspath(__file__))
@@ -57,6 +57,11 @@ _SIGNATURES = {
     "msgla_workspace_tensor": (c_int, [c_void_p, c_int, c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_int)]),
     "msgla_test_skip_arrival": (c_int, [c_void_p, c_int]),
     "msgla_launch_plan": (c_int, [c_void_p, c_int, c_int, c_char_p, c_size_t]),
+    "msgla_cache_size": (c_int, [c_void_p, c_int, POINTER(c_size_t)]),
+    "msgla_cache_reset": (c_int, [c_void_p, c_void_p, c_int, c_void_p]),
+    "msgla_step_workspace_size": (c_int, [c_void_p, c_int, POINTER(c_size_t)]),
+    "msgla_step": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_longlong, c_void_p, c_void_p, c_size_t,
+                           c_void_p]),
     "msgla_status_string": (c_char_p, [c_int]),
     "msgla_last_error": (c_char_p, []),
 }

@@ -1,0 +1,230 @@
+// k_decode.cu -- one token per sequence through the per-branch cache
+// (token-by-token inference of the MS-GLA reading notes, the item on training
+// and per-token inference, after the authors' cache):
+//   dec_pool_kernel  coarse branches add the token to their running block sums;
+//                    a branch whose block of s tokens completes emits the mean
+//                    (Eq. (8)) as an fp16 row for its projection and clears it.
+//   dec_gla_kernel   one GLA step (Sec. 2.1) of a stepping branch: the gate
+//                    alpha from the low-rank projection, S = Diag(alpha) S + k^T v
+//                    on the fp32 state in the cache, o = qk_scale * q S.
+//   dec_fuse_kernel  w = softmax(W_fuse x + b_fuse) from the token itself
+//                    (Eq. (10)) and O = sum_s w_s Y_s over the branches' latest
+//                    outputs (Eq. (11); a coarse branch repeats its output until
+//                    its next block completes, which is the causal hold).
+// The projections and output projections of the stepping branches run on the
+// grouped tcgen05 GEMM with the B sequences as rows.
+#include "msgla_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace msgla {
+namespace {
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 t = __bfloat1622float2(h[e]);
+    f[2 * e] = t.x;
+    f[2 * e + 1] = t.y;
+  }
+}
+
+// one thread per (sequence, 8 columns)
+__global__ void __launch_bounds__(256) dec_pool_kernel(const DecPoolParams p) {
+  const int groups = p.d / 8;
+  const size_t gid = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (gid >= static_cast<size_t>(p.B) * groups) return;
+  const size_t off = gid * 8;  // = b * d + 8 * column group
+  float x[8];
+  bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(p.x + off)), x);
+  bool bad = false;
+  for (int j = 0; j < p.n_scales; ++j) {
+    float* buf = p.buf[j];
+    if (!buf) continue;
+    float4* b4 = reinterpret_cast<float4*>(buf + off);
+    const float4 u0 = b4[0], u1 = b4[1];
+    const float s[8] = {u0.x + x[0], u0.y + x[1], u0.z + x[2], u0.w + x[3],
+                        u1.x + x[4], u1.y + x[5], u1.z + x[6], u1.w + x[7]};
+    if (p.xbar[j]) {
+      const float inv = 1.f / static_cast<float>(p.scales[j]);
+      uint4 o;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a0 = s[2 * e] * inv, a1 = s[2 * e + 1] * inv;
+        bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
+        ow[e] = pack_half2(a0, a1);
+      }
+      *reinterpret_cast<uint4*>(p.xbar[j] + off) = o;
+      b4[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      b4[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      b4[0] = make_float4(s[0], s[1], s[2], s[3]);
+      b4[1] = make_float4(s[4], s[5], s[6], s[7]);
+    }
+  }
+  if (bad) atomicCAS(p.err, 0, kDevRange);
+}
+
+constexpr int kDecTile = 128;  // value columns per CTA
+constexpr int kDecMaxDk = 256;
+
+// One CTA (256 threads) per (sequence, stepping branch, head, 128 value columns).
+// Thread (grp, col): value column col of the tile and half grp of the key channels.
+// Each key channel's state row segment is 128 consecutive floats, so every load
+// and store of the state is one coalesced 512-byte access per channel.
+__global__ void __launch_bounds__(256) dec_gla_kernel(const __grid_constant__ DecGlaParams p) {
+  __shared__ float alpha_s[kDecMaxDk], q_s[kDecMaxDk], k_s[kDecMaxDk];
+  __shared__ float v_s[kDecTile];
+  __shared__ float red[kDecTile];
+  int bi = 0;
+#pragma unroll 1
+  for (int j = 1; j < p.n_branches; ++j)
+    if (static_cast<int>(blockIdx.x) >= p.br[j].cta_begin) bi = j;
+  const DecGlaBranch& P = p.br[bi];
+  const int v_tiles = p.dvp / kDecTile;
+  int local = blockIdx.x - P.cta_begin;
+  const int vt = local % v_tiles;
+  local /= v_tiles;
+  const int head = local % P.heads;
+  const int b = local / P.heads;
+  const int dkp = p.dkp, rp = p.rp;
+  const size_t qk_row = static_cast<size_t>(b) * P.heads * dkp + static_cast<size_t>(head) * dkp;
+  const size_t v_row = static_cast<size_t>(b) * P.heads * p.dvp + static_cast<size_t>(head) * p.dvp + vt * kDecTile;
+
+  // gate, q and k of every key channel of this head
+  for (int c = threadIdx.x; c < dkp; c += blockDim.x) {
+    const float* w = P.Wg2 + (static_cast<size_t>(head) * dkp + c) * rp;
+    const float* g = P.g + static_cast<size_t>(b) * rp;
+    float z = __ldg(P.bg + head * dkp + c);
+    for (int r = 0; r < rp; ++r) z = fmaf(__ldg(g + r), __ldg(w + r), z);
+    // logsigmoid(z) = min(z, 0) - log(1 + e^{-|z|})
+    const float la = (fminf(z, 0.f) - __logf(1.f + __expf(-fabsf(z)))) * p.inv_normalizer;
+    alpha_s[c] = __expf(la);
+    q_s[c] = __half2float(P.q[qk_row + c]);
+    k_s[c] = __half2float(P.k[qk_row + c]);
+  }
+  if (threadIdx.x < kDecTile) v_s[threadIdx.x] = __half2float(P.v[v_row + threadIdx.x]);
+  __syncthreads();
+
+  const int col = threadIdx.x & (kDecTile - 1), grp = threadIdx.x / kDecTile;
+  const int half = dkp / 2;
+  const int c0 = grp * half;
+  float* S = P.S + ((static_cast<size_t>(b) * P.heads + head) * dkp + c0) * p.dvp + vt * kDecTile + col;
+  const float vc = v_s[col];
+  float acc = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < half; c += 8) {
+    float s[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s[e] = S[static_cast<size_t>(c + e) * p.dvp];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int ch = c0 + c + e;
+      s[e] = fmaf(alpha_s[ch], s[e], k_s[ch] * vc);
+      acc = fmaf(q_s[ch], s[e], acc);
+      S[static_cast<size_t>(c + e) * p.dvp] = s[e];
+    }
+  }
+  if (grp == 1) red[col] = acc;
+  __syncthreads();
+  if (grp == 0) {
+    const float o = p.qk_scale * (acc + red[col]);
+    if (!(fabsf(o) <= 65504.f)) atomicCAS(p.err, 0, kDevRange);
+    P.o[v_row + col] = __float2half_rn(o);
+  }
+}
+
+// One CTA (256 threads) per sequence: fusion logits from the token, softmax,
+// then the weighted sum of the branches' latest outputs, 8 columns per thread.
+__global__ void __launch_bounds__(256) dec_fuse_kernel(const DecFuseParams p) {
+  __shared__ float red[8][kMaxScales];
+  __shared__ float w_s[kMaxScales];
+  const int b = blockIdx.x;
+  const int groups = p.d / 8;
+  const int ns = p.n_scales;
+  const __nv_bfloat16* xb = p.x + static_cast<size_t>(b) * p.d;
+  float part[kMaxScales];
+#pragma unroll
+  for (int j = 0; j < kMaxScales; ++j) part[j] = 0.f;
+  for (int cg = threadIdx.x; cg < groups; cg += blockDim.x) {
+    float x[8];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xb) + cg), x);
+#pragma unroll
+    for (int j = 0; j < kMaxScales; ++j) {
+      if (j >= ns) break;
+      float w[8];
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(p.Wfuse + static_cast<size_t>(j) * p.d) + cg), w);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part[j] = fmaf(x[e], w[e], part[j]);
+    }
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int j = 0; j < kMaxScales; ++j) {
+    float v = part[j];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0) red[warp][j] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float z[kMaxScales], zmax = -INFINITY;
+    for (int j = 0; j < ns; ++j) {
+      z[j] = (p.bfuse ? p.bfuse[j] : 0.f);
+      for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) z[j] += red[w][j];
+      zmax = fmaxf(zmax, z[j]);
+    }
+    float sum = 0.f;
+    for (int j = 0; j < ns; ++j) {
+      z[j] = __expf(z[j] - zmax);
+      sum += z[j];
+    }
+    for (int j = 0; j < ns; ++j) w_s[j] = z[j] / sum;
+  }
+  __syncthreads();
+  for (int cg = threadIdx.x; cg < groups; cg += blockDim.x) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < ns; ++j) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(p.Y[j] + static_cast<size_t>(b) * p.d) + cg);
+      const __half2* h = reinterpret_cast<const __half2*>(&u);
+      const float wj = w_s[j];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        acc[2 * e] = fmaf(wj, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(wj, f.y, acc[2 * e + 1]);
+      }
+    }
+    uint4 o;
+    o.x = pack_bf162(acc[0], acc[1]);
+    o.y = pack_bf162(acc[2], acc[3]);
+    o.z = pack_bf162(acc[4], acc[5]);
+    o.w = pack_bf162(acc[6], acc[7]);
+    reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.d)[cg] = o;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dec_pool(const DecPoolParams& p, cudaStream_t st) {
+  const size_t n = static_cast<size_t>(p.B) * (p.d / 8);
+  if (n == 0) return cudaSuccess;
+  dec_pool_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dec_gla(const DecGlaParams& p, cudaStream_t st) {
+  if (p.total_ctas <= 0) return cudaSuccess;
+  if (p.dkp > kDecMaxDk || p.dkp % 16 || p.dvp % kDecTile) return cudaErrorInvalidValue;
+  dec_gla_kernel<<<p.total_ctas, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dec_fuse(const DecFuseParams& p, cudaStream_t st) {
+  if (p.B <= 0) return cudaSuccess;
+  dec_fuse_kernel<<<p.B, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace msgla

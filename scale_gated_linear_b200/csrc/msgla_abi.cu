@@ -650,6 +650,220 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   return MSGLA_OK;
 }
 
+// ---------------------------------------------------------------- decode step
+// Cache (caller-owned, zeroed by msgla_cache_reset), per branch j:
+//   S fp32 [B, h, dkp, dvp] GLA state; for s > 1 also buf fp32 [B, d] (sum of the
+//   tokens of the unfinished block) and Y fp16 [B, d] (latest branch output).
+struct CacheLayout {
+  Region S[MSGLA_MAX_SCALES], buf[MSGLA_MAX_SCALES], Y[MSGLA_MAX_SCALES];
+  size_t total = 0;
+};
+CacheLayout cache_layout(const msgla_handle* h, int B) {
+  CacheLayout c;
+  size_t cur = 0;
+  const size_t BB = static_cast<size_t>(B);
+  for (int j = 0; j < h->n_scales; ++j) {
+    add(c.S[j], cur, BB * h->br[j].heads * h->dkp * h->dvp * 4);
+    if (h->br[j].scale > 1) {
+      add(c.buf[j], cur, BB * h->cfg.d * 4);
+      add(c.Y[j], cur, BB * h->cfg.d * 2);
+    }
+  }
+  c.total = cur;
+  return c;
+}
+
+// Step workspace: per branch the pooled row (s > 1), q, k, v, g, o; Y of the scale-1 branch.
+struct StepLayout {
+  Region xbar[MSGLA_MAX_SCALES], q[MSGLA_MAX_SCALES], k[MSGLA_MAX_SCALES], v[MSGLA_MAX_SCALES],
+      g[MSGLA_MAX_SCALES], o[MSGLA_MAX_SCALES];
+  Region Y1;
+  size_t total = 0;
+};
+StepLayout step_layout(const msgla_handle* h, int B) {
+  StepLayout w;
+  size_t cur = 0;
+  const size_t BB = static_cast<size_t>(B);
+  for (int j = 0; j < h->n_scales; ++j) {
+    const int hh = h->br[j].heads;
+    if (h->br[j].scale > 1) add(w.xbar[j], cur, BB * h->cfg.d * 2);
+    add(w.q[j], cur, BB * hh * h->dkp * 2);
+    add(w.k[j], cur, BB * hh * h->dkp * 2);
+    add(w.v[j], cur, BB * hh * h->dvp * 2);
+    add(w.g[j], cur, BB * h->rp * 4);
+    add(w.o[j], cur, BB * hh * h->dvp * 2);
+  }
+  if (h->main_index >= 0) add(w.Y1, cur, BB * h->cfg.d * 2);
+  w.total = cur;
+  return w;
+}
+
+int step_impl(msgla_handle* h, void* cache, const void* x, int B, long long t, void* O, void* wsp,
+              cudaStream_t st) {
+  const msgla_config& c = h->cfg;
+  const int d = c.d, ns = h->n_scales;
+  const CacheLayout cl = cache_layout(h, B);
+  const StepLayout sl = step_layout(h, B);
+  uint8_t* cb = static_cast<uint8_t*>(cache);
+  uint8_t* wb = static_cast<uint8_t*>(wsp);
+  auto cat = [&](const Region& r) { return static_cast<void*>(cb + r.off); };
+  auto wat = [&](const Region& r) { return static_cast<void*>(wb + r.off); };
+  bool fires[MSGLA_MAX_SCALES];
+  bool any_fires = false;
+  for (int j = 0; j < ns; ++j) {
+    fires[j] = (t + 1) % h->br[j].scale == 0;  // the branch's block ends at this token
+    any_fires |= fires[j];
+  }
+
+  // 1. running block sums of the coarse branches; pooled rows of those that step
+  if (h->main_index < 0 || ns > 1) {
+    DecPoolParams pp{};
+    pp.x = static_cast<const __nv_bfloat16*>(x);
+    pp.B = B;
+    pp.d = d;
+    pp.n_scales = ns;
+    pp.err = h->d_err;
+    for (int j = 0; j < ns; ++j) {
+      pp.scales[j] = h->br[j].scale;
+      if (h->br[j].scale == 1) continue;
+      pp.buf[j] = static_cast<float*>(cat(cl.buf[j]));
+      pp.xbar[j] = fires[j] ? static_cast<__half*>(wat(sl.xbar[j])) : nullptr;
+    }
+    CUDA_TRY(launch_dec_pool(pp, st));
+  }
+
+  if (any_fires) {
+    // 2. projections of the stepping branches (grouped GEMM, the B sequences as rows)
+    static thread_local GemmParams gp;
+    memset(&gp, 0, sizeof(gp));
+    gp.err = h->d_err;
+    int tiles = 0, nt = 0;
+    for (int j = 0; j < ns; ++j) {
+      if (!fires[j]) continue;
+      const Branch& b = h->br[j];
+      const bool bf = (b.scale == 1);
+      GemmTask& tk = gp.task[nt++];
+      if (!encode_3d(&tk.tmA, bf, bf ? x : wat(sl.xbar[j]), d, B, 1, kGemmBM) ||
+          !encode_2d(&tk.tmB, bf, b.Bproj, d, b.np, 128))
+        return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (step projection, scale %d)", b.scale);
+      tk.rows = B;
+      tk.m_tiles = ceil_div(B, kGemmBM);
+      tk.n_tiles = ceil_div(b.np, 256);
+      tk.N = b.np;
+      tk.K = d;
+      tk.tile_begin = tiles;
+      tk.ab_bf16 = bf ? 1 : 0;
+      tk.epi = kEpiProj;
+      tk.nq = tk.nk = b.heads * h->dkp;
+      tk.nv = b.heads * h->dvp;
+      tk.ng = h->rp;
+      tk.nz = 0;  // the step forms the fusion logits itself
+      tk.ldz = h->ldz;
+      tk.q = static_cast<__half*>(wat(sl.q[j]));
+      tk.k = static_cast<__half*>(wat(sl.k[j]));
+      tk.v = static_cast<__half*>(wat(sl.v[j]));
+      tk.g = static_cast<float*>(wat(sl.g[j]));
+      tiles += tk.m_tiles * tk.n_tiles;
+    }
+    gp.n_tasks = nt;
+    gp.total_tiles = tiles;
+    CUDA_TRY(launch_gemm(gp, 256, st));
+
+    // 3. one GLA step per stepping branch and head
+    DecGlaParams dp{};
+    int ctas = 0, nb = 0;
+    for (int j = 0; j < ns; ++j) {
+      if (!fires[j]) continue;
+      const Branch& b = h->br[j];
+      DecGlaBranch& q = dp.br[nb++];
+      q.q = static_cast<const __half*>(wat(sl.q[j]));
+      q.k = static_cast<const __half*>(wat(sl.k[j]));
+      q.v = static_cast<const __half*>(wat(sl.v[j]));
+      q.g = static_cast<const float*>(wat(sl.g[j]));
+      q.Wg2 = b.Wg2p;
+      q.bg = b.bgp;
+      q.S = static_cast<float*>(cat(cl.S[j]));
+      q.o = static_cast<__half*>(wat(sl.o[j]));
+      q.heads = b.heads;
+      q.cta_begin = ctas;
+      ctas += B * b.heads * (h->dvp / kGlaTile);
+    }
+    dp.n_branches = nb;
+    dp.total_ctas = ctas;
+    dp.dkp = h->dkp;
+    dp.dvp = h->dvp;
+    dp.rp = h->rp;
+    dp.inv_normalizer = 1.f / c.gate_normalizer;
+    dp.qk_scale = c.qk_scale;
+    dp.err = h->d_err;
+    CUDA_TRY(launch_dec_gla(dp, st));
+
+    // 3b. optional per-head RMS norm of o
+    if (c.head_norm) {
+      HeadNormParams np{};
+      long long warps = 0;
+      int n = 0;
+      for (int j = 0; j < ns; ++j) {
+        if (!fires[j]) continue;
+        HeadNormBranch& q = np.br[n++];
+        q.o = static_cast<__half*>(wat(sl.o[j]));
+        q.w = h->br[j].normw;
+        q.rows = B;
+        q.heads = h->br[j].heads;
+        q.warp_begin = warps;
+        warps += q.rows * q.heads;
+      }
+      np.n_branches = n;
+      np.total_warps = warps;
+      np.dvp = h->dvp;
+      np.dv = c.d_v;
+      np.eps = c.head_norm_eps;
+      np.err = h->d_err;
+      CUDA_TRY(launch_head_norm(np, st));
+    }
+
+    // 4. output projections: coarse outputs replace the cached ones
+    memset(&gp, 0, sizeof(gp));
+    gp.err = h->d_err;
+    tiles = nt = 0;
+    for (int j = 0; j < ns; ++j) {
+      if (!fires[j]) continue;
+      const Branch& b = h->br[j];
+      GemmTask& tk = gp.task[nt++];
+      if (!encode_3d(&tk.tmA, false, wat(sl.o[j]), b.heads * h->dvp, B, 1, kGemmBM) ||
+          !encode_2d(&tk.tmB, false, b.Wop, b.heads * h->dvp, d, 128))
+        return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (step output, scale %d)", b.scale);
+      tk.rows = B;
+      tk.m_tiles = ceil_div(B, kGemmBM);
+      tk.n_tiles = ceil_div(d, 256);
+      tk.N = d;
+      tk.K = b.heads * h->dvp;
+      tk.tile_begin = tiles;
+      tk.ab_bf16 = 0;
+      tk.epi = kEpiStoreF16;
+      tk.y = static_cast<__half*>(b.scale == 1 ? wat(sl.Y1) : cat(cl.Y[j]));
+      tiles += tk.m_tiles * tk.n_tiles;
+    }
+    gp.n_tasks = nt;
+    gp.total_tiles = tiles;
+    CUDA_TRY(launch_gemm(gp, 256, st));
+  }
+
+  // 5. fusion of the branches' latest outputs
+  DecFuseParams fp{};
+  fp.x = static_cast<const __nv_bfloat16*>(x);
+  fp.Wfuse = h->Wfuse;
+  fp.bfuse = h->bfuse;
+  for (int j = 0; j < ns; ++j)
+    fp.Y[j] = static_cast<const __half*>(h->br[j].scale == 1 ? wat(sl.Y1) : cat(cl.Y[j]));
+  fp.out = static_cast<__nv_bfloat16*>(O);
+  fp.B = B;
+  fp.d = d;
+  fp.n_scales = ns;
+  CUDA_TRY(launch_dec_fuse(fp, st));
+  return MSGLA_OK;
+}
+
 int check_forward_args(const msgla_handle* h, int B, int L) {
   if (!h) return fail(MSGLA_ERR_INVALID_ARG, "handle is NULL");
   if (B < 0 || L < 0) return fail(MSGLA_ERR_INVALID_ARG, "B=%d, L=%d must be >= 0", B, L);
@@ -942,6 +1156,56 @@ int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index,
   dims[1] = bw.rows;
   dims[2] = cols;
   return MSGLA_OK;
+}
+
+int msgla_cache_size(const msgla_handle* h, int B, size_t* bytes) {
+  if (!h || !bytes) return fail(MSGLA_ERR_INVALID_ARG, "NULL argument");
+  if (B < 0 || B > 65535) return fail(MSGLA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
+  *bytes = cache_layout(h, B).total;
+  return MSGLA_OK;
+}
+
+int msgla_cache_reset(msgla_handle* h, void* cache, int B, void* stream) {
+  if (!h) return fail(MSGLA_ERR_INVALID_ARG, "handle is NULL");
+  if (B < 0 || B > 65535) return fail(MSGLA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
+  const size_t n = cache_layout(h, B).total;
+  if (n == 0) return MSGLA_OK;
+  if (!cache || reinterpret_cast<uintptr_t>(cache) % 256)
+    return fail(MSGLA_ERR_INVALID_ARG, "cache is NULL or not 256-byte aligned");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
+  CUDA_TRY(cudaMemsetAsync(cache, 0, n, static_cast<cudaStream_t>(stream)));
+  return MSGLA_OK;
+}
+
+int msgla_step_workspace_size(const msgla_handle* h, int B, size_t* bytes) {
+  if (!h || !bytes) return fail(MSGLA_ERR_INVALID_ARG, "NULL argument");
+  if (B < 0 || B > 65535) return fail(MSGLA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
+  *bytes = step_layout(h, B).total;
+  return MSGLA_OK;
+}
+
+int msgla_step(msgla_handle* h, void* cache, const void* x, int B, long long t, void* O, void* workspace,
+               size_t workspace_bytes, void* stream) {
+  if (!h) return fail(MSGLA_ERR_INVALID_ARG, "handle is NULL");
+  if (B < 0 || B > 65535) return fail(MSGLA_ERR_INVALID_ARG, "B=%d outside [0, 65535]", B);
+  if (t < 0) return fail(MSGLA_ERR_INVALID_ARG, "t=%lld must be >= 0", t);
+  if (B == 0) return MSGLA_OK;
+  if (!cache || !x || !O) return fail(MSGLA_ERR_INVALID_ARG, "cache, x or O is NULL");
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(O) % 16)
+    return fail(MSGLA_ERR_INVALID_ARG, "x and O must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(cache) % 256) return fail(MSGLA_ERR_INVALID_ARG, "cache not 256-byte aligned");
+  const size_t need = step_layout(h, B).total;
+  if (!workspace || workspace_bytes < need)
+    return fail(MSGLA_ERR_WORKSPACE, "step workspace of %zu bytes, %zu needed", workspace_bytes, need);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(MSGLA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  const size_t nb = static_cast<size_t>(B) * h->cfg.d * 2;
+  const uint8_t* x0 = static_cast<const uint8_t*>(x);
+  const uint8_t* o0 = static_cast<const uint8_t*>(O);
+  if (x0 < o0 + nb && o0 < x0 + nb) return fail(MSGLA_ERR_INVALID_ARG, "O overlaps x");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
+  return step_impl(h, cache, x, B, t, O, workspace, static_cast<cudaStream_t>(stream));
 }
 
 int msgla_launch_plan(const msgla_handle* h, int B, int L, char* names, size_t len) {

@@ -157,6 +157,51 @@ struct HoldFuseParams {
 };
 cudaError_t launch_hold_fuse(const HoldFuseParams& p, cudaStream_t st);
 
+// ---------------------------------------------------------------- decode step
+// One token of each of B sequences (all at the same position t).
+// Coarse branches: buf += x; a branch whose block completes at t writes its fp16
+// pooled row xbar = buf / s and clears buf.
+struct DecPoolParams {
+  const __nv_bfloat16* x;      // [B, d]
+  float* buf[kMaxScales];      // [B, d] running sums (null for scale 1)
+  __half* xbar[kMaxScales];    // [B, d] pooled row of a branch that steps at t, else null
+  int scales[kMaxScales];
+  int B, d, n_scales;
+  int* err;
+};
+// One GLA step per (sequence, stepping branch, head, 128 value columns):
+// alpha = exp(logsigmoid(g W_g2^T + b_g) / normalizer), S = Diag(alpha) S + k^T v,
+// o = qk_scale * q S.
+struct DecGlaBranch {
+  const __half* q;   // [B, h*dkp]
+  const __half* k;   // [B, h*dkp]
+  const __half* v;   // [B, h*dvp]
+  const float* g;    // [B, rp]
+  const float* Wg2;  // [h*dkp, rp]
+  const float* bg;   // [h*dkp]
+  float* S;          // [B, h, dkp, dvp] state in the cache
+  __half* o;         // [B, h*dvp]
+  int heads, cta_begin;
+};
+struct DecGlaParams {
+  DecGlaBranch br[kMaxScales];
+  int n_branches, total_ctas, dkp, dvp, rp;
+  float inv_normalizer, qk_scale;
+  int* err;
+};
+// w = softmax(W_fuse x + b_fuse), O = sum_s w_s Y_s (one CTA per sequence)
+struct DecFuseParams {
+  const __nv_bfloat16* x;      // [B, d]
+  const __nv_bfloat16* Wfuse;  // [n_scales, d]
+  const float* bfuse;          // [n_scales]
+  const __half* Y[kMaxScales]; // [B, d] latest output of each branch
+  __nv_bfloat16* out;          // [B, d]
+  int B, d, n_scales;
+};
+cudaError_t launch_dec_pool(const DecPoolParams& p, cudaStream_t st);
+cudaError_t launch_dec_gla(const DecGlaParams& p, cudaStream_t st);
+cudaError_t launch_dec_fuse(const DecFuseParams& p, cudaStream_t st);
+
 // bf16 -> fp16 with an overflow count; bf16 -> bf16 copy into a strided block
 cudaError_t launch_bf16_to_f16_rows(const __nv_bfloat16* src, int src_ld, int rows, int cols, __half* dst,
                                     int dst_ld, int* overflow, cudaStream_t st);

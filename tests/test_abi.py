@@ -81,6 +81,10 @@ def test_null_arguments():
     assert lib.msgla_workspace_size(None, 1, 1, ctypes.byref(n)) == -1
     assert lib.msgla_forward(None, None, 1, 1, None, None, 0, None) == -1
     assert lib.msgla_forward_masked(None, None, None, 1, 1, None, None, 0, None) == -1
+    assert lib.msgla_cache_size(None, 1, ctypes.byref(n)) == -1
+    assert lib.msgla_cache_reset(None, None, 1, None) == -1
+    assert lib.msgla_step_workspace_size(None, 1, ctypes.byref(n)) == -1
+    assert lib.msgla_step(None, None, None, 1, 0, None, None, 0, None) == -1
     assert lib.msgla_forward_host(None, None, 1, 1, None, None, 0, None) == -1
     assert lib.msgla_sync_status(None) == -1
     lib.msgla_destroy(None)
