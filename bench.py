@@ -254,6 +254,124 @@ def run_reference(args) -> int:
     return 0
 
 
+# --------------------------------------------------------------------- decode
+def decode_bytes(w, B: int, t: int) -> int:
+    """Algorithmic HBM bytes of the decode step at position t: packed weights of
+    the branches that step (projection rows and W_o, 2 bytes each), their fp32
+    state read and written, every coarse branch's block sum read and written and
+    latest output read, the token in and the output out."""
+    dkp = 128 if w.d_k <= 128 else 256
+    dvp = -(-w.d_v // 128) * 128
+    rp = -(-w.gate_rank // 16) * 16
+    n = 2 * B * w.d * 2 + len(w.scales) * w.d * 2  # x, O, W_fuse
+    for s, h in zip(w.scales, w.heads):
+        if s > 1:
+            n += B * w.d * (4 + 4 + 2)
+        if (t + 1) % s == 0:
+            n += (h * (2 * dkp + dvp) + rp) * w.d * 2 + w.d * h * dvp * 2
+            n += 2 * B * h * dkp * dvp * 4
+    return n
+
+
+def run_decode(args) -> int:
+    import torch
+
+    from scale_gated_linear_b200 import MSGLA
+    from scale_gated_linear_b200 import workloads as wl
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1 and rank > 0:  # decode is measured on one GPU (independent replicas otherwise)
+        return 0
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = wl.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.replace(B=args.batch)
+    if args.head_norm:
+        w = w.replace(head_norm=True)
+    period = 1
+    for s in w.scales:
+        period = period * s // math.gcd(period, s)
+    inp = wl.make_inputs(w, L=period)
+    layer = MSGLA.from_workload(w, inp, device=local)
+    X = inp["X"].to(dev)
+    B = w.B
+    cache = layer.new_cache(B)
+    ws = torch.empty(max(layer.step_workspace_size(B), 1), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, w.d, dtype=torch.bfloat16, device=dev)
+    xs = [X[:, i].contiguous() for i in range(period)]
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    t = 0
+
+    def cycle(st=stream):
+        nonlocal t
+        for i in range(period):
+            layer.step(xs[i], t, cache, out=out, workspace=ws, stream=st)
+            t += 1
+
+    for _ in range(args.warmup):
+        flush_buf.fill_(1)
+        cycle()
+    torch.cuda.synchronize()
+    layer.check_status()
+    graph = None
+    if args.graph:
+        # which branches step depends only on t mod period: one captured cycle
+        # replays every later cycle (the tokens are read from the fixed buffers xs)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cycle(torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
+        layer.check_status()
+    sampler = ClockSampler(None)
+    sampler.start()
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_first = t
+    for k in range(args.steps):
+        flush_buf.fill_(1)
+        ev[k][0].record(stream)
+        if graph is not None:
+            graph.replay()
+            t += period
+        else:
+            cycle()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    layer.check_status()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    tokens = B * period * args.steps
+    nbytes = sum(decode_bytes(w, B, tt) for tt in range(t_first, t_first + period))
+    cyc_ms = total_ms / args.steps
+    peaks, peak_kind = load_peaks()
+    achieved = nbytes / (cyc_ms * 1e-3) / 1e9
+    line = {
+        "metric": "MS-GLA decode tokens/sec (one token per sequence per step)", "value": tokens / (total_ms / 1e3),
+        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": cyc_ms, "tokens_per_step": B * period, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 state, f16/bf16 tensor-core operands; bf16 in/out", "data": "synthetic",
+        "config": {"workload": f"{w.name}: decode of B={B} sequences, one step = {period} tokens (every branch "
+                               f"steps once), d={w.d}, scales {list(w.scales)} heads {list(w.heads)}, "
+                               f"d_k={w.d_k}, d_v={w.d_v}", "l2": "flushed between timed steps (256 MiB write)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "kernel": "whole decode step",
+                     "bytes_per_step": nbytes, "peak_source": peak_kind},
+        "us_per_token_position": 1e3 * cyc_ms / period,
+        "launch": "one CUDA graph per step (captured cycle)" if graph is not None else "eager msgla_step calls",
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    del graph
+    layer.close()
+    return 0
+
+
 # --------------------------------------------------------------------- our arm
 def time_layer(layer, X, O, ws, steps: int, warmup: int, flush, n_events: int, mask=None):
     import torch
@@ -435,7 +553,12 @@ def main(argv=None) -> int:
                     help="time the masked forward with this valid-token mask")
     ap.add_argument("--head-norm", action="store_true", help="enable the per-head RMS norm of the GLA output")
     ap.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's)")
+    ap.add_argument("--graph", action="store_true", help="with --decode: replay one captured step as a CUDA graph")
+    ap.add_argument("--decode", action="store_true",
+                    help="time token-by-token decode (msgla_step) instead of the whole-sequence forward")
     args = ap.parse_args(argv)
+    if args.decode:
+        return run_decode(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -68,15 +68,19 @@ __global__ void __launch_bounds__(256) dec_pool_kernel(const DecPoolParams p) {
 
 constexpr int kDecTile = 128;  // value columns per CTA
 constexpr int kDecMaxDk = 256;
+constexpr int kDecThreads = 512;
+constexpr int kDecGroups = kDecThreads / 32;  // key-channel groups; a warp covers the 128 columns
 
-// One CTA (256 threads) per (sequence, stepping branch, head, 128 value columns).
-// Thread (grp, col): value column col of the tile and half grp of the key channels.
-// Each key channel's state row segment is 128 consecutive floats, so every load
-// and store of the state is one coalesced 512-byte access per channel.
-__global__ void __launch_bounds__(256) dec_gla_kernel(const __grid_constant__ DecGlaParams p) {
+// One CTA (512 threads) per (sequence, stepping branch, head, 128 value columns).
+// Warp g handles key channels [g*dkp/16, (g+1)*dkp/16), lane l value columns
+// [4l, 4l+4): each key channel's state row segment (512 bytes) is one coalesced
+// warp access, and all of a thread's state (16 x 16 bytes) is loaded before any
+// of it is used, so the whole 128 KB tile is in flight at once. The partial
+// o = q S of the 16 channel groups are summed through shared memory.
+__global__ void __launch_bounds__(kDecThreads) dec_gla_kernel(const __grid_constant__ DecGlaParams p) {
   __shared__ float alpha_s[kDecMaxDk], q_s[kDecMaxDk], k_s[kDecMaxDk];
-  __shared__ float v_s[kDecTile];
-  __shared__ float red[kDecTile];
+  __shared__ __align__(16) float v_s[kDecTile];
+  __shared__ __align__(16) float red[kDecGroups][kDecTile];
   int bi = 0;
 #pragma unroll 1
   for (int j = 1; j < p.n_branches; ++j)
@@ -91,8 +95,17 @@ __global__ void __launch_bounds__(256) dec_gla_kernel(const __grid_constant__ De
   const int dkp = p.dkp, rp = p.rp;
   const size_t qk_row = static_cast<size_t>(b) * P.heads * dkp + static_cast<size_t>(head) * dkp;
   const size_t v_row = static_cast<size_t>(b) * P.heads * p.dvp + static_cast<size_t>(head) * p.dvp + vt * kDecTile;
+  const int grp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per = dkp / kDecGroups;  // 16 (dkp = 256) or 8 (dkp = 128)
+  const int c0 = grp * per;
+  float* S = P.S + ((static_cast<size_t>(b) * P.heads + head) * dkp + c0) * p.dvp + vt * kDecTile + 4 * lane;
 
-  // gate, q and k of every key channel of this head
+  // issue the state loads first; the gate and the small operands follow
+  float4 s[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e)
+    if (e < per) s[e] = *reinterpret_cast<const float4*>(S + static_cast<size_t>(e) * p.dvp);
+
   for (int c = threadIdx.x; c < dkp; c += blockDim.x) {
     const float* w = P.Wg2 + (static_cast<size_t>(head) * dkp + c) * rp;
     const float* g = P.g + static_cast<size_t>(b) * rp;
@@ -107,31 +120,33 @@ __global__ void __launch_bounds__(256) dec_gla_kernel(const __grid_constant__ De
   if (threadIdx.x < kDecTile) v_s[threadIdx.x] = __half2float(P.v[v_row + threadIdx.x]);
   __syncthreads();
 
-  const int col = threadIdx.x & (kDecTile - 1), grp = threadIdx.x / kDecTile;
-  const int half = dkp / 2;
-  const int c0 = grp * half;
-  float* S = P.S + ((static_cast<size_t>(b) * P.heads + head) * dkp + c0) * p.dvp + vt * kDecTile + col;
-  const float vc = v_s[col];
-  float acc = 0.f;
-#pragma unroll 1
-  for (int c = 0; c < half; c += 8) {
-    float s[8];
+  const float4 v4 = *reinterpret_cast<const float4*>(&v_s[4 * lane]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) s[e] = S[static_cast<size_t>(c + e) * p.dvp];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int ch = c0 + c + e;
-      s[e] = fmaf(alpha_s[ch], s[e], k_s[ch] * vc);
-      acc = fmaf(q_s[ch], s[e], acc);
-      S[static_cast<size_t>(c + e) * p.dvp] = s[e];
-    }
+  for (int e = 0; e < 16; ++e) {
+    if (e >= per) break;
+    const int ch = c0 + e;
+    const float a = alpha_s[ch], kk = k_s[ch], qq = q_s[ch];
+    float4 t = s[e];
+    t.x = fmaf(a, t.x, kk * v4.x);
+    t.y = fmaf(a, t.y, kk * v4.y);
+    t.z = fmaf(a, t.z, kk * v4.z);
+    t.w = fmaf(a, t.w, kk * v4.w);
+    acc.x = fmaf(qq, t.x, acc.x);
+    acc.y = fmaf(qq, t.y, acc.y);
+    acc.z = fmaf(qq, t.z, acc.z);
+    acc.w = fmaf(qq, t.w, acc.w);
+    *reinterpret_cast<float4*>(S + static_cast<size_t>(e) * p.dvp) = t;
   }
-  if (grp == 1) red[col] = acc;
+  *reinterpret_cast<float4*>(&red[grp][4 * lane]) = acc;
   __syncthreads();
-  if (grp == 0) {
-    const float o = p.qk_scale * (acc + red[col]);
+  if (threadIdx.x < kDecTile) {
+    float o = 0.f;
+#pragma unroll
+    for (int g2 = 0; g2 < kDecGroups; ++g2) o += red[g2][threadIdx.x];
+    o *= p.qk_scale;
     if (!(fabsf(o) <= 65504.f)) atomicCAS(p.err, 0, kDevRange);
-    P.o[v_row + col] = __float2half_rn(o);
+    P.o[v_row + threadIdx.x] = __float2half_rn(o);
   }
 }
 
@@ -216,8 +231,8 @@ cudaError_t launch_dec_pool(const DecPoolParams& p, cudaStream_t st) {
 
 cudaError_t launch_dec_gla(const DecGlaParams& p, cudaStream_t st) {
   if (p.total_ctas <= 0) return cudaSuccess;
-  if (p.dkp > kDecMaxDk || p.dkp % 16 || p.dvp % kDecTile) return cudaErrorInvalidValue;
-  dec_gla_kernel<<<p.total_ctas, 256, 0, st>>>(p);
+  if ((p.dkp != 128 && p.dkp != 256) || p.dvp % kDecTile) return cudaErrorInvalidValue;
+  dec_gla_kernel<<<p.total_ctas, kDecThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
