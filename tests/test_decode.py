@@ -104,3 +104,50 @@ def test_decode_long_memory_gates():
     got, _ = decode_all(layer, inp["X"].cuda())
     layer.close()
     assert_parity(got, oracle_forward(w, inp))
+
+
+@needs_gpu
+def test_decode_cycle_replays_as_cuda_graph():
+    """Which branches step depends only on t modulo lcm(scales), so one captured
+    cycle of msgla_step calls replays every later cycle: graph replay and eager
+    calls give bit-identical outputs and caches."""
+    from scale_gated_linear_b200 import MSGLA
+    w = SMALL.replace(L=12)
+    inp = gpu_inputs(w)
+    X = inp["X"].cuda()
+    B = w.B
+    period = 4
+    outs_eager = []
+    layer = MSGLA.from_workload(w, inp, device=0)
+    cache = layer.new_cache(B)
+    for t in range(w.L):
+        outs_eager.append(layer.step(X[:, t].contiguous(), t, cache).clone())
+    torch.cuda.synchronize()
+    eager_cache = cache.clone()
+
+    layer.reset_cache(cache, B)
+    xs = [torch.empty(B, w.d, dtype=torch.bfloat16, device="cuda") for _ in range(period)]
+    outs = [torch.empty(B, w.d, dtype=torch.bfloat16, device="cuda") for _ in range(period)]
+    ws = torch.empty(layer.step_workspace_size(B), dtype=torch.uint8, device="cuda")
+    for i in range(period):  # the first cycle runs eagerly (also warms the launch paths)
+        xs[i].copy_(X[:, i])
+        layer.step(xs[i], i, cache, out=outs[i], workspace=ws)
+    got = [o.clone() for o in outs]
+    graph = torch.cuda.CUDAGraph()
+    snapshot = cache.clone()
+    with torch.cuda.graph(graph):
+        for i in range(period):
+            layer.step(xs[i], period + i, cache, out=outs[i], workspace=ws, stream=torch.cuda.current_stream())
+    cache.copy_(snapshot)  # capture does not run the kernels; start the replays from cycle 1
+    for c in range(1, w.L // period):
+        for i in range(period):
+            xs[i].copy_(X[:, c * period + i])
+        graph.replay()
+        got += [o.clone() for o in outs]
+    torch.cuda.synchronize()
+    layer.check_status()
+    del graph
+    layer.close()
+    np.testing.assert_array_equal(torch.stack(got, 1).float().cpu().numpy(),
+                                  torch.stack(outs_eager, 1).float().cpu().numpy())
+    assert torch.equal(cache, eager_cache)
