@@ -403,9 +403,6 @@ constexpr int kGateChannels = 128;  // key channels per CTA
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
 
 // tf32 split of an fp32 value: hi has the top 10 mantissa bits, lo the rest.
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
@@ -428,24 +425,40 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 
 // One CTA per (branch, batch, head, 64-row half of a 128-row GLA chunk, 128 key
 // channels), 256 threads.
+//  0. cp.async stages the half chunk's low-rank gate rows g [64 x RP] and its q
+//     and k rows [64 x 128] (fp16; the 16-byte chunks of a row are XOR-swizzled
+//     by (row / 4) mod 8 so that phase 2 reads them without bank conflicts).
 //  1. z = g W_g2^T for the 64 x 128 block on tensor cores (mma.sync m16n8k8 tf32;
 //     each operand split into tf32 hi + lo parts, three products, so z keeps
-//     fp32-level accuracy), then log alpha = logsigmoid(z + b_g) / normalizer in
-//     registers, stored to shared memory.
-//  2. 64 channel pairs x 4 row groups of 16 rows (q, k staged in shared memory by
-//     cp.async during phase 1): each thread forms the local cumulative sum of log alpha over its rows, adds the
-//     totals of the preceding row groups, and writes Qs = q e^{b - m},
-//     Ks = k e^{m - b}. With b_loc the cumulative sum from the half's first row
-//     and T its total: in the first half b - m = b_loc - T, in the second half
-//     b - m = b_loc (m is the first half's total), so each half needs only its
-//     own rows. Per chunk: gamma = e^{b_last - m}, mid = e^{m}.
+//     fp32-level accuracy), then log alpha = logsigmoid(z + b_g) / normalizer,
+//     kept in base-2 units (times log2 e) in shared memory; rows past the end of
+//     the sequence get 0.
+//  2. Thread (channel group cg of 8 channels, row group rg of 4 rows): the
+//     cumulative sum of log alpha over its 4 rows, the exclusive prefix over the
+//     16 row groups by a 16-lane shuffle scan, and Qs = q 2^{b - m},
+//     Ks = k 2^{m - b} stored 16 bytes at a time. With b_loc the cumulative sum
+//     from the half's first row and T its total: in the first half b - m =
+//     b_loc - T, in the second half b - m = b_loc (m is the first half's total),
+//     so each half needs only its own rows. Per chunk: gamma = e^{b_last - m},
+//     mid = e^{m}.
+constexpr int kGateBlk = 36;  // floats per (channel group, row group) block of log alpha: 4 x 8 + 4 padding
+
 template <int RP>
-__global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_constant__ GateParams p) {
-  constexpr int R = 16, kGroups = kChunk / R, kPairs = kGateChannels / 2;
-  static_assert(kPairs * kGroups == kGateThreads, "thread layout");
-  __shared__ float la_s[kChunk][kGateChannels + 4];  // log alpha (row, channel), padded rows
-  __shared__ float tot[kGroups][kGateChannels];
-  extern __shared__ __align__(16) __half qk_s[];      // [2][64][128]: this CTA's q and k rows
+struct GateSmem {
+  static constexpr int kQK = 2 * kChunk * kGateChannels * 2;              // q, k rows (fp16)
+  static constexpr int kLA = (kGateChannels / 8) * (kChunk / 4) * kGateBlk * 4;
+  static constexpr int kGS = RP + 4;                                      // padded g row (floats)
+  static constexpr int kG = kChunk * kGS * 4;
+  static constexpr int kBytes = kQK + kLA + kG;
+};
+
+template <int RP>
+__global__ void __launch_bounds__(kGateThreads, 3) gate_kernel(const __grid_constant__ GateParams p) {
+  using L = GateSmem<RP>;
+  extern __shared__ __align__(16) uint8_t gate_smem[];
+  __half* qk_s = reinterpret_cast<__half*>(gate_smem);
+  float* la_s = reinterpret_cast<float*>(gate_smem + L::kQK);
+  float* g_s = reinterpret_cast<float*>(gate_smem + L::kQK + L::kLA);
   const int dkp = p.dkp;
   const int cblocks = dkp / kGateChannels;
   int bi = 0;
@@ -459,27 +472,42 @@ __global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_cons
   const int hc = local % P.n_halves;
   const int head = (local / P.n_halves) % P.heads;
   const int b = local / (P.n_halves * P.heads);
-  const int c = hc >> 1, second = hc & 1;
+  const int ci = hc >> 1, second = hc & 1;
   const int n_chunks = (P.n_halves + 1) >> 1;
   const int t0 = hc * kChunk;
   const int nrows = min(kChunk, P.rows - t0);
   const int ldk = P.heads * dkp;
   const int cbase = head * dkp + cb * kGateChannels;  // first channel of this CTA
   const size_t row_base = static_cast<size_t>(b) * P.rows + t0;
+  const int tid = threadIdx.x;
 
-  // ---- the q and k rows of this CTA go to shared memory asynchronously while
-  // phase 1 runs (16-byte copies: 16 per row and tensor)
-  for (int i = threadIdx.x; i < 2 * nrows * 16; i += blockDim.x) {
-    const int tsel = i / (nrows * 16), rem = i % (nrows * 16);
-    const int row = rem >> 4, seg = rem & 15;
-    const __half* src = (tsel ? P.k : P.q) + (row_base + row) * ldk + cbase + seg * 8;
-    cp_async16(qk_s + (tsel * kChunk + row) * kGateChannels + seg * 8, src);
+  // ---- phase 0: g rows (group 0), then q and k rows (group 1)
+  constexpr int kGChunks = kChunk * RP / 4;
+  for (int i = tid; i < kGChunks; i += kGateThreads) {
+    const int row = i / (RP / 4), seg = i % (RP / 4);
+    float* dst = g_s + row * L::kGS + seg * 4;
+    if (row < nrows)
+      cp_async16(dst, P.g + (row_base + row) * RP + seg * 4);
+    else
+      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+#pragma unroll
+  for (int it = 0; it < 2 * kChunk * 16 / kGateThreads; ++it) {
+    const int flat = tid + it * kGateThreads;
+    const int tsel = flat >> 10, row = (flat >> 4) & (kChunk - 1), seg = flat & 15;
+    if (row < nrows) {
+      const __half* src = (tsel ? P.k : P.q) + (row_base + row) * ldk + cbase + seg * 8;
+      cp_async16(qk_s + (tsel * kChunk + row) * kGateChannels + ((seg ^ ((row >> 2) & 7)) * 8), src);
+    }
+  }
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 1;" ::: "memory");
+  __syncthreads();
 
   // ---- phase 1: z = g W^T on tensor cores. Warp w owns channels [16w, 16w+16)
   // (two n8 tiles) for all 64 rows (four m16 tiles); K = RP in steps of 8.
   {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
     float acc[4][2][4];
 #pragma unroll
@@ -488,7 +516,6 @@ __global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_cons
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-    const float* gsrc = P.g + row_base * RP;
 #pragma unroll
     for (int k8 = 0; k8 < RP / 8; ++k8) {
       // B fragments: W[channel][k]; b0 = (k = tq, n = gq), b1 = (k = tq + 4, n = gq)
@@ -502,16 +529,13 @@ __global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_cons
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
         // A fragments: g[row][k]; a0 = (gq, tq), a1 = (gq + 8, tq), a2 = (gq, tq + 4), a3 = (gq + 8, tq + 4)
-        const int ra = mt * 16 + gq, rb = ra + 8;
-        const float* g0 = gsrc + static_cast<size_t>(ra) * RP + k8 * 8;
-        const float* g1 = gsrc + static_cast<size_t>(rb) * RP + k8 * 8;
-        const float x0 = ra < nrows ? __ldg(g0 + tq) : 0.f, x1 = rb < nrows ? __ldg(g1 + tq) : 0.f;
-        const float x2 = ra < nrows ? __ldg(g0 + tq + 4) : 0.f, x3 = rb < nrows ? __ldg(g1 + tq + 4) : 0.f;
+        const float* g0 = g_s + (mt * 16 + gq) * L::kGS + k8 * 8;
+        const float* g1 = g0 + 8 * L::kGS;
         uint32_t ah[4], al[4];
-        split_tf32(x0, ah[0], al[0]);
-        split_tf32(x1, ah[1], al[1]);
-        split_tf32(x2, ah[2], al[2]);
-        split_tf32(x3, ah[3], al[3]);
+        split_tf32(g0[tq], ah[0], al[0]);
+        split_tf32(g1[tq], ah[1], al[1]);
+        split_tf32(g0[tq + 4], ah[2], al[2]);
+        split_tf32(g1[tq + 4], ah[3], al[3]);
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           mma_tf32(acc[mt][nt], al, bh[nt]);
@@ -520,8 +544,9 @@ __global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_cons
         }
       }
     }
-    // log alpha into shared memory; D fragment: d0 = (gq, 2tq), d1 = (gq, 2tq+1),
-    // d2 = (gq+8, 2tq), d3 = (gq+8, 2tq+1)
+    // log alpha (base 2) into the blocked layout; D fragment: d0 = (gq, 2tq),
+    // d1 = (gq, 2tq+1), d2 = (gq+8, 2tq), d3 = (gq+8, 2tq+1)
+    const float scale = p.inv_normalizer * 1.4426950408889634f;  // 1/normalizer * log2(e)
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const int chl = warp * 16 + nt * 8 + 2 * tq;
@@ -530,87 +555,98 @@ __global__ void __launch_bounds__(kGateThreads, 2) gate_kernel(const __grid_cons
       for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
+          const int row = mt * 16 + gq + ((e & 2) ? 8 : 0), ch = chl + (e & 1);
           const float z = acc[mt][nt][e] + ((e & 1) ? bias1 : bias0);
           // logsigmoid(z) = min(z, 0) - log(1 + e^{-|z|}); the log argument lies in (1, 2]
-          const float la = (fminf(z, 0.f) - __logf(1.f + __expf(-fabsf(z)))) * p.inv_normalizer;
-          la_s[mt * 16 + gq + ((e & 2) ? 8 : 0)][chl + (e & 1)] = la;
+          const float la = (fminf(z, 0.f) - __logf(1.f + __expf(-fabsf(z)))) * scale;
+          la_s[((ch >> 3) * (kChunk / 4) + (row >> 2)) * kGateBlk + (row & 3) * 8 + (ch & 7)] =
+              row < nrows ? la : 0.f;
         }
       }
     }
   }
-  cp_async_wait_all();
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
-  // ---- phase 2: cumulative sums along rows and the scaled operands
-  const int pair = threadIdx.x % kPairs, grp = threadIdx.x / kPairs;
-  const int a0 = 2 * pair;
-  const int r0 = grp * R;
-  float c0[R], c1[R];
-  float run0 = 0.f, run1 = 0.f;
+  // ---- phase 2: warp w holds channel groups 2w (lanes 0-15) and 2w+1 (lanes
+  // 16-31); lane rg of a 16-lane segment holds rows [4rg, 4rg+4).
+  const int lane = tid & 31;
+  const int cg = 2 * (tid >> 5) + (lane >> 4), rg = lane & 15;
+  const float* blk = la_s + (cg * (kChunk / 4) + rg) * kGateBlk;
+  float c[4][8];
+  float run[8];
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    if (r0 + r < nrows) {
-      const float2 l2 = *reinterpret_cast<const float2*>(&la_s[r0 + r][a0]);
-      run0 += l2.x;
-      run1 += l2.y;
+  for (int e = 0; e < 8; ++e) run[e] = 0.f;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float4 x0 = *reinterpret_cast<const float4*>(blk + r * 8);
+    const float4 x1 = *reinterpret_cast<const float4*>(blk + r * 8 + 4);
+    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      run[e] += x[e];
+      c[r][e] = run[e];
     }
-    c0[r] = run0;
-    c1[r] = run1;
   }
-  tot[grp][a0] = run0;
-  tot[grp][a0 + 1] = run1;
-  __syncthreads();
-  float pre0 = 0.f, pre1 = 0.f, all0 = 0.f, all1 = 0.f;
+  // exclusive prefix over the row groups before this one, and the half's total
+  float pre[8], tot[8];
 #pragma unroll
-  for (int g2 = 0; g2 < kGroups; ++g2) {
-    const float x0 = tot[g2][a0], x1 = tot[g2][a0 + 1];
-    if (g2 < grp) {
-      pre0 += x0;
-      pre1 += x1;
+  for (int e = 0; e < 8; ++e) {
+    float v = run[e];
+#pragma unroll
+    for (int off = 1; off < 16; off <<= 1) {
+      const float u = __shfl_up_sync(0xffffffffu, v, off, 16);
+      if (rg >= off) v += u;
     }
-    all0 += x0;
-    all1 += x1;
+    pre[e] = v - run[e];
+    tot[e] = __shfl_sync(0xffffffffu, v, 15, 16);
   }
   // reference: b - m = b_loc - T in the first half, b_loc in the second
-  pre0 -= second ? 0.f : all0;
-  pre1 -= second ? 0.f : all1;
-  bool bad = false;
-  __half* qrow = P.qs + (row_base + r0) * ldk + cbase + a0;
-  __half* krow = P.ks + (row_base + r0) * ldk + cbase + a0;
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    if (r0 + r < nrows) {
-      const float b0 = pre0 + c0[r], b1 = pre1 + c1[r];
-      const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(qk_s + (r0 + r) * kGateChannels + a0));
-      const float2 kf =
-          __half22float2(*reinterpret_cast<const __half2*>(qk_s + (kChunk + r0 + r) * kGateChannels + a0));
-      const float ks0 = kf.x * __expf(-b0), ks1 = kf.y * __expf(-b1);
-      const float qs0 = qf.x * __expf(b0), qs1 = qf.y * __expf(b1);
-      bad |= fmaxf(fmaxf(fabsf(ks0), fabsf(ks1)), fmaxf(fabsf(qs0), fabsf(qs1))) > 65504.f;
-      *reinterpret_cast<__half2*>(qrow + static_cast<size_t>(r) * ldk) = __floats2half2_rn(qs0, qs1);
-      *reinterpret_cast<__half2*>(krow + static_cast<size_t>(r) * ldk) = __floats2half2_rn(ks0, ks1);
+  for (int e = 0; e < 8; ++e) pre[e] -= second ? 0.f : tot[e];
+
+  float mx = 0.f;
+  const int sw = rg & 7;  // (row >> 2) & 7 for all four rows of this thread
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int row = 4 * rg + r;
+    if (row >= nrows) break;
+    const uint4 qv = *reinterpret_cast<const uint4*>(qk_s + row * kGateChannels + ((cg ^ sw) * 8));
+    const uint4 kv = *reinterpret_cast<const uint4*>(qk_s + (kChunk + row) * kGateChannels + ((cg ^ sw) * 8));
+    const __half2* qh = reinterpret_cast<const __half2*>(&qv);
+    const __half2* kh = reinterpret_cast<const __half2*>(&kv);
+    uint4 qo, ko;
+    uint32_t* qw = reinterpret_cast<uint32_t*>(&qo);
+    uint32_t* kw = reinterpret_cast<uint32_t*>(&ko);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float b0 = pre[2 * e] + c[r][2 * e], b1 = pre[2 * e + 1] + c[r][2 * e + 1];
+      const float2 qf = __half22float2(qh[e]), kf = __half22float2(kh[e]);
+      const float qs0 = qf.x * exp2f(b0), qs1 = qf.y * exp2f(b1);
+      const float ks0 = kf.x * exp2f(-b0), ks1 = kf.y * exp2f(-b1);
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(qs0), fabsf(qs1)), fmaxf(fabsf(ks0), fabsf(ks1))));
+      qw[e] = pack_half2(qs0, qs1);
+      kw[e] = pack_half2(ks0, ks1);
     }
+    const size_t go = (row_base + row) * ldk + cbase + cg * 8;
+    *reinterpret_cast<uint4*>(P.qs + go) = qo;
+    *reinterpret_cast<uint4*>(P.ks + go) = ko;
   }
-  if (grp == 0) {
-    const size_t gi = (static_cast<size_t>(b) * n_chunks + c) * ldk + cbase + a0;
-    if (second) {
-      P.gamma[gi] = __expf(all0);
-      P.gamma[gi + 1] = __expf(all1);
-    } else {
-      P.mid[gi] = __expf(all0);
-      P.mid[gi + 1] = __expf(all1);
-      if (hc + 1 >= P.n_halves) {  // chunk without a second half: b_last = m
-        P.gamma[gi] = 1.f;
-        P.gamma[gi + 1] = 1.f;
-      }
-    }
+  if (!(mx <= 65504.f)) atomicCAS(p.err, 0, kDevRange);
+  if (rg == 15) {
+    const size_t gi = (static_cast<size_t>(b) * n_chunks + ci) * ldk + cbase + cg * 8;
+    float* dst = second ? P.gamma : P.mid;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dst[gi + e] = exp2f(tot[e]);
+    if (!second && hc + 1 >= P.n_halves)  // chunk without a second half: b_last = m
+#pragma unroll
+      for (int e = 0; e < 8; ++e) P.gamma[gi + e] = 1.f;
   }
-  if (bad) atomicCAS(p.err, 0, kDevRange);
 }
 
 template <int RP>
 cudaError_t launch_gate_t(const GateParams& p, cudaStream_t st) {
-  const int smem = 2 * kChunk * kGateChannels * static_cast<int>(sizeof(__half));
+  const int smem = GateSmem<RP>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(gate_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   gate_kernel<RP><<<p.total_blocks, kGateThreads, smem, st>>>(p);
