@@ -10,7 +10,10 @@
 //               accumulators (2 x BN columns)
 //   warps 2..9  epilogue of the other accumulator (tcgen05.ld, one row per thread,
 //               two warps per TMEM lane quadrant splitting the columns),
-//               overlapping the next tile's main loop
+//               overlapping the next tile's main loop; 16-bit results are staged
+//               per warp in shared memory (32 rows x 64 columns, 128-byte
+//               swizzle) and written by TMA stores, so global writes are whole
+//               lines instead of one 16-byte piece per row and instruction
 // Epilogues (MS-GLA reading notes, Secs. 3.2-3.3):
 //   kEpiProj      q | k | v columns to fp16, the low-rank gate columns to fp32
 //   kEpiStoreF16  a coarse branch's Y^(s) = o W_o^T to fp16
@@ -23,39 +26,22 @@
 namespace msgla {
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr int kEpiThreads = 256;
+constexpr int kStagerBytes = 32 * 128;              // one epilogue warp's staging buffer
+constexpr int kStagingBytes = 8 * 2 * kStagerBytes;  // eight epilogue warps, two buffers each
 
 template <int BN>
 struct GemmLayout {
   static constexpr int kABytes = kGemmBM * kGemmBK * 2;
   static constexpr int kBBytes = BN * kGemmBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kStagingOffset = kStages * kStageBytes;
+  static constexpr int kBarOffset = kStagingOffset + kStagingBytes;
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + 1024 B alignment slack
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
-
-__device__ __forceinline__ void cvt_store_f16x32(__half* dst, const uint32_t (&r)[32]) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    uint4 u;
-    u.x = pack_half2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
-    u.y = pack_half2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
-    u.z = pack_half2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
-    u.w = pack_half2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
-    d4[j] = u;
-  }
-}
-
-__device__ __forceinline__ void store_f32(float* dst, const uint32_t* r, int n) {
-  // n is a multiple of 4 and dst is 16-byte aligned
-  float4* d4 = reinterpret_cast<float4*>(dst);
-  for (int j = 0; j < n / 4; ++j)
-    d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]), __uint_as_float(r[4 * j + 2]),
-                        __uint_as_float(r[4 * j + 3]));
-}
 
 __device__ __forceinline__ void add_scaled_f16x32(float (&acc)[32], const __half* src, float wgt) {
   const uint4* s4 = reinterpret_cast<const uint4*>(src);
@@ -96,71 +82,6 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int tile, 
   return c;
 }
 
-// kEpiFuse with one or two coarse branches: the held rows of the next 32-column
-// chunk are loaded while the current chunk is combined, so the L2 latency of the
-// gather overlaps the arithmetic and the stores.
-__device__ __forceinline__ void epilogue_fuse_prefetch(const GemmTask& T, const TileCoord& tc, uint32_t tacc,
-                                                       int quad, int row, bool valid, size_t grow,
-                                                       const float (&wts)[kMaxScales], int c_lo, int c_hi) {
-  const uint4* base[2] = {nullptr, nullptr};
-  float wc[2] = {0.f, 0.f};
-  for (int c = 0; c < T.n_coarse; ++c) {
-    const int s = T.coarse_scale[c];
-    const int i = (row + 1) / s - 1;
-    if (valid && i >= 0) {
-      base[c] = reinterpret_cast<const uint4*>(T.coarse_y[c] +
-                                               (static_cast<size_t>(tc.b) * T.coarse_rows[c] + i) * T.N + tc.n0);
-      wc[c] = wts[T.coarse_index[c]];
-    }
-  }
-  const float wmain = valid ? wts[T.main_index] : 0.f;
-  uint4 cur[2][4], nxt[2][4];
-  auto load = [&](uint4 (&dst)[2][4], int c0) {
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dst[c][j] = base[c] ? __ldg(base[c] + (c0 >> 3) + j) : make_uint4(0, 0, 0, 0);
-  };
-  load(cur, c_lo);
-  for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
-    if (c0 + 32 < c_hi) load(nxt, c0 + 32);
-    uint32_t v[32];
-    tmem_ld32(tmem_addr(tacc, quad * 32, c0), v);
-    tmem_wait_ld();
-    if (valid) {
-      float acc[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) acc[j] = wmain * __uint_as_float(v[j]);
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const __half2* h = reinterpret_cast<const __half2*>(&cur[c][j]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(h[e]);
-            acc[8 * j + 2 * e] = fmaf(wc[c], f.x, acc[8 * j + 2 * e]);
-            acc[8 * j + 2 * e + 1] = fmaf(wc[c], f.y, acc[8 * j + 2 * e + 1]);
-          }
-        }
-      uint4* d4 = reinterpret_cast<uint4*>(T.out + grow * T.N + tc.n0 + c0);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint4 u;
-        u.x = pack_bf162(acc[8 * j + 0], acc[8 * j + 1]);
-        u.y = pack_bf162(acc[8 * j + 2], acc[8 * j + 3]);
-        u.z = pack_bf162(acc[8 * j + 4], acc[8 * j + 5]);
-        u.w = pack_bf162(acc[8 * j + 6], acc[8 * j + 7]);
-        d4[j] = u;
-      }
-    }
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) cur[c][j] = nxt[c][j];
-  }
-}
-
 // Whether this thread's accumulator row is a padded token of a masked scale-1
 // projection. Read before the wait for the accumulator so that the load's latency
 // hides behind the MMAs.
@@ -171,103 +92,237 @@ __device__ __forceinline__ bool row_is_padded(const GemmParams& p, const TileCoo
   return row < T.rows && !__ldg(T.mask + static_cast<size_t>(tc.b) * T.rows + row);
 }
 
-// Columns [c_lo, c_hi) of the tile (multiples of 32 from 0) for the accumulator
-// rows of TMEM lane quadrant `quad`.
-template <int BN>
+// Per-warp staging of 16-bit output tiles: 32 accumulator rows x 64 columns in
+// 32 rows of 128 bytes with the 128-byte swizzle (16-byte chunk j of row r at
+// chunk j ^ (r & 7)), written by the warp and sent to global memory by one TMA
+// store. Two buffers alternate, so a store's read of its buffer overlaps the
+// filling of the other. Row r is the warp's lane r; every row's 64 columns
+// arrive as two halves of 32 (one TMEM load each).
+struct Stager {
+  uint8_t* buf;  // 2 x 4 KB, 1024-byte aligned
+  int lane;
+  // buffer `sel` is free once at most the latest store (which used the other
+  // buffer) is still reading
+  __device__ __forceinline__ void acquire() const {
+    if (lane == 0) bulk_wait_read1();
+    __syncwarp();
+  }
+  __device__ __forceinline__ void put(int sel, int half, const uint32_t (&pk)[16]) const {
+    uint8_t* row = buf + sel * kStagerBytes + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      st_shared_v4(smem_u32(row + (((4 * half + j) ^ (lane & 7)) << 4)), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2],
+                   pk[4 * j + 3]);
+  }
+  // columns [col, col + 64) of rows [row0, row0 + 32) of batch element b
+  __device__ __forceinline__ void store(int sel, const CUtensorMap* map, int col, int row0, int b) const {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(map, buf + sel * kStagerBytes, col, row0, b);
+      bulk_commit();
+    }
+  }
+};
+
+__device__ __forceinline__ void pack_f16x32(uint32_t (&pk)[16], const uint32_t (&v)[32]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) pk[e] = pack_half2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+}
+__device__ __forceinline__ void pack_bf16x32(uint32_t (&pk)[16], const float (&a)[32]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) pk[e] = pack_bf162(a[2 * e], a[2 * e + 1]);
+}
+
+// Columns [c_lo, c_hi) of the tile for the accumulator rows of TMEM lane
+// quadrant `quad` (c_lo a multiple of 64). 16-bit destinations go through the
+// warp's staging buffers in steps of 64 columns; the fp32 gate and fusion-logit
+// columns of the projection are stored directly. For plain stores the TMEM load
+// of the next 32 columns is in flight while the current ones are processed; the
+// fused epilogue instead prefetches the held coarse rows one chunk ahead (both
+// at once would not fit the register budget). `sel` is the warp's running
+// staging-buffer index.
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
-                                              int lane, int c_lo, int c_hi, bool padded) {
+                                              int lane, int c_lo, int c_hi, bool padded, const Stager& stg,
+                                              int& sel) {
   const GemmTask& T = p.task[tc.task];
-  const int r = quad * 32 + lane;
-  const int row = tc.m0 + r;
+  const int row = tc.m0 + quad * 32 + lane;
+  const int row0 = tc.m0 + quad * 32;
   const bool valid = row < T.rows;
   const size_t grow = static_cast<size_t>(tc.b) * T.rows + row;
   float wts[kMaxScales];
-  if (T.epi == kEpiFuse && valid) {
-    // w = softmax(W_fuse x + b_fuse) from the logits of the projection GEMM (Eq. (10))
-    float zmax = -INFINITY;
-    for (int j = 0; j < T.n_scales; ++j) {
-      wts[j] = __ldg(T.zf + grow * T.ldz + j) + __ldg(T.bfuse + j);
-      zmax = fmaxf(zmax, wts[j]);
+  float wmain = 0.f;
+  const bool prefetch = T.epi == kEpiFuse && T.n_coarse <= 2;
+  const uint4* base0 = nullptr;
+  const uint4* base1 = nullptr;
+  float wc0 = 0.f, wc1 = 0.f;
+  if (T.epi == kEpiFuse) {
+    if (valid) {
+      // w = softmax(W_fuse x + b_fuse) from the logits of the projection GEMM (Eq. (10))
+      float zmax = -INFINITY;
+      for (int j = 0; j < T.n_scales; ++j) {
+        wts[j] = __ldg(T.zf + grow * T.ldz + j) + __ldg(T.bfuse + j);
+        zmax = fmaxf(zmax, wts[j]);
+      }
+      float sum = 0.f;
+      for (int j = 0; j < T.n_scales; ++j) {
+        wts[j] = __expf(wts[j] - zmax);
+        sum += wts[j];
+      }
+      const float inv = 1.f / sum;
+      for (int j = 0; j < T.n_scales; ++j) wts[j] *= inv;
+      if (tc.n0 == 0 && c_lo == 0)
+        for (int j = 0; j < T.n_scales; ++j) T.w[grow * T.n_scales + j] = wts[j];
+      wmain = wts[T.main_index];
     }
-    float sum = 0.f;
-    for (int j = 0; j < T.n_scales; ++j) {
-      wts[j] = __expf(wts[j] - zmax);
-      sum += wts[j];
+    if (prefetch && valid) {
+      auto held = [&](int c, const uint4*& base, float& wc) {
+        if (c >= T.n_coarse) return;
+        const int i = (row + 1) / T.coarse_scale[c] - 1;
+        if (i < 0) return;
+        base = reinterpret_cast<const uint4*>(T.coarse_y[c] +
+                                              (static_cast<size_t>(tc.b) * T.coarse_rows[c] + i) * T.N + tc.n0);
+        wc = wts[T.coarse_index[c]];
+      };
+      held(0, base0, wc0);
+      held(1, base1, wc1);
     }
-    const float inv = 1.f / sum;
-    for (int j = 0; j < T.n_scales; ++j) wts[j] *= inv;
-    if (tc.n0 == 0 && c_lo == 0)
-      for (int j = 0; j < T.n_scales; ++j) T.w[grow * T.n_scales + j] = wts[j];
   }
-  if (T.epi == kEpiFuse && T.n_coarse >= 1 && T.n_coarse <= 2) {
-    epilogue_fuse_prefetch(T, tc, tacc, quad, row, valid, grow, wts, c_lo, c_hi);
-    return;
-  }
-  const float wmain = (T.epi == kEpiFuse && valid) ? wts[T.main_index] : 0.f;
-  // Eq. (8) at scale 1 zeroes a padded row; the projections have no bias, so its
-  // q | k | v | g columns are zero (the fusion logits read x_t and are kept)
-  const int n_zeroed = T.nq + T.nk + T.nv + T.ng;
-  for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
-    uint32_t v[32];
-    tmem_ld32(tmem_addr(tacc, quad * 32, c0), v);
-    tmem_wait_ld();
-    if (!valid) continue;
+  uint4 cur0[4], cur1[4], nxt0[4], nxt1[4];
+  auto load = [&](uint4 (&d0)[4], uint4 (&d1)[4], int c0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      d0[j] = base0 ? __ldg(base0 + (c0 >> 3) + j) : make_uint4(0, 0, 0, 0);
+      d1[j] = base1 ? __ldg(base1 + (c0 >> 3) + j) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  const int n_f16 = T.epi == kEpiProj ? T.nq + T.nk + T.nv : T.N;
+  // one 32-column chunk (tile columns [c0, c0 + 32), values v); `half` places it
+  // in the current staging buffer, `last` = no chunk of this tile follows
+  auto chunk = [&](int c0, uint32_t (&v)[32], int half, bool last) __attribute__((always_inline)) {
+    if (prefetch && !last) load(nxt0, nxt1, c0 + 32);
     const int col = tc.n0 + c0;
-    if (T.epi == kEpiProj) {
+    if (col >= n_f16) {
+      // fp32 gate / fusion-logit columns of the projection. Eq. (8) at scale 1
+      // zeroes a padded row; the projections have no bias, so its q | k | v | g
+      // columns are zero (the fusion logits read x_t and are kept)
+      if (!valid) return;
+      const int n_zeroed = T.nq + T.nk + T.nv + T.ng;
       if (padded)
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           if (col + j < n_zeroed) v[j] = 0u;
-      if (col < T.nq) {
-        cvt_store_f16x32(T.q + grow * T.nq + col, v);
-      } else if (col < T.nq + T.nk) {
-        cvt_store_f16x32(T.k + grow * T.nk + (col - T.nq), v);
-      } else if (col < T.nq + T.nk + T.nv) {
-        cvt_store_f16x32(T.v + grow * T.nv + (col - T.nq - T.nk), v);
-      } else {
-        const int gc = col - T.nq - T.nk - T.nv;
-        if (gc < T.ng) store_f32(T.g + grow * T.ng + gc, v, (T.ng - gc) < 32 ? (T.ng - gc) : 32);
-        const int zs = (gc > T.ng ? gc : T.ng);  // first z column in this chunk (in gc units)
-        const int zc = zs - T.ng;
-        if (T.nz > 0 && zc < T.ldz && zs - gc < 32) {
-          const int n = (T.ldz - zc) < (32 - (zs - gc)) ? (T.ldz - zc) : (32 - (zs - gc));
-          store_f32(T.z + grow * T.ldz + zc, v + (zs - gc), n);
-        }
+      // chunk column j is gate column gc + j (j < ng - gc), then logit column
+      // gc + j - ng (< ldz when the branch carries logits); static indices keep
+      // v in registers
+      const int gc = col - n_f16;
+      float* gp = T.g + grow * T.ng;
+      float* zp = T.z ? T.z + grow * T.ldz : nullptr;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int c = gc + j;
+        if (c < T.ng)
+          gp[c] = __uint_as_float(v[j]);
+        else if (T.nz > 0 && c - T.ng < T.ldz)
+          zp[c - T.ng] = __uint_as_float(v[j]);
       }
+      return;
+    }
+    const int col64 = col - 32 * half;
+    const CUtensorMap* map = &T.tmOut[0];
+    int dcol = col64;
+    uint32_t pk[16];
+    if (T.epi == kEpiProj) {
+      if (col64 >= T.nq + T.nk) {
+        map = &T.tmOut[2];
+        dcol = col64 - T.nq - T.nk;
+      } else if (col64 >= T.nq) {
+        map = &T.tmOut[1];
+        dcol = col64 - T.nq;
+      }
+      if (padded)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0u;
+      pack_f16x32(pk, v);
     } else if (T.epi == kEpiStoreF16) {
-      cvt_store_f16x32(T.y + grow * T.N + col, v);
+      pack_f16x32(pk, v);
     } else {
       float acc[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) acc[j] = wmain * __uint_as_float(v[j]);
-      for (int c = 0; c < T.n_coarse; ++c) {
-        const int s = T.coarse_scale[c];
-        const int i = (row + 1) / s - 1;
-        if (i < 0) continue;
-        const float wc = wts[T.coarse_index[c]];
-        const __half* src = T.coarse_y[c] + (static_cast<size_t>(tc.b) * T.coarse_rows[c] + i) * T.N + col;
-        add_scaled_f16x32(acc, src, wc);
-      }
-      uint4* d4 = reinterpret_cast<uint4*>(T.out + grow * T.N + col);
+      if (prefetch) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint4 u;
-        u.x = pack_bf162(acc[8 * j + 0], acc[8 * j + 1]);
-        u.y = pack_bf162(acc[8 * j + 2], acc[8 * j + 3]);
-        u.z = pack_bf162(acc[8 * j + 4], acc[8 * j + 5]);
-        u.w = pack_bf162(acc[8 * j + 6], acc[8 * j + 7]);
-        d4[j] = u;
+        for (int j = 0; j < 4; ++j) {
+          const __half2* h0 = reinterpret_cast<const __half2*>(&cur0[j]);
+          const __half2* h1 = reinterpret_cast<const __half2*>(&cur1[j]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f0 = __half22float2(h0[q]), f1 = __half22float2(h1[q]);
+            acc[8 * j + 2 * q] = fmaf(wc1, f1.x, fmaf(wc0, f0.x, acc[8 * j + 2 * q]));
+            acc[8 * j + 2 * q + 1] = fmaf(wc1, f1.y, fmaf(wc0, f0.y, acc[8 * j + 2 * q + 1]));
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          cur0[j] = nxt0[j];
+          cur1[j] = nxt1[j];
+        }
+      } else if (valid) {
+        for (int c = 0; c < T.n_coarse; ++c) {
+          const int i = (row + 1) / T.coarse_scale[c] - 1;
+          if (i < 0) continue;
+          const __half* src = T.coarse_y[c] + (static_cast<size_t>(tc.b) * T.coarse_rows[c] + i) * T.N + col;
+          add_scaled_f16x32(acc, src, wts[T.coarse_index[c]]);
+        }
       }
+      pack_bf16x32(pk, acc);
     }
+    if (half == 0) stg.acquire();
+    stg.put(sel, half, pk);
+    if (half == 1) stg.store(sel, map, dcol, row0, tc.b);
+  };
+  if (c_lo >= c_hi) return;
+  uint32_t va[32], vb[32];
+  if (prefetch) {
+    load(cur0, cur1, c_lo);
+    for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
+      const int half = ((c0 - c_lo) >> 5) & 1;
+      tmem_ld32(tmem_addr(tacc, quad * 32, c0), va);
+      tmem_wait_ld(va);
+      chunk(c0, va, half, c0 + 32 >= c_hi);
+      if (half) sel ^= 1;
+    }
+    return;
+  }
+  tmem_ld32(tmem_addr(tacc, quad * 32, c_lo), va);
+  tmem_wait_ld(va);
+  for (int c0 = c_lo; c0 < c_hi; c0 += 64) {
+    const bool has_b = c0 + 32 < c_hi, has_next = c0 + 64 < c_hi;
+    if (has_b) tmem_ld32(tmem_addr(tacc, quad * 32, c0 + 32), vb);
+    chunk(c0, va, 0, !has_b);
+    if (has_b) {
+      tmem_wait_ld(vb);
+      if (has_next) tmem_ld32(tmem_addr(tacc, quad * 32, c0 + 64), va);
+      chunk(c0 + 32, vb, 1, !has_next);
+      if (has_next) tmem_wait_ld(va);
+    }
+    sel ^= 1;
   }
 }
 
-// Two epilogue warps share each TMEM lane quadrant and split the tile's columns.
+// Two epilogue warps share each TMEM lane quadrant and split the tile's columns
+// at a multiple of 64 (one staging step).
 __device__ __forceinline__ void epi_columns(int warp, int n_eff, int& lo, int& hi) {
-  const int mid = min(n_eff, ((n_eff / 2 + 31) / 32) * 32);
+  const int mid = min(n_eff, ((n_eff / 2 + 63) / 64) * 64);
   const bool second = (warp - 2) >= 4;
   lo = second ? mid : 0;
   hi = second ? n_eff : mid;
+}
+
+// Prefetch the output tensor maps of every task (epilogue warps).
+__device__ __forceinline__ void prefetch_out_maps(const GemmParams& p) {
+  for (int t = 0; t < p.n_tasks; ++t)
+    for (int m = 0; m < 3; ++m) prefetch_tmap(&p.task[t].tmOut[m]);
 }
 
 template <int BN>
@@ -363,6 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   } else if (warp >= 2) {
     // ---------------- epilogue: one accumulator row per thread
     const int quad = warp & 3;
+    const Stager stg{smem + Lay::kStagingOffset + (warp - 2) * 2 * kStagerBytes, lane};
+    int sel = 0;
+    if (lane == 0) prefetch_out_maps(p);
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
       const TileCoord tc = decode_tile(p, tile, BN);
@@ -372,10 +430,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       tc_fence_after();
       int lo, hi;
       epi_columns(warp, tc.n_eff, lo, hi);
-      epilogue_tile<BN>(p, tc, tmem + buf * BN, quad, lane, lo, hi, padded);
+      epilogue_tile(p, tc, tmem + buf * BN, quad, lane, lo, hi, padded, stg, sel);
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
     }
+    if (lane == 0) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -394,10 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 // MMAs; each CTA holds its 128 rows of the accumulator in its own TMEM and runs
 // its own epilogue. Loads carry no multicast: both CTAs fetch their own halves
 // and signal the leader's full barrier; the leader's commits reach both CTAs.
-constexpr int kPairStages = 7;
+constexpr int kPairStages = 5;
 constexpr int kPairStageBytes = 2 * kGemmBM * kGemmBK * 2;  // A half + B half = 32 KB
-constexpr int kPairBarOffset = kPairStages * kPairStageBytes;
+constexpr int kPairStagingOffset = kPairStages * kPairStageBytes;
+constexpr int kPairBarOffset = kPairStagingOffset + kStagingBytes;
 constexpr int kPairSmemBytes = kPairBarOffset + 256 + 1024;
+static_assert(kPairSmemBytes <= 227 * 1024, "shared memory budget");
 constexpr int kPairBN = 256, kPairBM = 256;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -496,6 +557,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;
     const uint32_t lead_empty0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     const uint32_t lead_empty1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
+    const Stager stg{smem + kPairStagingOffset + (warp - 2) * 2 * kStagerBytes, lane};
+    int sel = 0;
+    if (lane == 0) prefetch_out_maps(p);
     uint32_t it = 0;
     for (int tile = pair; tile < ntiles; tile += npairs, ++it) {
       TileCoord tc = decode_tile(p, tile, kPairBN, kPairBM);
@@ -506,10 +570,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       int lo, hi;
       epi_columns(warp, tc.n_eff, lo, hi);
-      epilogue_tile<kPairBN>(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded);
+      epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel);
       tc_fence_before();
       mbar_arrive_cluster(buf ? lead_empty1 : lead_empty0);
     }
+    if (lane == 0) bulk_wait0();
   }
   tc_fence_before();
   cluster_sync();

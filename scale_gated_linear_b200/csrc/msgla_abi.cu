@@ -92,6 +92,19 @@ bool encode_2d(CUtensorMap* m, bool bf16, const void* base, uint64_t inner, uint
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output map of the GEMM epilogue: 16-bit [batch][rows][inner], {64, 32, 1} box, 128B swizzle.
+bool encode_out_3d(CUtensorMap* m, bool bf16, void* base, uint64_t inner, uint64_t rows, uint64_t batch) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {64, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, base, dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DeviceGuard {
   int prev = -1;
   bool ok = false;
@@ -432,6 +445,10 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.v = static_cast<__half*>(at(bw.v));
     t.g = static_cast<float*>(at(bw.g));
     t.mask = bf ? M : nullptr;
+    if (!encode_out_3d(&t.tmOut[0], false, t.q, t.nq, bw.rows, B) ||
+        !encode_out_3d(&t.tmOut[1], false, t.k, t.nk, bw.rows, B) ||
+        !encode_out_3d(&t.tmOut[2], false, t.v, t.nv, bw.rows, B))
+      return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (projection outputs, scale %d)", b.scale);
     tiles += B * t.m_tiles * t.n_tiles;
   }
   gp.n_tasks = ns;
@@ -582,6 +599,8 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.ab_bf16 = 0;
     t.epi = kEpiStoreF16;
     t.y = static_cast<__half*>(at(bw.Y));
+    if (!encode_out_3d(&t.tmOut[0], false, t.y, d, bw.rows, B))
+      return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (output store, scale %d)", b.scale);
     tiles += B * t.m_tiles * t.n_tiles;
   }
   if (nt > 0) {
@@ -611,6 +630,8 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.ab_bf16 = 0;
     t.epi = kEpiFuse;
     t.out = static_cast<__nv_bfloat16*>(O);
+    if (!encode_out_3d(&t.tmOut[0], true, O, d, L, B))
+      return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (layer output)");
     t.zf = static_cast<const float*>(at(ws.z));
     t.ldz = h->ldz;
     t.bfuse = h->bfuse;
@@ -763,6 +784,10 @@ int step_impl(msgla_handle* h, void* cache, const void* x, int B, long long t, v
       tk.k = static_cast<__half*>(wat(sl.k[j]));
       tk.v = static_cast<__half*>(wat(sl.v[j]));
       tk.g = static_cast<float*>(wat(sl.g[j]));
+      if (!encode_out_3d(&tk.tmOut[0], false, tk.q, tk.nq, B, 1) ||
+          !encode_out_3d(&tk.tmOut[1], false, tk.k, tk.nk, B, 1) ||
+          !encode_out_3d(&tk.tmOut[2], false, tk.v, tk.nv, B, 1))
+        return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (step projection outputs, scale %d)", b.scale);
       tiles += tk.m_tiles * tk.n_tiles;
     }
     gp.n_tasks = nt;
@@ -842,6 +867,8 @@ int step_impl(msgla_handle* h, void* cache, const void* x, int B, long long t, v
       tk.ab_bf16 = 0;
       tk.epi = kEpiStoreF16;
       tk.y = static_cast<__half*>(b.scale == 1 ? wat(sl.Y1) : cat(cl.Y[j]));
+      if (!encode_out_3d(&tk.tmOut[0], false, tk.y, d, B, 1))
+        return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (step output store, scale %d)", b.scale);
       tiles += tk.m_tiles * tk.n_tiles;
     }
     gp.n_tasks = nt;

@@ -29,6 +29,10 @@ enum EpiKind : int {
 struct alignas(64) GemmTask {
   CUtensorMap tmA;  // 3D {K, rows, B}, box {64, 128, 1}, 128B swizzle
   CUtensorMap tmB;  // 2D {K, N}, box {64, 128}, 128B swizzle
+  // 16-bit outputs, 3D {columns, rows, B}, box {64, 32, 1}, 128B swizzle (TMA stores
+  // of 32 rows x 64 columns staged per epilogue warp): kEpiProj q, k, v;
+  // kEpiStoreF16 y; kEpiFuse out
+  CUtensorMap tmOut[3];
   int rows, m_tiles, n_tiles, N, K, tile_begin, ab_bf16, epi;
   // kEpiProj (columns: q | k | v | g (ng) | fusion logits z (nz, scale-1 branch))
   int nq, nk, nv, ng, nz, ldz;
