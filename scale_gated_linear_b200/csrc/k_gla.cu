@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer. Per chunk: Qs S', scores, S' update, A V.
+      // ---------------- MMA issuer. Per chunk: Qs S', S' update, A V, then the
+      // scores of the next chunk.
       const uint32_t id_kk = idesc_f16(128, 128, 0, 0, 0);  // K-major x K-major
       const uint32_t id_km = idesc_f16(128, 128, 0, 0, 1);  // K-major (smem or TMEM) x MN-major
       const uint32_t id_mm = idesc_f16(128, 128, 0, 1, 1);  // MN-major x MN-major
@@ -159,10 +160,26 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
         umma_commit(&bar[B_K_EMPTY]);
         umma_commit(&bar[B_V_EMPTY]);
       }
+      // Full pass. The scores of chunk c + 1 are issued right after the A V
+      // product of chunk c, so their conversion overlaps the Qs S' and S' update
+      // products of chunk c + 1, and the o drain and state epilogue of chunk c
+      // overlap the next scores: per chunk the chain is the scores, Qs S' and
+      // the S' update, plus the wait for the next K tile.
+      auto scores = [&](int c) {  // A = Qs Ks^T  (K = d_k)
+        for (int ks = 0; ks < dkp / 16; ++ks)
+          umma_f16(tmem + kColA, sdesc_sw128(sQ + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024),
+                   sdesc_sw128(sK + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024), id_kk, ks > 0);
+        umma_commit(&bar[B_A_FULL]);
+      };
+      if (!state_pass && nch > 0) {
+        if (mbar_wait(&bar[B_Q_FULL], 0, abort_flag, p.err) && mbar_wait(&bar[B_K_FULL], 0, abort_flag, p.err)) {
+          tc_fence_after();
+          scores(0);
+        }
+      }
       for (int c = 0; c < nch && !state_pass; ++c) {
         const uint32_t ph = c & 1, pp = (c - 1) & 1;
         const bool carried = c > 0 || has_init;  // a state enters this chunk
-        if (!mbar_wait(&bar[B_Q_FULL], ph, abort_flag, p.err)) break;
         if (carried) {
           if (!mbar_wait(&bar[B_S_DONE], (c - 1 + sd0) & 1, abort_flag, p.err)) break;
           if (c > 0 && !mbar_wait(&bar[B_O_EMPTY], pp, abort_flag, p.err)) break;
@@ -172,14 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
             umma_f16(tmem + kColO, sdesc_sw128(sQ + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024),
                      sdesc_sw128(sS + ks * 2048, lbo_s, 1024), id_km, ks > 0);
         }
-        if (!mbar_wait(&bar[B_K_FULL], ph, abort_flag, p.err)) break;
-        tc_fence_after();
-        // A = Qs Ks^T  (K = d_k)
-        for (int ks = 0; ks < dkp / 16; ++ks)
-          umma_f16(tmem + kColA, sdesc_sw128(sQ + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024),
-                   sdesc_sw128(sK + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024), id_kk, ks > 0);
-        umma_commit(&bar[B_A_FULL]);
-        umma_commit(&bar[B_Q_EMPTY]);
+        umma_commit(&bar[B_Q_EMPTY]);  // Qs of chunk c: scores and Qs S' issued
         if (!mbar_wait(&bar[B_V_FULL], ph, abort_flag, p.err)) break;
         tc_fence_after();
         // S' += Ks^T V per 128-row half of d_k  (K = chunk rows j)
@@ -197,6 +207,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
                       (carried || ks > 0) ? 1u : 0u);
         umma_commit(&bar[B_O_FULL]);
         umma_commit(&bar[B_V_EMPTY]);
+        if (c + 1 < nch) {
+          if (!mbar_wait(&bar[B_Q_FULL], ph ^ 1, abort_flag, p.err)) break;
+          if (!mbar_wait(&bar[B_K_FULL], ph ^ 1, abort_flag, p.err)) break;
+          tc_fence_after();
+          scores(c + 1);
+        }
       }
     }
   } else if (warp >= 4 && warp < 8) {
