@@ -400,6 +400,19 @@ __global__ void __launch_bounds__(256) head_norm_kernel(const HeadNormParams p) 
 constexpr int kGateThreads = 256;
 constexpr int kGateChannels = 128;  // key channels per CTA
 
+// 2^x by the hardware approximation (relative error about 2^-22, far below the
+// fp16 rounding of the scaled q and k it feeds)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Nonzero if either half of a packed fp16 pair is inf or nan (exponent all ones).
+__device__ __forceinline__ uint32_t half2_nonfinite(uint32_t h) {
+  return ((h & 0x7c00u) == 0x7c00u) | ((h & 0x7c000000u) == 0x7c000000u);
+}
+
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
@@ -605,7 +618,7 @@ __global__ void __launch_bounds__(kGateThreads, 3) gate_kernel(const __grid_cons
 #pragma unroll
   for (int e = 0; e < 8; ++e) pre[e] -= second ? 0.f : tot[e];
 
-  float mx = 0.f;
+  uint32_t over = 0;  // a scaled value left the fp16 range
   const int sw = rg & 7;  // (row >> 2) & 7 for all four rows of this thread
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
@@ -622,17 +635,15 @@ __global__ void __launch_bounds__(kGateThreads, 3) gate_kernel(const __grid_cons
     for (int e = 0; e < 4; ++e) {
       const float b0 = pre[2 * e] + c[r][2 * e], b1 = pre[2 * e + 1] + c[r][2 * e + 1];
       const float2 qf = __half22float2(qh[e]), kf = __half22float2(kh[e]);
-      const float qs0 = qf.x * exp2f(b0), qs1 = qf.y * exp2f(b1);
-      const float ks0 = kf.x * exp2f(-b0), ks1 = kf.y * exp2f(-b1);
-      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(qs0), fabsf(qs1)), fmaxf(fabsf(ks0), fabsf(ks1))));
-      qw[e] = pack_half2(qs0, qs1);
-      kw[e] = pack_half2(ks0, ks1);
+      qw[e] = pack_half2(qf.x * ex2_approx(b0), qf.y * ex2_approx(b1));
+      kw[e] = pack_half2(kf.x * ex2_approx(-b0), kf.y * ex2_approx(-b1));
+      over |= half2_nonfinite(qw[e]) | half2_nonfinite(kw[e]);
     }
     const size_t go = (row_base + row) * ldk + cbase + cg * 8;
     *reinterpret_cast<uint4*>(P.qs + go) = qo;
     *reinterpret_cast<uint4*>(P.ks + go) = ko;
   }
-  if (!(mx <= 65504.f)) atomicCAS(p.err, 0, kDevRange);
+  if (over) atomicCAS(p.err, 0, kDevRange);
   if (rg == 15) {
     const size_t gi = (static_cast<size_t>(b) * n_chunks + ci) * ldk + cbase + cg * 8;
     float* dst = second ? P.gamma : P.mid;
