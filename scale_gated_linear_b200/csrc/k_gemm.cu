@@ -99,16 +99,23 @@ __device__ __forceinline__ bool row_is_padded(const GemmParams& p, const TileCoo
 // filling of the other. Row r is the warp's lane r; every row's 64 columns
 // arrive as two halves of 32 (one TMEM load each).
 struct Stager {
-  uint8_t* buf;  // 2 x 4 KB, 1024-byte aligned
+  uint8_t* buf;  // 1 or 2 x 4 KB, 1024-byte aligned
   int lane;
-  // buffer `sel` is free once at most the latest store (which used the other
-  // buffer) is still reading
+  bool dbl;      // two buffers alternate (else one)
+  // the buffer about to be filled is free: with two buffers at most the latest
+  // store (which used the other one) may still be reading
   __device__ __forceinline__ void acquire() const {
-    if (lane == 0) bulk_wait_read1();
+    if (lane == 0) {
+      if (dbl)
+        bulk_wait_read1();
+      else
+        bulk_wait_read0();
+    }
     __syncwarp();
   }
+  __device__ __forceinline__ uint8_t* at(int sel) const { return buf + (dbl ? sel : 0) * kStagerBytes; }
   __device__ __forceinline__ void put(int sel, int half, const uint32_t (&pk)[16]) const {
-    uint8_t* row = buf + sel * kStagerBytes + lane * 128;
+    uint8_t* row = at(sel) + lane * 128;
 #pragma unroll
     for (int j = 0; j < 4; ++j)
       st_shared_v4(smem_u32(row + (((4 * half + j) ^ (lane & 7)) << 4)), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2],
@@ -119,10 +126,22 @@ struct Stager {
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_3d(map, buf + sel * kStagerBytes, col, row0, b);
+      tma_store_3d(map, at(sel), col, row0, b);
       bulk_commit();
     }
   }
+};
+
+// Held coarse rows of one CTA tile in shared memory (kEpiFuse with one or two
+// coarse branches): for coarse branch c, the rows i = floor((t+1)/s) - 1 of the
+// tile's output rows t in [m0, m0 + 128) as four 64-column boxes of
+// held_box_rows(s) rows of 128 bytes (128-byte swizzle), starting at row
+// held_base(m0, s); rows before the first block and past the end are zero.
+__device__ __forceinline__ int held_base(int m0, int s) { return (m0 + 1) / s - 1; }
+struct Held {
+  const uint8_t* smem[2];  // box 0 of each coarse branch
+  int box_bytes[2];
+  int lrow[2];             // this thread's held row within the boxes
 };
 
 __device__ __forceinline__ void pack_f16x32(uint32_t (&pk)[16], const uint32_t (&v)[32]) {
@@ -144,7 +163,7 @@ __device__ __forceinline__ void pack_bf16x32(uint32_t (&pk)[16], const float (&a
 // staging-buffer index.
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
                                               int lane, int c_lo, int c_hi, bool padded, const Stager& stg,
-                                              int& sel) {
+                                              int& sel, const Held* held = nullptr) {
   const GemmTask& T = p.task[tc.task];
   const int row = tc.m0 + quad * 32 + lane;
   const int row0 = tc.m0 + quad * 32;
@@ -152,7 +171,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
   const size_t grow = static_cast<size_t>(tc.b) * T.rows + row;
   float wts[kMaxScales];
   float wmain = 0.f;
-  const bool prefetch = T.epi == kEpiFuse && T.n_coarse <= 2;
+  const bool prefetch = T.epi == kEpiFuse && T.n_coarse <= 2 && !held;
   const uint4* base0 = nullptr;
   const uint4* base1 = nullptr;
   float wc0 = 0.f, wc1 = 0.f;
@@ -250,7 +269,29 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
       float acc[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) acc[j] = wmain * __uint_as_float(v[j]);
-      if (prefetch) {
+      if (held) {
+        // held coarse rows from shared memory: 16-byte pieces q of the chunk's
+        // 64-column box, swizzled by the row
+        const int box = c0 >> 6, q0 = (c0 & 63) >> 3;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (c >= T.n_coarse) break;
+          const float wgt = valid ? wts[T.coarse_index[c]] : 0.f;
+          const int lr = held->lrow[c];
+          const uint8_t* rowp = held->smem[c] + box * held->box_bytes[c] + lr * 128;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 u = *reinterpret_cast<const uint4*>(rowp + (((q0 + j) ^ (lr & 7)) << 4));
+            const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 f = __half22float2(h[q]);
+              acc[8 * j + 2 * q] = fmaf(wgt, f.x, acc[8 * j + 2 * q]);
+              acc[8 * j + 2 * q + 1] = fmaf(wgt, f.y, acc[8 * j + 2 * q + 1]);
+            }
+          }
+        }
+      } else if (prefetch) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const __half2* h0 = reinterpret_cast<const __half2*>(&cur0[j]);
@@ -453,30 +494,50 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 // MMAs; each CTA holds its 128 rows of the accumulator in its own TMEM and runs
 // its own epilogue. Loads carry no multicast: both CTAs fetch their own halves
 // and signal the leader's full barrier; the leader's commits reach both CTAs.
-constexpr int kPairStages = 5;
+//
+// kHeld (the fused output launch with one or two coarse branches): warp 10 of
+// each CTA TMA-loads the held coarse rows of the CTA's tile into shared memory
+// during the tile's main loop, so the epilogue reads them there instead of
+// gathering them from L2. This takes a 60 KB region: the ring has 4 stages and
+// every epilogue warp one staging buffer.
 constexpr int kPairStageBytes = 2 * kGemmBM * kGemmBK * 2;  // A half + B half = 32 KB
-constexpr int kPairStagingOffset = kPairStages * kPairStageBytes;
-constexpr int kPairBarOffset = kPairStagingOffset + kStagingBytes;
-constexpr int kPairSmemBytes = kPairBarOffset + 256 + 1024;
-static_assert(kPairSmemBytes <= 227 * 1024, "shared memory budget");
 constexpr int kPairBN = 256, kPairBM = 256;
+constexpr int kHeldBytes = 60 * 1024;
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <bool kHeld>
+struct PairLayout {
+  static constexpr int kStages = kHeld ? 4 : 5;
+  static constexpr int kThreadsT = kHeld ? 352 : 320;  // + warp 10: held-row loader
+  static constexpr int kStagingOffset = kStages * kPairStageBytes;
+  static constexpr int kStagingBytesT = kHeld ? 8 * kStagerBytes : kStagingBytes;
+  static constexpr int kHeldOffset = kStagingOffset + kStagingBytesT;
+  static constexpr int kBarOffset = kHeldOffset + (kHeld ? kHeldBytes : 0);
+  static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+template <bool kHeld>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::kThreadsT, 1)
     gemm_pair_kernel(const __grid_constant__ GemmParams p) {
+  using Lay = PairLayout<kHeld>;
+  constexpr int kStagesT = Lay::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kPairBarOffset);
-  uint64_t* empty_bar = full_bar + kPairStages;
-  uint64_t* acc_full = empty_bar + kPairStages;  // [2]
-  uint64_t* acc_empty = acc_full + 2;            // [2] (used in the leader)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Lay::kBarOffset);
+  uint64_t* empty_bar = full_bar + kStagesT;
+  uint64_t* acc_full = empty_bar + kStagesT;  // [2]
+  uint64_t* acc_empty = acc_full + 2;         // [2] (used in the leader)
+  uint64_t* held_full = acc_empty + 2;        // kHeld: this CTA's held rows landed
+  uint64_t* held_empty = held_full + 1;       // kHeld: this CTA's epilogue is done with them
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(held_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* held_smem = smem + Lay::kHeldOffset;
 
   const int warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPairStages; ++s) {
+    for (int s = 0; s < kStagesT; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
@@ -484,6 +545,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 2 * kEpiThreads);
     }
+    mbar_init(held_full, 1);
+    mbar_init(held_empty, kEpiThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -496,6 +559,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int ntiles = p.total_tiles;
+  // held rows: coarse branch c occupies [held_off[c], +4 boxes)
+  int held_off[2] = {0, 0}, held_box[2] = {0, 0};
+  if (kHeld) {
+    const GemmTask& T0 = p.task[0];
+    for (int c = 0; c < 2 && c < T0.n_coarse; ++c) {
+      held_box[c] = held_box_rows(T0.coarse_scale[c]) * 128;
+      if (c == 1) held_off[1] = 4 * held_box[0];
+    }
+  }
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer of this CTA's halves
@@ -511,8 +583,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int arow = tc.m0 + 128 * static_cast<int>(rank);
       const int brow = tc.n0 + static_cast<int>(rank) * (tc.n_eff >> 1);
       for (int kb = 0; kb < tc.kblocks; ++kb, ++kbg) {
-        const uint32_t s = kbg % kPairStages;
-        if (kbg >= kPairStages && !mbar_wait(&empty_bar[s], ((kbg / kPairStages) - 1) & 1, abort_flag, p.err)) {
+        const uint32_t s = kbg % kStagesT;
+        if (kbg >= kStagesT && !mbar_wait(&empty_bar[s], ((kbg / kStagesT) - 1) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
@@ -536,8 +608,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t idesc = idesc_f16(kPairBM, tc.n_eff, p.task[tc.task].ab_bf16, 0, 0);
       const uint32_t tacc = tmem + buf * kPairBN;
       for (int kb = 0; kb < tc.kblocks; ++kb, ++kbg) {
-        const uint32_t s = kbg % kPairStages;
-        if (!mbar_wait(&full_bar[s], (kbg / kPairStages) & 1, abort_flag, p.err)) {
+        const uint32_t s = kbg % kStagesT;
+        if (!mbar_wait(&full_bar[s], (kbg / kStagesT) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
@@ -552,12 +624,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (ok) umma_commit_pair(&acc_full[buf], 0x3);
     }
-  } else if (warp >= 2) {
+  } else if (kHeld && warp == 10) {
+    // ---------------- held coarse rows of this CTA's tiles (one tile ahead at most)
+    if (lane == 0) {
+      const GemmTask& T = p.task[0];
+      for (int c = 0; c < 2 && c < T.n_coarse; ++c) prefetch_tmap(&T.tmOut[1 + c]);
+      uint32_t it = 0;
+      for (int tile = pair; tile < ntiles; tile += npairs, ++it) {
+        const TileCoord tc = decode_tile(p, tile, kPairBN, kPairBM);
+        const int m0 = tc.m0 + 128 * static_cast<int>(rank);
+        if (it >= 1 && !mbar_wait(held_empty, (it - 1) & 1, abort_flag, p.err)) break;
+        uint32_t bytes = 0;
+        for (int c = 0; c < 2 && c < T.n_coarse; ++c) bytes += 4 * held_box[c];
+        mbar_arrive_expect_tx(held_full, bytes);
+        for (int c = 0; c < 2 && c < T.n_coarse; ++c) {
+          const int base = held_base(m0, T.coarse_scale[c]);
+          for (int j = 0; j < 4; ++j)
+            tma_load_3d(&T.tmOut[1 + c], held_full, held_smem + held_off[c] + j * held_box[c], tc.n0 + 64 * j, base,
+                        tc.b);
+        }
+      }
+    }
+  } else if (warp >= 2 && warp < 10) {
     // ---------------- epilogue of this CTA's 128 accumulator rows
     const int quad = warp & 3;
     const uint32_t lead_empty0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     const uint32_t lead_empty1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
-    const Stager stg{smem + kPairStagingOffset + (warp - 2) * 2 * kStagerBytes, lane};
+    const Stager stg{smem + Lay::kStagingOffset + (warp - 2) * (kHeld ? 1 : 2) * kStagerBytes, lane, !kHeld};
     int sel = 0;
     if (lane == 0) prefetch_out_maps(p);
     uint32_t it = 0;
@@ -570,7 +663,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       int lo, hi;
       epi_columns(warp, tc.n_eff, lo, hi);
-      epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel);
+      if (kHeld) {
+        if (!mbar_wait(held_full, it & 1, abort_flag, p.err)) break;
+        const GemmTask& T = p.task[tc.task];
+        const int t = tc.m0 + quad * 32 + lane;
+        Held h;
+        for (int c = 0; c < 2; ++c) {
+          h.smem[c] = held_smem + held_off[c];
+          h.box_bytes[c] = held_box[c];
+          h.lrow[c] = 0;
+          if (c < T.n_coarse) {
+            const int s = T.coarse_scale[c];
+            h.lrow[c] = (t + 1) / s - 1 - held_base(tc.m0, s);
+          }
+        }
+        epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel, &h);
+        fence_proxy_async_smem();
+        mbar_arrive(held_empty);
+      } else {
+        epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel);
+      }
       tc_fence_before();
       mbar_arrive_cluster(buf ? lead_empty1 : lead_empty0);
     }
@@ -597,16 +709,18 @@ int sm_count() {
 }
 
 // Pairs of CTAs that can be resident at once (0 if the pair kernel cannot run).
+template <bool kHeld>
 int max_active_pairs() {
+  using Lay = PairLayout<kHeld>;
   static int n = -1;
   if (n < 0) {
     n = 0;
-    if (cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) ==
-        cudaSuccess) {
+    if (cudaFuncSetAttribute(gemm_pair_kernel<kHeld>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Lay::kSmemBytes) == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * sm_count(), 1, 1);
-      cfg.blockDim = dim3(kThreads, 1, 1);
-      cfg.dynamicSmemBytes = kPairSmemBytes;
+      cfg.blockDim = dim3(Lay::kThreadsT, 1, 1);
+      cfg.dynamicSmemBytes = Lay::kSmemBytes;
       cudaLaunchAttribute attr;
       attr.id = cudaLaunchAttributeClusterDimension;
       attr.val.clusterDim.x = 2;
@@ -615,7 +729,7 @@ int max_active_pairs() {
       cfg.attrs = &attr;
       cfg.numAttrs = 1;
       int c = 0;
-      if (cudaOccupancyMaxActiveClusters(&c, gemm_pair_kernel, &cfg) == cudaSuccess) n = c;
+      if (cudaOccupancyMaxActiveClusters(&c, gemm_pair_kernel<kHeld>, &cfg) == cudaSuccess) n = c;
     }
     cudaGetLastError();  // clear a failed query
   }
@@ -624,7 +738,11 @@ int max_active_pairs() {
 
 cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st) {
   if (p.total_tiles <= 0) return cudaSuccess;
-  const int pairs = (bn == 256) ? max_active_pairs() : 0;
+  // the fused output launch with one or two coarse branches stages their held
+  // rows in shared memory (the caller encodes tmOut[1 + c] for them)
+  const bool held = p.n_tasks == 1 && p.task[0].epi == kEpiFuse && p.task[0].n_coarse >= 1 &&
+                    p.task[0].n_coarse <= 2 && held_rows_fit(p.task[0].coarse_scale, p.task[0].n_coarse);
+  const int pairs = (bn != 256) ? 0 : held ? max_active_pairs<true>() : max_active_pairs<false>();
   if (pairs > 0) {
     // re-tile every task in 256 x 256 pair tiles
     static thread_local GemmParams q;
@@ -641,7 +759,10 @@ cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st) {
     }
     q.total_tiles = tiles;
     const int grid_pairs = tiles < pairs ? tiles : pairs;
-    gemm_pair_kernel<<<2 * grid_pairs, kThreads, kPairSmemBytes, st>>>(q);
+    if (held)
+      gemm_pair_kernel<true><<<2 * grid_pairs, PairLayout<true>::kThreadsT, PairLayout<true>::kSmemBytes, st>>>(q);
+    else
+      gemm_pair_kernel<false><<<2 * grid_pairs, PairLayout<false>::kThreadsT, PairLayout<false>::kSmemBytes, st>>>(q);
     return cudaGetLastError();
   }
   const int grid = p.total_tiles < sm_count() ? p.total_tiles : sm_count();

@@ -648,6 +648,23 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
       ++nc;
     }
     t.n_coarse = nc;
+    // held coarse rows of a CTA tile, staged by TMA in the fused GEMM: one
+    // 64-column box of held_box_rows(s) rows per load (rows before the first
+    // block and past the end read as zero)
+    if (nc >= 1 && nc <= 2 && held_rows_fit(t.coarse_scale, nc)) {
+      for (int c = 0; c < nc; ++c) {
+        EncodeTiledFn fn = encode_fn();
+        cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(t.coarse_rows[c]),
+                              static_cast<cuuint64_t>(B)};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(d) * t.coarse_rows[c] * 2};
+        cuuint32_t box[3] = {64, static_cast<cuuint32_t>(held_box_rows(t.coarse_scale[c])), 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (!fn || fn(&t.tmOut[1 + c], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<__half*>(t.coarse_y[c]), dims,
+                      strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+          return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (held coarse rows, scale %d)", t.coarse_scale[c]);
+      }
+    }
     gp.n_tasks = 1;
     gp.total_tiles = B * t.m_tiles * t.n_tiles;
     CUDA_TRY(launch_gemm(gp, 256, st));

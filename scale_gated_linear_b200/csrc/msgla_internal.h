@@ -57,6 +57,17 @@ struct alignas(64) GemmTask {
   const __half* coarse_y[kMaxScales];
 };
 
+// Rows of one 64-column box of held coarse rows staged by the fused output GEMM
+// for a 128-row CTA tile and coarse scale s (at most 127 / s + 2 distinct rows,
+// rounded up to 8 for the 128-byte swizzle), and whether the boxes of the given
+// coarse scales fit the 60 KB region.
+inline __host__ __device__ int held_box_rows(int s) { return ((127 / s + 2) + 7) / 8 * 8; }
+inline __host__ __device__ bool held_rows_fit(const int* scales, int n) {
+  int bytes = 0;
+  for (int c = 0; c < n; ++c) bytes += 4 * held_box_rows(scales[c]) * 128;
+  return bytes <= 60 * 1024;
+}
+
 struct GemmParams {
   GemmTask task[kMaxTasks];
   int n_tasks;
