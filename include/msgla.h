@@ -102,7 +102,8 @@ typedef struct msgla_handle msgla_handle;
 int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weights* w,
                  int device);
 
-/* Free everything the handle owns. NULL-safe. Synchronises the handle's device. */
+/* Free everything the handle owns (weights, counters, its second stream and
+ * events). NULL-safe. Synchronises the handle's device. */
 void msgla_destroy(msgla_handle* h);
 
 /* Bytes of device workspace msgla_forward needs for a [B, L, d] input.
@@ -117,7 +118,14 @@ int msgla_workspace_size(const msgla_handle* h, int B, int L, size_t* bytes);
  *   stream     cudaStream_t (NULL = legacy default stream).
  * Asynchronous: returns after enqueuing the kernels on `stream`. Errors found by
  * the kernels (timeouts, fp16 range) are latched in the handle and reported by
- * msgla_sync_status. B*L = 0 launches nothing. */
+ * msgla_sync_status. B*L = 0 launches nothing.
+ * With a scale-1 branch, the output projection of the coarse branches may run on
+ * a second stream owned by the handle, concurrently with the GLA kernel (forked
+ * after the gates, joined back before the final output projection), so all of
+ * the forward's work is still ordered before what follows it on `stream`; the
+ * fork and join use events, so the forward can be captured into a CUDA graph.
+ * The handle keeps per-forward counters: forwards on one handle must not run
+ * concurrently (serialise calls from several host threads or streams). */
 int msgla_forward(msgla_handle* h, const void* X, int B, int L, void* O,
                   void* workspace, size_t workspace_bytes, void* stream);
 
@@ -161,8 +169,11 @@ int msgla_forward_noalloc(msgla_handle* h, const void* X, int B, int L, void* O,
  * kernel on `stream` with events. `events` holds caller-created cudaEvent_t
  * handles: events[0] is recorded before the first kernel and events[i+1] after
  * the i-th kernel; msgla_launch_plan lists the kernels in launch order.
- * `max_events` is the length of `events` (it must be at least n_launches + 1);
- * *n_launches receives the number of kernels launched. `M` is the optional
+ * `max_events` is the length of `events` (it must be at least the number of
+ * msgla_launch_plan entries + 1); *n_launches receives the number of kernels
+ * launched, which includes the kernels run on the second stream (the coarse
+ * output projection and the one-warp wait before it; no plan entries and no
+ * events of their own). `M` is the optional
  * valid-token mask of msgla_forward_masked (NULL = every token valid). */
 int msgla_forward_profiled(msgla_handle* h, const void* X, const void* M, int B, int L, void* O,
                            void* workspace, size_t workspace_bytes, void* stream,
@@ -234,7 +245,10 @@ int msgla_step(msgla_handle* h, void* cache, const void* x, int B, long long t, 
  * [out_gemm_coarse], out_gemm_fused | out_gemm_coarse, hold_fuse. gla_state and
  * gla_scan appear when long sequences are cut into segments (few sequences: the
  * GLA kernel would fill less than half of the GPU); head_norm when the config
- * enables the head RMS norm. msgla_forward_profiled records one event per entry. */
+ * enables the head RMS norm. out_gemm_coarse is absent when it runs on the
+ * handle's second stream alongside gla (a scale-1 branch, no segments, no head
+ * norm, and SMs left free by the GLA CTAs). msgla_forward_profiled records one
+ * event per entry. */
 int msgla_launch_plan(const msgla_handle* h, int B, int L, char* names, size_t len);
 
 /* Failure-detection testing: with enable != 0, the next forward on this handle

@@ -366,6 +366,17 @@ __device__ __forceinline__ void prefetch_out_maps(const GemmParams& p) {
     for (int m = 0; m < 3; ++m) prefetch_tmap(&p.task[t].tmOut[m]);
 }
 
+// Producer side of a per-task input dependency (GemmTask::dep): before the first
+// load of a task, wait for its producer running on another stream.
+__device__ __forceinline__ bool task_ready(const GemmTask& T, int task, uint32_t& ready, volatile int* abort_flag,
+                                           int* err) {
+  if (!T.dep || ((ready >> task) & 1u)) return true;
+  if (!wait_count(T.dep, T.dep_target, abort_flag, err)) return false;
+  fence_proxy_async_global();
+  ready |= 1u << task;
+  return true;
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   using Lay = GemmLayout<BN>;
@@ -407,11 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       prefetch_tmap(&p.task[t].tmA);
       prefetch_tmap(&p.task[t].tmB);
     }
-    uint32_t kbg = 0;
+    uint32_t kbg = 0, ready = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const TileCoord tc = decode_tile(p, tile, BN);
       const GemmTask& T = p.task[tc.task];
+      if (!task_ready(T, tc.task, ready, abort_flag, p.err)) break;
       for (int kb = 0; kb < tc.kblocks; ++kb, ++kbg) {
         const uint32_t s = kbg % kStages;
         if (kbg >= kStages && !mbar_wait(&empty_bar[s], ((kbg / kStages) - 1) & 1, abort_flag, p.err)) {
@@ -516,11 +528,22 @@ struct PairLayout {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
+// Dynamic tile scheduling (GemmParams::tile_counter set): the leader's producer
+// takes the next tile index from the counter and hands it to every role of both
+// CTAs through a ring of kTileRing slots in shared memory (tile_full in each CTA,
+// tile_empty in the leader, counting one arrival per consumer: the leader's MMA
+// thread, the peer's producer and the eight epilogue warps of each CTA). -1 ends
+// the sequence. A pair that starts late (its SMs still busy with another kernel)
+// then takes only the tiles that are left.
+constexpr int kTileRing = 4;
+constexpr int kTileConsumers = 1 + 1 + 2 * 8;
+
 template <bool kHeld>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::kThreadsT, 1)
     gemm_pair_kernel(const __grid_constant__ GemmParams p) {
   using Lay = PairLayout<kHeld>;
   constexpr int kStagesT = Lay::kStages;
+  static_assert((2 * kStagesT + 4 + 2 + 2 * kTileRing) * 8 + 4 * kTileRing + 8 <= 256, "barrier region");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Lay::kBarOffset);
@@ -529,13 +552,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
   uint64_t* acc_empty = acc_full + 2;         // [2] (used in the leader)
   uint64_t* held_full = acc_empty + 2;        // kHeld: this CTA's held rows landed
   uint64_t* held_empty = held_full + 1;       // kHeld: this CTA's epilogue is done with them
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(held_empty + 1);
+  uint64_t* tile_full = held_empty + 1;       // [kTileRing] dynamic tiles
+  uint64_t* tile_empty = tile_full + kTileRing;  // [kTileRing] (used in the leader)
+  volatile int* tile_slot = reinterpret_cast<volatile int*>(tile_empty + kTileRing);  // [kTileRing]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(tile_slot) + kTileRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* held_smem = smem + Lay::kHeldOffset;
 
   const int warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const bool dyn = p.tile_counter != nullptr;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesT; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -547,6 +574,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
     }
     mbar_init(held_full, 1);
     mbar_init(held_empty, kEpiThreads);
+    for (int r = 0; r < kTileRing; ++r) {
+      mbar_init(&tile_full[r], 1);
+      mbar_init(&tile_empty[r], kTileConsumers);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -559,6 +590,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int ntiles = p.total_tiles;
+  // The it-th tile of this pair, or -1 when there are no more. Dynamic mode:
+  // `fetch` (the leader's producer) takes it from the counter and publishes it;
+  // every other caller reads it from the ring; `elected` callers (one lane per
+  // warp, or the single-thread roles) arrive on the leader's tile_empty.
+  auto next_tile = [&](int it, bool fetch, bool elected) -> int {
+    if (!dyn) {
+      const int t = pair + it * npairs;
+      return t < ntiles ? t : -1;
+    }
+    const int slot = it % kTileRing;
+    int t = -1;
+    if (fetch) {
+      if (it >= kTileRing && !mbar_wait(&tile_empty[slot], ((it / kTileRing) - 1) & 1, abort_flag, p.err)) return -1;
+      t = static_cast<int>(atomicAdd(p.tile_counter, 1u));
+      if (t >= ntiles) t = -1;
+      tile_slot[slot] = t;
+      st_cluster_u32(mapa_shared(smem_u32(const_cast<int*>(&tile_slot[slot])), 1), static_cast<uint32_t>(t));
+      mbar_arrive(&tile_full[slot]);
+      mbar_arrive_cluster(mapa_shared(smem_u32(&tile_full[slot]), 1));
+      return t;
+    }
+    if (elected) {
+      if (!mbar_wait_cluster(&tile_full[slot], (it / kTileRing) & 1, abort_flag, p.err)) return -1;
+      t = tile_slot[slot];
+      mbar_arrive_cluster(mapa_shared(smem_u32(&tile_empty[slot]), 0));
+    }
+    return t;
+  };
   // held rows: coarse branch c occupies [held_off[c], +4 boxes)
   int held_off[2] = {0, 0}, held_box[2] = {0, 0};
   if (kHeld) {
@@ -575,11 +634,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
       prefetch_tmap(&p.task[t].tmA);
       prefetch_tmap(&p.task[t].tmB);
     }
-    uint32_t kbg = 0;
+    uint32_t kbg = 0, ready = 0;
     bool ok = true;
-    for (int tile = pair; tile < ntiles && ok; tile += npairs) {
+    for (int it = 0; ok; ++it) {
+      const int tile = next_tile(it, rank == 0, true);
+      if (tile < 0) break;
       const TileCoord tc = decode_tile(p, tile, kPairBN, kPairBM);
       const GemmTask& T = p.task[tc.task];
+      if (!task_ready(T, tc.task, ready, abort_flag, p.err)) break;
       const int arow = tc.m0 + 128 * static_cast<int>(rank);
       const int brow = tc.n0 + static_cast<int>(rank) * (tc.n_eff >> 1);
       for (int kb = 0; kb < tc.kblocks; ++kb, ++kbg) {
@@ -598,9 +660,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
     }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ---------------- MMA issuer (leader only)
-    uint32_t kbg = 0, it = 0;
+    uint32_t kbg = 0;
     bool ok = true;
-    for (int tile = pair; tile < ntiles && ok; tile += npairs, ++it) {
+    for (uint32_t it = 0; ok; ++it) {
+      const int tile = next_tile(static_cast<int>(it), false, true);
+      if (tile < 0) break;
       const TileCoord tc = decode_tile(p, tile, kPairBN, kPairBM);
       const uint32_t buf = it & 1;
       if (it >= 2 && !mbar_wait(&acc_empty[buf], ((it >> 1) - 1) & 1, abort_flag, p.err)) break;
@@ -625,7 +689,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
       if (ok) umma_commit_pair(&acc_full[buf], 0x3);
     }
   } else if (kHeld && warp == 10) {
-    // ---------------- held coarse rows of this CTA's tiles (one tile ahead at most)
+    // ---------------- held coarse rows of this CTA's tiles (one tile ahead at most;
+    // the fused launch schedules its tiles statically)
     if (lane == 0) {
       const GemmTask& T = p.task[0];
       for (int c = 0; c < 2 && c < T.n_coarse; ++c) prefetch_tmap(&T.tmOut[1 + c]);
@@ -653,8 +718,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
     const Stager stg{smem + Lay::kStagingOffset + (warp - 2) * (kHeld ? 1 : 2) * kStagerBytes, lane, !kHeld};
     int sel = 0;
     if (lane == 0) prefetch_out_maps(p);
-    uint32_t it = 0;
-    for (int tile = pair; tile < ntiles; tile += npairs, ++it) {
+    for (uint32_t it = 0;; ++it) {
+      int tile = next_tile(static_cast<int>(it), false, lane == 0);
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      if (tile < 0) break;
       TileCoord tc = decode_tile(p, tile, kPairBN, kPairBM);
       tc.m0 += 128 * static_cast<int>(rank);
       const uint32_t buf = it & 1;
@@ -736,13 +803,14 @@ int max_active_pairs() {
   return n;
 }
 
-cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st) {
+cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pairs) {
   if (p.total_tiles <= 0) return cudaSuccess;
   // the fused output launch with one or two coarse branches stages their held
   // rows in shared memory (the caller encodes tmOut[1 + c] for them)
   const bool held = p.n_tasks == 1 && p.task[0].epi == kEpiFuse && p.task[0].n_coarse >= 1 &&
                     p.task[0].n_coarse <= 2 && held_rows_fit(p.task[0].coarse_scale, p.task[0].n_coarse);
-  const int pairs = (bn != 256) ? 0 : held ? max_active_pairs<true>() : max_active_pairs<false>();
+  int pairs = (bn != 256) ? 0 : held ? max_active_pairs<true>() : max_active_pairs<false>();
+  if (max_pairs > 0 && pairs > max_pairs) pairs = max_pairs;
   if (pairs > 0) {
     // re-tile every task in 256 x 256 pair tiles
     static thread_local GemmParams q;
@@ -765,7 +833,8 @@ cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st) {
       gemm_pair_kernel<false><<<2 * grid_pairs, PairLayout<false>::kThreadsT, PairLayout<false>::kSmemBytes, st>>>(q);
     return cudaGetLastError();
   }
-  const int grid = p.total_tiles < sm_count() ? p.total_tiles : sm_count();
+  int grid = p.total_tiles < sm_count() ? p.total_tiles : sm_count();
+  if (max_pairs > 0 && grid > 2 * max_pairs) grid = 2 * max_pairs;
   if (bn == 256) {
     const int smem = GemmLayout<256>::kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
   const size_t seq_slot = ((static_cast<size_t>(b) * T.heads + head) * T.v_tiles + vt) * T.n_segs;
 
   const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0 && p.started && !state_pass) atomicAdd(p.started, 1ull);
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], 1);
     mbar_init(&bar[B_A_READY], 128);
@@ -380,6 +381,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (threadIdx.x == 0 && p.done && !state_pass) {
+    // every o row of this CTA is stored (the barrier above orders the stores of
+    // all its threads before this release)
+    __threadfence();
+    atomicAdd(p.done + ti, 1ull);
+  }
 }
 
 // Initial state of every segment: S'_init(s+1) = G_s * S'_init(s) + A_s with
@@ -406,7 +413,21 @@ __global__ void gla_scan_kernel(const __grid_constant__ GlaParams p, int B) {
   }
 }
 
+__global__ void wait_started_kernel(const unsigned long long* started, unsigned long long target, int* err) {
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    wait_count(started, target, &abort_flag, err);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_wait_started(const unsigned long long* started, unsigned long long target, int* err,
+                                cudaStream_t st) {
+  wait_started_kernel<<<1, 32, 0, st>>>(started, target, err);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gla_scan(const GlaParams& p, int B, cudaStream_t st) {
   size_t n = 0;

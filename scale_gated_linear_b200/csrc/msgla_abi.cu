@@ -140,6 +140,15 @@ struct msgla_handle {
   float* bfuse;
   int* d_err;  // device error word
   int test_skip_arrival;  // failure-detection tests (msgla_test_skip_arrival)
+  // Coarse output projection overlapped with the GLA kernel: a second stream,
+  // fork/join events, and per-branch GLA completion counters (monotonic) with
+  // the host's running count of GLA CTAs launched against each.
+  cudaStream_t side;
+  cudaEvent_t ev_fork, ev_join;
+  unsigned long long* d_gla_done;  // [MSGLA_MAX_SCALES] completion, then [1] start counter
+  unsigned long long gla_total[MSGLA_MAX_SCALES];
+  unsigned long long gla_started;
+  unsigned int* d_tiles;           // dynamic tile counter of the overlapped GEMM
 };
 
 namespace {
@@ -275,6 +284,11 @@ void free_handle(msgla_handle* h) {
   cudaFree(h->Wfuse);
   cudaFree(h->bfuse);
   cudaFree(h->d_err);
+  cudaFree(h->d_gla_done);
+  cudaFree(h->d_tiles);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
+  if (h->side) cudaStreamDestroy(h->side);
   delete h;
 }
 
@@ -351,6 +365,13 @@ int create_impl(msgla_handle* h, const msgla_weights* w) {
   CUDA_TRY(cudaMemcpy(h->Wfuse, w->Wfuse, static_cast<size_t>(h->n_scales) * d * 2, cudaMemcpyDeviceToDevice));
   if (w->bfuse) CUDA_TRY(cudaMemcpy(h->bfuse, w->bfuse, h->n_scales * 4, cudaMemcpyDeviceToDevice));
   if ((st = dmalloc_zero(&h->d_err, sizeof(int)))) return st;
+  if ((st = dmalloc_zero(&h->d_gla_done, (MSGLA_MAX_SCALES + 1) * sizeof(unsigned long long)))) return st;
+  if ((st = dmalloc_zero(&h->d_tiles, sizeof(unsigned int)))) return st;
+  for (int j = 0; j < MSGLA_MAX_SCALES; ++j) h->gla_total[j] = 0;
+  h->gla_started = 0;
+  CUDA_TRY(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
+  CUDA_TRY(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
+  CUDA_TRY(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
   CUDA_TRY(cudaDeviceSynchronize());
   int over = 0;
   CUDA_TRY(cudaMemcpy(&over, d_over, sizeof(int), cudaMemcpyDeviceToHost));
@@ -363,12 +384,31 @@ struct Recorder {
   void* const* events = nullptr;
   int max_events = 0;
   int n = 0;
+  int unmarked = 0;  // launches on the second stream (no event of their own)
   cudaError_t mark(cudaStream_t st) {
     if (!events) return cudaSuccess;
     if (n + 1 >= max_events) return cudaErrorInvalidValue;
     return cudaEventRecord(static_cast<cudaEvent_t>(events[++n]), st);
   }
 };
+
+// Whether the coarse output projection runs concurrently with the GLA kernel on
+// the second stream: with a scale-1 branch, no sequence segments, no head norm,
+// and GLA CTAs (one per SM) that leave SMs free. The GEMM starts only once every
+// GLA CTA is resident (launch_wait_started) and takes its tiles dynamically, so
+// it runs on the SMs the GLA leaves free and on those its coarse-branch CTAs
+// release, and it can never keep a GLA CTA from starting.
+bool coarse_overlap(const msgla_handle* h, const Workspace& ws, int B, long long* gla_ctas) {
+  *gla_ctas = 0;
+  if (h->main_index < 0 || h->n_scales < 2 || h->cfg.head_norm) return false;
+  long long ctas = 0;
+  for (int j = 0; j < h->n_scales; ++j) {
+    if (ws.br[j].n_segs > 1) return false;
+    ctas += static_cast<long long>(B) * h->br[j].heads * (h->dvp / kGlaTile);
+  }
+  *gla_ctas = ctas;
+  return h->sm_count - ctas >= 2;
+}
 
 int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* wsp, size_t ws_bytes,
                  cudaStream_t st, Recorder* rec = nullptr, const uint8_t* M = nullptr) {
@@ -551,7 +591,20 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   lp.mode = 0;
   lp.skip_arrival = h->test_skip_arrival;
   h->test_skip_arrival = 0;
+  long long gla_ctas = 0;
+  const bool overlap = coarse_overlap(h, ws, B, &gla_ctas);
+  if (overlap) {
+    // the second stream starts once the gates are done, alongside the GLA
+    lp.done = h->d_gla_done;
+    lp.started = h->d_gla_done + MSGLA_MAX_SCALES;
+    CUDA_TRY(cudaEventRecord(h->ev_fork, st));
+  }
   CUDA_TRY(launch_gla(lp, st));
+  if (overlap) {
+    for (int j = 0; j < ns; ++j)
+      h->gla_total[j] += static_cast<unsigned long long>(B) * lp.task[j].heads * lp.task[j].v_tiles;
+    h->gla_started += static_cast<unsigned long long>(gla_ctas);
+  }
   CUDA_TRY(rec->mark(st));
 
   // 4b. optional per-head RMS norm of the GLA output (in place)
@@ -577,12 +630,15 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     CUDA_TRY(rec->mark(st));
   }
 
-  // 5. coarse branches: Y^(s) = o W_o^T (fp16)
+  // 5. coarse branches: Y^(s) = o W_o^T (fp16). Overlapped with the GLA, the
+  // branches with the fewest chunks (largest scale) come first: their GLA CTAs
+  // finish first.
   memset(&gp, 0, sizeof(gp));
   gp.err = h->d_err;
   tiles = 0;
   int nt = 0;
-  for (int j = 0; j < ns; ++j) {
+  for (int jj = 0; jj < ns; ++jj) {
+    const int j = overlap ? ns - 1 - jj : jj;
     if (j == h->main_index) continue;
     const Branch& b = h->br[j];
     const BranchWs& bw = ws.br[j];
@@ -601,13 +657,28 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.y = static_cast<__half*>(at(bw.Y));
     if (!encode_out_3d(&t.tmOut[0], false, t.y, d, bw.rows, B))
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (output store, scale %d)", b.scale);
+    if (overlap) {
+      t.dep = h->d_gla_done + j;
+      t.dep_target = h->gla_total[j];
+    }
     tiles += B * t.m_tiles * t.n_tiles;
   }
   if (nt > 0) {
     gp.n_tasks = nt;
     gp.total_tiles = tiles;
-    CUDA_TRY(launch_gemm(gp, 256, st));
-    CUDA_TRY(rec->mark(st));
+    if (overlap) {
+      CUDA_TRY(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+      CUDA_TRY(launch_wait_started(h->d_gla_done + MSGLA_MAX_SCALES, h->gla_started, h->d_err, h->side));
+      CUDA_TRY(cudaMemsetAsync(h->d_tiles, 0, sizeof(unsigned int), h->side));
+      gp.tile_counter = h->d_tiles;
+      CUDA_TRY(launch_gemm(gp, 256, h->side));
+      rec->unmarked += 2;
+      CUDA_TRY(cudaEventRecord(h->ev_join, h->side));
+      CUDA_TRY(cudaStreamWaitEvent(st, h->ev_join, 0));
+    } else {
+      CUDA_TRY(launch_gemm(gp, 256, st));
+      CUDA_TRY(rec->mark(st));
+    }
   }
 
   // 6. scale-1 branch fused with hold + fusion, or the stand-alone hold + fusion
@@ -973,6 +1044,10 @@ int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weight
   if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", device);
   msgla_handle* h = new msgla_handle();
   memset(h->br, 0, sizeof(h->br));
+  h->side = nullptr;
+  h->ev_fork = h->ev_join = nullptr;
+  h->d_gla_done = nullptr;
+  h->d_tiles = nullptr;
   h->Wfuse = nullptr;
   h->bfuse = nullptr;
   h->d_err = nullptr;
@@ -1114,7 +1189,7 @@ int msgla_forward_profiled(msgla_handle* h, const void* X, const void* M, int B,
   rec.max_events = max_events;
   st = forward_impl(h, X, B, L, O, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), &rec,
                     static_cast<const uint8_t*>(M));
-  *n_launches = rec.n;
+  *n_launches = rec.n + rec.unmarked;
   return st;
 }
 
@@ -1274,8 +1349,12 @@ int msgla_launch_plan(const msgla_handle* h, int B, int L, char* names, size_t l
     }
     add_name("gla");
     if (h->cfg.head_norm) add_name("head_norm");
+    long long gla_ctas = 0;
+    const bool overlap = coarse_overlap(h, ws, B, &gla_ctas);
     if (h->main_index >= 0) {
-      if (h->n_scales > 1) add_name("out_gemm_coarse");
+      // overlapped with the GLA on the second stream, the coarse output GEMM has
+      // no interval of its own on the caller's stream
+      if (h->n_scales > 1 && !overlap) add_name("out_gemm_coarse");
       add_name("out_gemm_fused");
     } else {
       add_name("out_gemm_coarse");

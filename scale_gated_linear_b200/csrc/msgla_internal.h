@@ -51,6 +51,10 @@ struct alignas(64) GemmTask {
   const float* bfuse;  // [n_scales]
   float* w;            // fusion weights [B, L, n_scales] (written by the n0 == 0 tiles)
   int n_scales, main_index, n_coarse, pad_;
+  // A operand produced by a kernel running concurrently (the GLA of this branch
+  // on the other stream): loads start once *dep >= dep_target (null: no wait)
+  const unsigned long long* dep;
+  unsigned long long dep_target;
   int coarse_scale[kMaxScales];
   int coarse_index[kMaxScales];
   int coarse_rows[kMaxScales];
@@ -73,6 +77,8 @@ struct GemmParams {
   int n_tasks;
   int total_tiles;
   int* err;
+  // non-null: CTA pairs take tiles dynamically from *tile_counter (zero at launch)
+  unsigned int* tile_counter;
 };
 
 // Chunkwise GLA over one or more branches.
@@ -97,11 +103,22 @@ struct GlaParams {
   int mode;          // 0: full pass; 1: state pass over segments 0..n_segs-2
   int skip_arrival;  // failure-detection tests: CTA 0 omits one barrier arrival
   int* err;
+  // full pass only: every CTA of task t adds 1 to done[t] once its outputs are
+  // stored (release), for a concurrent consumer, and 1 to *started when it
+  // begins (null: none)
+  unsigned long long* done;
+  unsigned long long* started;
 };
+// Wait (one warp, bounded) until *started reaches target: ordered on a stream
+// before a kernel that may only take SMs once every CTA of a running GLA launch
+// is resident.
+cudaError_t launch_wait_started(const unsigned long long* started, unsigned long long target, int* err,
+                                cudaStream_t st);
 
 // ---------------------------------------------------------------- launchers
 // (each returns the cudaError_t of the launch)
-cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st);
+// max_pairs > 0 caps the number of CTA pairs of the persistent grid.
+cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pairs = 0);
 cudaError_t launch_gla(const GlaParams& p, cudaStream_t st);
 // initial state of every segment from the state pass's end states (sequential over segments)
 cudaError_t launch_gla_scan(const GlaParams& p, int B, cudaStream_t st);

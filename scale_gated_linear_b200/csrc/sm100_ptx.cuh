@@ -81,6 +81,66 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait with cluster-scope acquire: for data another CTA of the cluster
+// wrote into this CTA's shared memory before a release-cluster arrive.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  int* err) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (*abort_flag) return false;
+      const uint64_t now = globaltimer_ns();
+      if (it == 0 || now < t0) t0 = now;
+      if (now - t0 > kWaitTimeoutNs) {
+        *abort_flag = 1;
+        atomicCAS(err, 0, kDevTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait until the 64-bit counter at `c` (global memory, advanced by other
+// CTAs with release semantics) reaches `target`; acquire ordering. Same error
+// behaviour as mbar_wait.
+__device__ __forceinline__ bool wait_count(const unsigned long long* c, unsigned long long target,
+                                           volatile int* abort_flag, int* err) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(c) : "memory");
+    if (v >= target) return true;
+    if ((it & 15u) == 0) {
+      if (*abort_flag) return false;
+      const uint64_t now = globaltimer_ns();
+      if (it == 0 || now < t0) t0 = now;
+      if (now - t0 > kWaitTimeoutNs) {
+        *abort_flag = 1;
+        atomicCAS(err, 0, kDevTimeout);
+        return false;
+      }
+    }
+    __nanosleep(256);
+  }
+}
+// Orders this thread's earlier generic-proxy accesses (such as the acquire
+// above) before its later async-proxy (TMA) accesses of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* smem, int c0,
                                             int c1) {
@@ -245,6 +305,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
+}
+// 32-bit store into shared memory given by its shared::cluster address (possibly
+// in the peer CTA).
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 // Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
