@@ -184,8 +184,14 @@ int msgla_workspace_size_host(const msgla_handle* h, int B, int L, size_t* bytes
 
 /* Host-buffer forward: copies X (HOST bf16 [B, L, d]) to the device part of
  * `workspace`, runs the layer, copies O back to HOST bf16 [B, L, d] and
- * synchronises `stream`. Pinned host memory gives the fastest copies. Returns the
- * status of the whole call, including device-side errors. */
+ * synchronises. The batch goes through in chunks of whole sequences (one
+ * sequence first and last, max(2, ceil((B - 2) / 4)) in each chunk between): the
+ * upload of the next chunk and the download of the previous one run
+ * on two copy streams owned by the handle while the current chunk's forward runs
+ * on `stream`, so PCIe transfers in both directions overlap each other and the
+ * compute. Pinned host memory is needed for that overlap (pageable memory works,
+ * with staged copies). Returns the status of the whole call, including
+ * device-side errors. */
 int msgla_forward_host(msgla_handle* h, const void* X_host, int B, int L, void* O_host,
                        void* workspace, size_t workspace_bytes, void* stream);
 

@@ -149,6 +149,9 @@ struct msgla_handle {
   unsigned long long gla_total[MSGLA_MAX_SCALES];
   unsigned long long gla_started;
   unsigned int* d_tiles;           // dynamic tile counter of the overlapped GEMM
+  // host-buffer forward: copy streams and events of its pipeline
+  cudaStream_t copy_in, copy_out;
+  cudaEvent_t ev_start, ev_in, ev_done;
 };
 
 namespace {
@@ -286,6 +289,10 @@ void free_handle(msgla_handle* h) {
   cudaFree(h->d_err);
   cudaFree(h->d_gla_done);
   cudaFree(h->d_tiles);
+  for (cudaEvent_t e : {h->ev_start, h->ev_in, h->ev_done})
+    if (e) cudaEventDestroy(e);
+  if (h->copy_in) cudaStreamDestroy(h->copy_in);
+  if (h->copy_out) cudaStreamDestroy(h->copy_out);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
   if (h->ev_join) cudaEventDestroy(h->ev_join);
   if (h->side) cudaStreamDestroy(h->side);
@@ -372,6 +379,11 @@ int create_impl(msgla_handle* h, const msgla_weights* w) {
   CUDA_TRY(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
   CUDA_TRY(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
   CUDA_TRY(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
+  CUDA_TRY(cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking));
+  CUDA_TRY(cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking));
+  CUDA_TRY(cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming));
+  CUDA_TRY(cudaEventCreateWithFlags(&h->ev_in, cudaEventDisableTiming));
+  CUDA_TRY(cudaEventCreateWithFlags(&h->ev_done, cudaEventDisableTiming));
   CUDA_TRY(cudaDeviceSynchronize());
   int over = 0;
   CUDA_TRY(cudaMemcpy(&over, d_over, sizeof(int), cudaMemcpyDeviceToHost));
@@ -1048,6 +1060,8 @@ int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weight
   h->ev_fork = h->ev_join = nullptr;
   h->d_gla_done = nullptr;
   h->d_tiles = nullptr;
+  h->copy_in = h->copy_out = nullptr;
+  h->ev_start = h->ev_in = h->ev_done = nullptr;
   h->Wfuse = nullptr;
   h->bfuse = nullptr;
   h->d_err = nullptr;
@@ -1212,10 +1226,37 @@ int msgla_forward_host(msgla_handle* h, const void* X_host, int B, int L, void* 
   uint8_t* Xd = static_cast<uint8_t*>(workspace) + core;
   uint8_t* Od = Xd + round_up(nbytes, 256);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  CUDA_TRY(cudaMemcpyAsync(Xd, X_host, nbytes, cudaMemcpyHostToDevice, s));
-  st = forward_impl(h, Xd, B, L, Od, workspace, core, s);
-  if (st) return st;
-  CUDA_TRY(cudaMemcpyAsync(O_host, Od, nbytes, cudaMemcpyDeviceToHost, s));
+  // Pipeline over chunks of whole sequences: the upload of chunk c + 1 (copy_in)
+  // and the download of chunk c - 1 (copy_out) overlap the forward of chunk c on
+  // `stream`; the chunks' forwards run one after another in the workspace's core
+  // region (sized for all B sequences). One sequence first and last keeps the
+  // pipeline's fill and drain short; the chunks between hold
+  // max(2, ceil((B - 2) / 4)) sequences, so their forwards stay efficient
+  // enough to hide under the copies.
+  const int mid = B <= 2 ? 1 : std::max(2, (B - 2 + 3) / 4);
+  const size_t row_bytes = static_cast<size_t>(L) * h->cfg.d * 2;  // one sequence
+  const uint8_t* Xh = static_cast<const uint8_t*>(X_host);
+  uint8_t* Oh = static_cast<uint8_t*>(O_host);
+  CUDA_TRY(cudaEventRecord(h->ev_start, s));
+  CUDA_TRY(cudaStreamWaitEvent(h->copy_in, h->ev_start, 0));
+  for (int b0 = 0; b0 < B;) {
+    const int bc = (b0 == 0 || B - b0 <= 1) ? 1 : std::min(mid, B - b0 - 1);
+    const size_t off = static_cast<size_t>(b0) * row_bytes, bytes = static_cast<size_t>(bc) * row_bytes;
+    CUDA_TRY(cudaMemcpyAsync(Xd + off, Xh + off, bytes, cudaMemcpyHostToDevice, h->copy_in));
+    CUDA_TRY(cudaEventRecord(h->ev_in, h->copy_in));
+    CUDA_TRY(cudaStreamWaitEvent(s, h->ev_in, 0));
+    st = forward_impl(h, Xd + off, bc, L, Od + off, workspace, core, s);
+    if (st) {
+      cudaStreamSynchronize(h->copy_in);
+      cudaStreamSynchronize(h->copy_out);
+      return st;
+    }
+    CUDA_TRY(cudaEventRecord(h->ev_done, s));
+    CUDA_TRY(cudaStreamWaitEvent(h->copy_out, h->ev_done, 0));
+    CUDA_TRY(cudaMemcpyAsync(Oh + off, Od + off, bytes, cudaMemcpyDeviceToHost, h->copy_out));
+    b0 += bc;
+  }
+  CUDA_TRY(cudaStreamSynchronize(h->copy_out));
   CUDA_TRY(cudaStreamSynchronize(s));
   int err = 0;
   CUDA_TRY(cudaMemcpy(&err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost));
