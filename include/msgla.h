@@ -168,7 +168,10 @@ int msgla_forward_noalloc(msgla_handle* h, const void* X, int B, int L, void* O,
 /* msgla_forward that also records CUDA events around its kernels, for timing each
  * kernel on `stream` with events. `events` holds caller-created cudaEvent_t
  * handles: events[0] is recorded before the first kernel and events[i+1] after
- * the i-th kernel; msgla_launch_plan lists the kernels in launch order.
+ * the i-th kernel; msgla_launch_plan lists the kernels in launch order. A NULL
+ * entry skips that record: the kernels are launched so that each may start
+ * while the previous one finishes, and an event recorded between two kernels
+ * takes that overlap away, so time only the boundaries needed.
  * `max_events` is the length of `events` (it must be at least the number of
  * msgla_launch_plan entries + 1); *n_launches receives the number of kernels
  * launched, which includes the kernels run on the second stream (the coarse

@@ -174,16 +174,17 @@ class MSGLA:
 
     def forward_profiled(self, X, out, workspace, events, stream=None, mask=None):
         """forward() recording events[0] before the first kernel and events[i+1]
-        after kernel i (torch.cuda.Event objects with timing enabled). Returns the
-        number of kernels launched. ``mask`` as for forward()."""
+        after kernel i (torch.cuda.Event objects with timing enabled; None skips a
+        record -- an event between two kernels keeps the second from starting
+        early). Returns the number of kernels launched. ``mask`` as for forward()."""
         import torch
         B, L, d = X.shape
         if stream is None:
             stream = torch.cuda.current_stream(X.device)
         for e in events:  # torch creates the underlying cudaEvent_t on first record
-            if not e.cuda_event:
+            if e is not None and not e.cuda_event:
                 e.record(stream)
-        arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        arr = (ctypes.c_void_p * len(events))(*[None if e is None else e.cuda_event for e in events])
         n = ctypes.c_int()
         if mask is not None:
             assert mask.shape == (B, L) and mask.is_cuda and mask.is_contiguous()

@@ -33,6 +33,8 @@ constexpr int kPoolThreads = 128;
 
 // grid (ceil(L / block_rows), B); each thread owns 8 consecutive columns at a time.
 __global__ void __launch_bounds__(kPoolThreads) pool_fuse_kernel(const PoolParams p) {
+  griddep_wait();
+  griddep_launch();
   __shared__ float logit[64 * kMaxScales];
   const int b = blockIdx.y;
   const int row0 = blockIdx.x * p.block_rows;
@@ -147,6 +149,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_fuse_kernel(const PoolParam
 // the end. NS bounds the number of scales held in registers.
 template <int P, int GPL, int NS>
 __global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p) {
+  griddep_wait();
+  griddep_launch();
   extern __shared__ float wf_s[];  // [n_scales][d] fp32
   const int ns = p.n_scales;
   for (int i = threadIdx.x; i < ns * p.d; i += blockDim.x) wf_s[i] = __bfloat162float(p.Wfuse[i]);
@@ -258,6 +262,8 @@ __global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p)
 // (sequence, block of P rows, 8 columns); all P row loads are issued together.
 template <int P>
 __global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
+  griddep_wait();
+  griddep_launch();
   const int groups = p.d / 8;
   const int nblk = (p.L + P - 1) / P;
   const size_t gid = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
@@ -347,6 +353,8 @@ __global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
 // scaled; the padding columns are zero and stay zero (their weight is zero).
 constexpr int kNormMaxLoads = 4;  // 16-byte loads per lane: 4 * 32 * 8 = 1024 values
 __global__ void __launch_bounds__(256) head_norm_kernel(const HeadNormParams p) {
+  griddep_wait();
+  griddep_launch();
   const long long gw = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (gw >= p.total_warps) return;
   int j = 0;
@@ -467,6 +475,8 @@ struct GateSmem {
 
 template <int RP>
 __global__ void __launch_bounds__(kGateThreads, 3) gate_kernel(const __grid_constant__ GateParams p) {
+  griddep_wait();
+  griddep_launch();
   using L = GateSmem<RP>;
   extern __shared__ __align__(16) uint8_t gate_smem[];
   __half* qk_s = reinterpret_cast<__half*>(gate_smem);
@@ -660,12 +670,13 @@ cudaError_t launch_gate_t(const GateParams& p, cudaStream_t st) {
   const int smem = GateSmem<RP>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(gate_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  gate_kernel<RP><<<p.total_blocks, kGateThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(gate_kernel<RP>, dim3(p.total_blocks), dim3(kGateThreads), smem, st, p);
 }
 
 // one thread per 8 output columns of one row; flat grid over B*L*(d/8)
 __global__ void hold_fuse_kernel(const HoldFuseParams p) {
+  griddep_wait();
+  griddep_launch();
   const int groups = p.d / 8;
   const size_t gid = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
   if (gid >= static_cast<size_t>(p.B) * p.L * groups) return;
@@ -727,15 +738,14 @@ cudaError_t launch_pool_rows(const PoolParams& p, cudaStream_t st) {
       cudaFuncSetAttribute(pool_fuse_rows_kernel<P, GPL, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const size_t warps = static_cast<size_t>(p.B) * ((p.L + P - 1) / P);
-  pool_fuse_rows_kernel<P, GPL, NS><<<static_cast<unsigned>((warps + 7) / 8), 256, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(pool_fuse_rows_kernel<P, GPL, NS>, dim3(static_cast<unsigned>((warps + 7) / 8)), dim3(256), smem,
+                    st, p);
 }
 
 template <int P>
 cudaError_t launch_pool_only(const PoolParams& p, cudaStream_t st) {
   const size_t n = static_cast<size_t>(p.B) * ((p.L + P - 1) / P) * (p.d / 8);
-  pool_rows_kernel<P><<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(pool_rows_kernel<P>, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st, p);
 }
 
 cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st) {
@@ -760,15 +770,13 @@ cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st) {
   PoolParams q = p;
   while (q.block_rows < 32) q.block_rows *= 2;
   dim3 grid((p.L + q.block_rows - 1) / q.block_rows, p.B);
-  pool_fuse_kernel<<<grid, kPoolThreads, 0, st>>>(q);
-  return cudaGetLastError();
+  return launch_pdl(pool_fuse_kernel, grid, dim3(kPoolThreads), 0, st, q);
 }
 
 cudaError_t launch_head_norm(const HeadNormParams& p, cudaStream_t st) {
   if (p.total_warps <= 0) return cudaSuccess;
   if (p.dvp % 128 || p.dvp > kNormMaxLoads * 32 * 8) return cudaErrorInvalidValue;
-  head_norm_kernel<<<static_cast<unsigned>((p.total_warps + 7) / 8), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(head_norm_kernel, dim3(static_cast<unsigned>((p.total_warps + 7) / 8)), dim3(256), 0, st, p);
 }
 
 cudaError_t launch_gate(const GateParams& p, cudaStream_t st) {
@@ -780,8 +788,7 @@ cudaError_t launch_gate(const GateParams& p, cudaStream_t st) {
 cudaError_t launch_hold_fuse(const HoldFuseParams& p, cudaStream_t st) {
   if (p.B * p.L == 0) return cudaSuccess;
   const size_t n = static_cast<size_t>(p.B) * p.L * (p.d / 8);
-  hold_fuse_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(hold_fuse_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st, p);
 }
 
 cudaError_t launch_bf16_to_f16_rows(const __nv_bfloat16* src, int src_ld, int rows, int cols, __half* dst,

@@ -31,6 +31,8 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
 
 // one thread per (sequence, 8 columns)
 __global__ void __launch_bounds__(256) dec_pool_kernel(const DecPoolParams p) {
+  griddep_wait();
+  griddep_launch();
   const int groups = p.d / 8;
   const size_t gid = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
   if (gid >= static_cast<size_t>(p.B) * groups) return;
@@ -78,6 +80,8 @@ constexpr int kDecGroups = kDecThreads / 32;  // key-channel groups; a warp cove
 // of it is used, so the whole 128 KB tile is in flight at once. The partial
 // o = q S of the 16 channel groups are summed through shared memory.
 __global__ void __launch_bounds__(kDecThreads) dec_gla_kernel(const __grid_constant__ DecGlaParams p) {
+  griddep_wait();
+  griddep_launch();
   __shared__ float alpha_s[kDecMaxDk], q_s[kDecMaxDk], k_s[kDecMaxDk];
   __shared__ __align__(16) float v_s[kDecTile];
   __shared__ __align__(16) float red[kDecGroups][kDecTile];
@@ -153,6 +157,8 @@ __global__ void __launch_bounds__(kDecThreads) dec_gla_kernel(const __grid_const
 // One CTA (256 threads) per sequence: fusion logits from the token, softmax,
 // then the weighted sum of the branches' latest outputs, 8 columns per thread.
 __global__ void __launch_bounds__(256) dec_fuse_kernel(const DecFuseParams p) {
+  griddep_wait();
+  griddep_launch();
   __shared__ float red[8][kMaxScales];
   __shared__ float w_s[kMaxScales];
   const int b = blockIdx.x;
@@ -225,21 +231,18 @@ __global__ void __launch_bounds__(256) dec_fuse_kernel(const DecFuseParams p) {
 cudaError_t launch_dec_pool(const DecPoolParams& p, cudaStream_t st) {
   const size_t n = static_cast<size_t>(p.B) * (p.d / 8);
   if (n == 0) return cudaSuccess;
-  dec_pool_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(dec_pool_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st, p);
 }
 
 cudaError_t launch_dec_gla(const DecGlaParams& p, cudaStream_t st) {
   if (p.total_ctas <= 0) return cudaSuccess;
   if ((p.dkp != 128 && p.dkp != 256) || p.dvp % kDecTile) return cudaErrorInvalidValue;
-  dec_gla_kernel<<<p.total_ctas, kDecThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(dec_gla_kernel, dim3(p.total_ctas), dim3(kDecThreads), 0, st, p);
 }
 
 cudaError_t launch_dec_fuse(const DecFuseParams& p, cudaStream_t st) {
   if (p.B <= 0) return cudaSuccess;
-  dec_fuse_kernel<<<p.B, 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(dec_fuse_kernel, dim3(p.B), dim3(256), 0, st, p);
 }
 
 }  // namespace msgla

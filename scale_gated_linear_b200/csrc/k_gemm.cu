@@ -409,6 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();
+  griddep_launch();
   const uint32_t tmem = *tmem_slot;
   const int ntiles = p.total_tiles;
 
@@ -588,6 +590,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
+  griddep_wait();
+  griddep_launch();
   const uint32_t tmem = *tmem_slot;
   const int ntiles = p.total_tiles;
   // The it-th tile of this pair, or -1 when there are no more. Dynamic mode:
@@ -828,10 +832,10 @@ cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pa
     q.total_tiles = tiles;
     const int grid_pairs = tiles < pairs ? tiles : pairs;
     if (held)
-      gemm_pair_kernel<true><<<2 * grid_pairs, PairLayout<true>::kThreadsT, PairLayout<true>::kSmemBytes, st>>>(q);
-    else
-      gemm_pair_kernel<false><<<2 * grid_pairs, PairLayout<false>::kThreadsT, PairLayout<false>::kSmemBytes, st>>>(q);
-    return cudaGetLastError();
+      return launch_pdl(gemm_pair_kernel<true>, dim3(2 * grid_pairs), dim3(PairLayout<true>::kThreadsT),
+                        PairLayout<true>::kSmemBytes, st, q);
+    return launch_pdl(gemm_pair_kernel<false>, dim3(2 * grid_pairs), dim3(PairLayout<false>::kThreadsT),
+                      PairLayout<false>::kSmemBytes, st, q);
   }
   int grid = p.total_tiles < sm_count() ? p.total_tiles : sm_count();
   if (max_pairs > 0 && grid > 2 * max_pairs) grid = 2 * max_pairs;
@@ -839,12 +843,12 @@ cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pa
     const int smem = GemmLayout<256>::kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    gemm_kernel<256><<<grid, kThreads, smem, st>>>(p);
+    return launch_pdl(gemm_kernel<256>, dim3(grid), dim3(kThreads), smem, st, p);
   } else if (bn == 128) {
     const int smem = GemmLayout<128>::kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    gemm_kernel<128><<<grid, kThreads, smem, st>>>(p);
+    return launch_pdl(gemm_kernel<128>, dim3(grid), dim3(kThreads), smem, st, p);
   } else {
     return cudaErrorInvalidValue;
   }

@@ -106,6 +106,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();
+  griddep_launch();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
 
@@ -392,6 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
 // Initial state of every segment: S'_init(s+1) = G_s * S'_init(s) + A_s with
 // S'_init(0) = 0, written over A_s. One thread per state element of a sequence.
 __global__ void gla_scan_kernel(const __grid_constant__ GlaParams p, int B) {
+  griddep_wait();
+  griddep_launch();
   size_t gid = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
   for (int t = 0; t < p.n_tasks; ++t) {
     const GlaTask& T = p.task[t];
@@ -434,16 +438,14 @@ cudaError_t launch_gla_scan(const GlaParams& p, int B, cudaStream_t st) {
   for (int t = 0; t < p.n_tasks; ++t)
     n += static_cast<size_t>(B) * p.task[t].heads * p.task[t].v_tiles * p.task[t].dkp * kGlaTile;
   if (n == 0) return cudaSuccess;
-  gla_scan_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p, B);
-  return cudaGetLastError();
+  return launch_pdl(gla_scan_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st, p, B);
 }
 
 cudaError_t launch_gla(const GlaParams& p, cudaStream_t st) {
   if (p.total_ctas <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(gla_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  gla_chunk_kernel<<<p.total_ctas, kThreads, kSmemBytes, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(gla_chunk_kernel, dim3(p.total_ctas), dim3(kThreads), kSmemBytes, st, p);
 }
 
 }  // namespace msgla

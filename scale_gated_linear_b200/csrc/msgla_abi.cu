@@ -400,7 +400,8 @@ struct Recorder {
   cudaError_t mark(cudaStream_t st) {
     if (!events) return cudaSuccess;
     if (n + 1 >= max_events) return cudaErrorInvalidValue;
-    return cudaEventRecord(static_cast<cudaEvent_t>(events[++n]), st);
+    ++n;
+    return events[n] ? cudaEventRecord(static_cast<cudaEvent_t>(events[n]), st) : cudaSuccess;
   }
 };
 
@@ -428,7 +429,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   if (!rec) rec = &none;
   if (rec->events) {
     if (rec->max_events < 1) return fail(MSGLA_ERR_INVALID_ARG, "max_events < 1");
-    CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(rec->events[0]), st));
+    if (rec->events[0]) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(rec->events[0]), st));
   }
   const msgla_config& c = h->cfg;
   const int d = c.d;

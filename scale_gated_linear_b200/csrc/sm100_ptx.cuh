@@ -366,6 +366,16 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mas
       : "memory");
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Kernels of the forward are launched with programmatic stream serialisation:
+// the next kernel may start (and run its prologue) while this one finishes.
+// griddep_wait blocks until every prerequisite grid has completed and its memory
+// is visible -- call it in every thread before touching data an earlier kernel
+// wrote (a no-op without a programmatic prerequisite); griddep_launch lets the
+// next kernel start launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
