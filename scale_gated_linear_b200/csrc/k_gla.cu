@@ -22,6 +22,7 @@
 //   warp 0        TMA loads of Qs, Ks (128 x dkp) and V (128 x 128)
 //   warp 1        TMEM allocation (512 columns) + tcgen05.mma issue
 //   warps 4..7    score epilogue (mask, fp16 back into TMEM) and the o store
+//                 (staged in the V buffer once A V is done, TMA tile stores)
 //   warps 8..15   state epilogue: S' <- factor * S' in TMEM and its fp16 copy
 //                 for the next chunk's Qs S' product (d_k rows 0..127 / 128..255)
 // TMEM columns: [0,256) S' (two 128-lane halves of d_k), [256,384) o,
@@ -96,6 +97,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
     mbar_init(&bar[B_A_READY], 128);
     mbar_init(&bar[B_O_EMPTY], 128);
     mbar_init(&bar[B_S_DONE], 128 * n_half);
+    // full pass: the four output warps release V once their staged o tile is read
+    mbar_init(&bar[B_V_EMPTY], state_pass ? 1 : 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -209,7 +212,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
           umma_f16_ts(tmem + kColO, tmem + kColA + ks * 8, sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_km,
                       (carried || ks > 0) ? 1u : 0u);
         umma_commit(&bar[B_O_FULL]);
-        umma_commit(&bar[B_V_EMPTY]);
         if (c + 1 < nch) {
           if (!mbar_wait(&bar[B_Q_FULL], ph ^ 1, abort_flag, p.err)) break;
           if (!mbar_wait(&bar[B_K_FULL], ph ^ 1, abort_flag, p.err)) break;
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
     // ---------------- scores -> fp16 in TMEM, then the output rows
     const int quad = warp & 3;
     const int i = quad * 32 + lane;  // chunk row (TMEM lane)
-    const size_t ld_o = static_cast<size_t>(T.heads) * T.dvp;
+    if (lane == 0 && !state_pass) prefetch_tmap(&T.tmO);
     for (int c = 0; c < nch && !state_pass; ++c) {
       if (!mbar_wait(&bar[B_A_FULL], c & 1, abort_flag, p.err)) break;
       tc_fence_after();
@@ -252,33 +254,49 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
 
       if (!mbar_wait(&bar[B_O_FULL], c & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      const int t = (c_begin + c) * kC + i;
-      __half* dst = T.o + (static_cast<size_t>(b) * T.rows + t) * ld_o + head * T.dvp + vt * kGlaTile;
+      // o rows of this warp, scaled and rounded to fp16, staged in the V buffer
+      // (free: A V has completed) with the 128-byte swizzle of the TMA store,
+      // which writes whole 128-byte rows instead of 16-byte pieces of 32 rows
+      uint8_t* stage = smem + kOffV + quad * 8192;
 #pragma unroll 1
       for (int h2 = 0; h2 < 2; ++h2) {
         uint32_t ra[32], rb[32];
         const uint32_t src = tmem_addr(tmem, quad * 32, kColO + h2 * 64);
         tmem_ld32(src, ra);
         tmem_ld32(src + 32, rb);
-        tmem_wait_ld();
+        tmem_wait_ld(ra);
+        tmem_wait_ld(rb);
         if (h2 == 1) {
           tc_fence_before();
           mbar_arrive(&bar[B_O_EMPTY]);
         }
-        if (t < T.rows) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + h2 * 64);
+        uint8_t* row = stage + h2 * 4096 + lane * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint32_t* r = q < 4 ? ra + 8 * q : rb + 8 * (q - 4);
-            uint4 u;
-            u.x = pack_half2(p.qk_scale * __uint_as_float(r[0]), p.qk_scale * __uint_as_float(r[1]));
-            u.y = pack_half2(p.qk_scale * __uint_as_float(r[2]), p.qk_scale * __uint_as_float(r[3]));
-            u.z = pack_half2(p.qk_scale * __uint_as_float(r[4]), p.qk_scale * __uint_as_float(r[5]));
-            u.w = pack_half2(p.qk_scale * __uint_as_float(r[6]), p.qk_scale * __uint_as_float(r[7]));
-            d4[q] = u;
-          }
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t* r = q < 4 ? ra + 8 * q : rb + 8 * (q - 4);
+          st_shared_v4(smem_u32(row + ((q ^ (lane & 7)) << 4)),
+                       pack_half2(p.qk_scale * __uint_as_float(r[0]), p.qk_scale * __uint_as_float(r[1])),
+                       pack_half2(p.qk_scale * __uint_as_float(r[2]), p.qk_scale * __uint_as_float(r[3])),
+                       pack_half2(p.qk_scale * __uint_as_float(r[4]), p.qk_scale * __uint_as_float(r[5])),
+                       pack_half2(p.qk_scale * __uint_as_float(r[6]), p.qk_scale * __uint_as_float(r[7])));
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        // rows past the sequence end are clipped by the tensor map
+        const int x = head * T.dvp + vt * kGlaTile, y = (c_begin + c) * kC + quad * 32;
+        tma_store_3d(&T.tmO, stage, x, y, b);
+        tma_store_3d(&T.tmO, stage + 4096, x + 64, y, b);
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(&bar[B_V_EMPTY]);  // the next V tile may overwrite the staging
+      }
+    }
+    if (lane == 0 && !state_pass) {
+      // the o rows are in global memory before the CTA reports them done
+      bulk_wait0();
+      fence_proxy_async_global();
     }
   } else if (warp >= 8) {
     // ---------------- state epilogue: S' <- gamma_c mid_{c+1} S', fp16 copy in smem

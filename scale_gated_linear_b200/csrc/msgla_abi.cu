@@ -556,7 +556,8 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     GlaTask& t = lp.task[j];
     if (!encode_3d(&t.tmQ, false, at(bw.qs), b.heads * h->dkp, bw.rows, B, kGlaChunk) ||
         !encode_3d(&t.tmK, false, at(bw.ks), b.heads * h->dkp, bw.rows, B, kGlaChunk) ||
-        !encode_3d(&t.tmV, false, at(bw.v), b.heads * h->dvp, bw.rows, B, kGlaChunk))
+        !encode_3d(&t.tmV, false, at(bw.v), b.heads * h->dvp, bw.rows, B, kGlaChunk) ||
+        !encode_out_3d(&t.tmO, false, at(bw.o), b.heads * h->dvp, bw.rows, B))
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (gla, scale %d)", b.scale);
     t.gamma = static_cast<const float*>(at(bw.gamma));
     t.mid = static_cast<const float*>(at(bw.mid));

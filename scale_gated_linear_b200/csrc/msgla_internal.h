@@ -103,9 +103,10 @@ struct GemmParams {
 
 // Chunkwise GLA over one or more branches.
 struct alignas(64) GlaTask {
-  CUtensorMap tmQ;  // 3D {h*dkp, n_s, B}, box {64, 64, 1}
+  CUtensorMap tmQ;  // 3D {h*dkp, n_s, B}, box {64, 128, 1}
   CUtensorMap tmK;  // same shape as tmQ
-  CUtensorMap tmV;  // 3D {h*dvp, n_s, B}, box {64, 64, 1}
+  CUtensorMap tmV;  // 3D {h*dvp, n_s, B}, box {64, 128, 1}
+  CUtensorMap tmO;  // output o: 3D {h*dvp, n_s, B}, box {64, 32, 1} (TMA store)
   const float* gamma;  // [B, n_chunks, h*dkp]: e^{b_last - m} per chunk
   const float* mid;    // [B, n_chunks, h*dkp]: e^{m}, m = b at the chunk's 64th row
   __half* o;           // [B, n_s, h*dvp]
