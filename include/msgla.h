@@ -124,6 +124,9 @@ int msgla_workspace_size(const msgla_handle* h, int B, int L, size_t* bytes);
  * after the gates, joined back before the final output projection), so all of
  * the forward's work is still ordered before what follows it on `stream`; the
  * fork and join use events, so the forward can be captured into a CUDA graph.
+ * The environment variable MSGLA_SERIAL=1 (read once per process) keeps every
+ * kernel on `stream`: needed under profilers that run kernels one at a time,
+ * where the concurrent GEMM's bounded wait for the GLA CTAs would time out.
  * The handle keeps per-forward counters: forwards on one handle must not run
  * concurrently (serialise calls from several host threads or streams). */
 int msgla_forward(msgla_handle* h, const void* X, int B, int L, void* O,

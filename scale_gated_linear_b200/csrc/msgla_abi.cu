@@ -14,6 +14,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -411,9 +412,16 @@ struct Recorder {
 // GLA CTA is resident (launch_wait_started) and takes its tiles dynamically, so
 // it runs on the SMs the GLA leaves free and on those its coarse-branch CTAs
 // release, and it can never keep a GLA CTA from starting.
+// MSGLA_SERIAL=1 in the environment keeps every kernel on the caller's stream
+// (for profilers that run kernels one at a time, under which the GEMM's wait
+// for the resident GLA CTAs could only time out).
 bool coarse_overlap(const msgla_handle* h, const Workspace& ws, int B, long long* gla_ctas) {
+  static const bool serial = [] {
+    const char* e = getenv("MSGLA_SERIAL");
+    return e && *e && *e != '0';
+  }();
   *gla_ctas = 0;
-  if (h->main_index < 0 || h->n_scales < 2 || h->cfg.head_norm) return false;
+  if (serial || h->main_index < 0 || h->n_scales < 2 || h->cfg.head_norm) return false;
   long long ctas = 0;
   for (int j = 0; j < h->n_scales; ++j) {
     if (ws.br[j].n_segs > 1) return false;

@@ -264,6 +264,49 @@ def test_forward_profiled_records_every_launch():
     layer.close()
 
 
+_SERIAL_CHILD = """
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+sys.path.insert(0, sys.argv[1] + "/tests")
+from helpers import gpu_inputs
+from scale_gated_linear_b200 import MSGLA
+from scale_gated_linear_b200 import workloads as wl
+w = wl.WORKLOADS["tiny"].replace(name="small", B=2, L=200, d=128, d_k=64, d_v=128, chunk=64)
+inp = gpu_inputs(w, L=100)
+layer = MSGLA.from_workload(w, inp, device=0)
+X = inp["X"].cuda()
+O = layer.forward(X, workspace=layer.alloc_workspace(*X.shape[:2]))
+torch.cuda.synchronize()
+layer.check_status()
+np.save(sys.argv[2], O.float().cpu().numpy())
+print(",".join(layer.launch_names(*X.shape[:2])))
+layer.close()
+"""
+
+
+@needs_gpu
+def test_serial_switch_runs_one_stream_with_identical_output(tmp_path):
+    """MSGLA_SERIAL=1 (read once per process, so in a child process) puts the
+    coarse output projection back on the caller's stream; the output is
+    bit-identical to the two-stream forward."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = tmp_path / "serial.npy"
+    env = dict(os.environ, MSGLA_SERIAL="1")
+    r = subprocess.run([sys.executable, "-c", _SERIAL_CHILD, root, str(out)], env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    names = r.stdout.strip().splitlines()[-1].split(",")
+    assert names == ["pool_fuse", "proj_gemm", "gate", "gla", "out_gemm_coarse", "out_gemm_fused"]
+    inp = gpu_inputs(SMALL, L=100)
+    got, layer, _ = run_gpu(SMALL, inp)
+    assert layer.launch_names(2, 100) == ["pool_fuse", "proj_gemm", "gate", "gla", "out_gemm_fused"]
+    layer.close()
+    np.testing.assert_array_equal(np.load(out), got)
+
+
 # ----------------------------------------------------------------- full sizes
 @needs_gpu
 def test_340m_layer_full_size_sampled_rows():
