@@ -142,7 +142,47 @@ struct Held {
   const uint8_t* smem[2];  // box 0 of each coarse branch
   int box_bytes[2];
   int lrow[2];             // this thread's held row within the boxes
+  // box j (64 columns of every coarse branch) has its own barriers: full[j]
+  // (the loader's TMA bytes landed, phase `parity` for this tile) and empty[j]
+  // (one arrival per epilogue warp that has read it: four per box)
+  uint64_t* full;
+  uint64_t* empty;
+  uint32_t parity;
+  volatile int* abort_flag;
 };
+
+// Fusion weights w = softmax(z_t + b_fuse) of this thread's output row
+// (Eq. (10), logits from the projection GEMM); the n0 == 0 tiles also store
+// them. Computed before the accumulator is ready: the logit loads' latency
+// hides behind the tile's MMAs.
+struct FuseW {
+  float wts[kMaxScales];
+  float wmain;
+};
+__device__ __forceinline__ void fuse_weights(const GemmParams& p, const TileCoord& tc, int quad, int lane, int c_lo,
+                                             FuseW& fw) {
+  const GemmTask& T = p.task[tc.task];
+  fw.wmain = 0.f;
+  if (T.epi != kEpiFuse) return;
+  const int row = tc.m0 + quad * 32 + lane;
+  if (row >= T.rows) return;
+  const size_t grow = static_cast<size_t>(tc.b) * T.rows + row;
+  float zmax = -INFINITY;
+  for (int j = 0; j < T.n_scales; ++j) {
+    fw.wts[j] = __ldg(T.zf + grow * T.ldz + j) + __ldg(T.bfuse + j);
+    zmax = fmaxf(zmax, fw.wts[j]);
+  }
+  float sum = 0.f;
+  for (int j = 0; j < T.n_scales; ++j) {
+    fw.wts[j] = __expf(fw.wts[j] - zmax);
+    sum += fw.wts[j];
+  }
+  const float inv = 1.f / sum;
+  for (int j = 0; j < T.n_scales; ++j) fw.wts[j] *= inv;
+  if (tc.n0 == 0 && c_lo == 0)
+    for (int j = 0; j < T.n_scales; ++j) T.w[grow * T.n_scales + j] = fw.wts[j];
+  fw.wmain = fw.wts[T.main_index];
+}
 
 __device__ __forceinline__ void pack_f16x32(uint32_t (&pk)[16], const uint32_t (&v)[32]) {
 #pragma unroll
@@ -161,39 +201,22 @@ __device__ __forceinline__ void pack_bf16x32(uint32_t (&pk)[16], const float (&a
 // fused epilogue instead prefetches the held coarse rows one chunk ahead (both
 // at once would not fit the register budget). `sel` is the warp's running
 // staging-buffer index.
-__device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
+// Returns false if a bounded wait for held rows gave up (the error word is set).
+__device__ __forceinline__ bool epilogue_tile(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
                                               int lane, int c_lo, int c_hi, bool padded, const Stager& stg,
-                                              int& sel, const Held* held = nullptr) {
+                                              int& sel, const FuseW& fw, const Held* held = nullptr) {
   const GemmTask& T = p.task[tc.task];
   const int row = tc.m0 + quad * 32 + lane;
   const int row0 = tc.m0 + quad * 32;
   const bool valid = row < T.rows;
   const size_t grow = static_cast<size_t>(tc.b) * T.rows + row;
-  float wts[kMaxScales];
-  float wmain = 0.f;
+  const float* wts = fw.wts;
+  const float wmain = fw.wmain;
   const bool prefetch = T.epi == kEpiFuse && T.n_coarse <= 2 && !held;
   const uint4* base0 = nullptr;
   const uint4* base1 = nullptr;
   float wc0 = 0.f, wc1 = 0.f;
   if (T.epi == kEpiFuse) {
-    if (valid) {
-      // w = softmax(W_fuse x + b_fuse) from the logits of the projection GEMM (Eq. (10))
-      float zmax = -INFINITY;
-      for (int j = 0; j < T.n_scales; ++j) {
-        wts[j] = __ldg(T.zf + grow * T.ldz + j) + __ldg(T.bfuse + j);
-        zmax = fmaxf(zmax, wts[j]);
-      }
-      float sum = 0.f;
-      for (int j = 0; j < T.n_scales; ++j) {
-        wts[j] = __expf(wts[j] - zmax);
-        sum += wts[j];
-      }
-      const float inv = 1.f / sum;
-      for (int j = 0; j < T.n_scales; ++j) wts[j] *= inv;
-      if (tc.n0 == 0 && c_lo == 0)
-        for (int j = 0; j < T.n_scales; ++j) T.w[grow * T.n_scales + j] = wts[j];
-      wmain = wts[T.main_index];
-    }
     if (prefetch && valid) {
       auto held = [&](int c, const uint4*& base, float& wc) {
         if (c >= T.n_coarse) return;
@@ -322,7 +345,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
     stg.put(sel, half, pk);
     if (half == 1) stg.store(sel, map, dcol, row0, tc.b);
   };
-  if (c_lo >= c_hi) return;
+  if (c_lo >= c_hi) return true;
   uint32_t va[32], vb[32];
   if (prefetch) {
     load(cur0, cur1, c_lo);
@@ -333,12 +356,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
       chunk(c0, va, half, c0 + 32 >= c_hi);
       if (half) sel ^= 1;
     }
-    return;
+    return true;
   }
   tmem_ld32(tmem_addr(tacc, quad * 32, c_lo), va);
   tmem_wait_ld(va);
   for (int c0 = c_lo; c0 < c_hi; c0 += 64) {
     const bool has_b = c0 + 32 < c_hi, has_next = c0 + 64 < c_hi;
+    // held rows: this 64-column box has landed
+    if (held && !mbar_wait(&held->full[c0 >> 6], held->parity, held->abort_flag, p.err)) return false;
     if (has_b) tmem_ld32(tmem_addr(tacc, quad * 32, c0 + 32), vb);
     chunk(c0, va, 0, !has_b);
     if (has_b) {
@@ -347,8 +372,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const TileCoo
       chunk(c0 + 32, vb, 1, !has_next);
       if (has_next) tmem_wait_ld(va);
     }
+    if (held) {
+      // this warp is done with the box: the loader may refill it for the next tile
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&held->empty[c0 >> 6]);
+    }
     sel ^= 1;
   }
+  return true;
 }
 
 // Two epilogue warps share each TMEM lane quadrant and split the tile's columns
@@ -481,11 +513,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       const TileCoord tc = decode_tile(p, tile, BN);
       const uint32_t buf = it & 1;
       const bool padded = row_is_padded(p, tc, quad, lane);
-      if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.err)) break;
-      tc_fence_after();
       int lo, hi;
       epi_columns(warp, tc.n_eff, lo, hi);
-      epilogue_tile(p, tc, tmem + buf * BN, quad, lane, lo, hi, padded, stg, sel);
+      FuseW fw;
+      fuse_weights(p, tc, quad, lane, lo, fw);
+      if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.err)) break;
+      tc_fence_after();
+      epilogue_tile(p, tc, tmem + buf * BN, quad, lane, lo, hi, padded, stg, sel, fw);
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
     }
@@ -545,16 +579,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
     gemm_pair_kernel(const __grid_constant__ GemmParams p) {
   using Lay = PairLayout<kHeld>;
   constexpr int kStagesT = Lay::kStages;
-  static_assert((2 * kStagesT + 4 + 2 + 2 * kTileRing) * 8 + 4 * kTileRing + 8 <= 256, "barrier region");
+  constexpr int kHeldBars = kHeld ? 4 : 1;
+  static_assert((2 * kStagesT + 4 + 2 * kHeldBars + 2 * kTileRing) * 8 + 4 * kTileRing + 8 <= 256, "barrier region");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Lay::kBarOffset);
   uint64_t* empty_bar = full_bar + kStagesT;
   uint64_t* acc_full = empty_bar + kStagesT;  // [2]
   uint64_t* acc_empty = acc_full + 2;         // [2] (used in the leader)
-  uint64_t* held_full = acc_empty + 2;        // kHeld: this CTA's held rows landed
-  uint64_t* held_empty = held_full + 1;       // kHeld: this CTA's epilogue is done with them
-  uint64_t* tile_full = held_empty + 1;       // [kTileRing] dynamic tiles
+  uint64_t* held_full = acc_empty + 2;        // kHeld [4]: box j of this CTA's held rows landed
+  uint64_t* held_empty = held_full + kHeldBars;  // kHeld [4]: the epilogue warps are done with box j
+  uint64_t* tile_full = held_empty + kHeldBars;  // [kTileRing] dynamic tiles
   uint64_t* tile_empty = tile_full + kTileRing;  // [kTileRing] (used in the leader)
   volatile int* tile_slot = reinterpret_cast<volatile int*>(tile_empty + kTileRing);  // [kTileRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(tile_slot) + kTileRing);
@@ -574,8 +609,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 2 * kEpiThreads);
     }
-    mbar_init(held_full, 1);
-    mbar_init(held_empty, kEpiThreads);
+    for (int j = 0; j < kHeldBars; ++j) {
+      mbar_init(&held_full[j], 1);
+      mbar_init(&held_empty[j], 4);  // the four epilogue warps of the box's column half
+    }
     for (int r = 0; r < kTileRing; ++r) {
       mbar_init(&tile_full[r], 1);
       mbar_init(&tile_empty[r], kTileConsumers);
@@ -699,18 +736,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
       const GemmTask& T = p.task[0];
       for (int c = 0; c < 2 && c < T.n_coarse; ++c) prefetch_tmap(&T.tmOut[1 + c]);
       uint32_t it = 0;
-      for (int tile = pair; tile < ntiles; tile += npairs, ++it) {
+      uint32_t bytes = 0;
+      for (int c = 0; c < 2 && c < T.n_coarse; ++c) bytes += held_box[c];
+      bool ok = true;
+      for (int tile = pair; ok && tile < ntiles; tile += npairs, ++it) {
         const TileCoord tc = decode_tile(p, tile, kPairBN, kPairBM);
         const int m0 = tc.m0 + 128 * static_cast<int>(rank);
-        if (it >= 1 && !mbar_wait(held_empty, (it - 1) & 1, abort_flag, p.err)) break;
-        uint32_t bytes = 0;
-        for (int c = 0; c < 2 && c < T.n_coarse; ++c) bytes += 4 * held_box[c];
-        mbar_arrive_expect_tx(held_full, bytes);
-        for (int c = 0; c < 2 && c < T.n_coarse; ++c) {
-          const int base = held_base(m0, T.coarse_scale[c]);
-          for (int j = 0; j < 4; ++j)
-            tma_load_3d(&T.tmOut[1 + c], held_full, held_smem + held_off[c] + j * held_box[c], tc.n0 + 64 * j, base,
-                        tc.b);
+        // boxes in the order the epilogue releases them (the first 64 columns of
+        // each column half first); each is refilled once its four warps are done
+        for (int q = 0; q < 4; ++q) {
+          const int j = (q >> 1) | ((q & 1) << 1);  // 0, 2, 1, 3
+          if (it >= 1 && !mbar_wait(&held_empty[j], (it - 1) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&held_full[j], bytes);
+          for (int c = 0; c < 2 && c < T.n_coarse; ++c)
+            tma_load_3d(&T.tmOut[1 + c], &held_full[j], held_smem + held_off[c] + j * held_box[c], tc.n0 + 64 * j,
+                        held_base(m0, T.coarse_scale[c]), tc.b);
         }
       }
     }
@@ -730,12 +773,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
       tc.m0 += 128 * static_cast<int>(rank);
       const uint32_t buf = it & 1;
       const bool padded = row_is_padded(p, tc, quad, lane);
-      if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.err)) break;
-      tc_fence_after();
       int lo, hi;
       epi_columns(warp, tc.n_eff, lo, hi);
+      FuseW fw;
+      fuse_weights(p, tc, quad, lane, lo, fw);
+      if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.err)) break;
+      tc_fence_after();
       if (kHeld) {
-        if (!mbar_wait(held_full, it & 1, abort_flag, p.err)) break;
         const GemmTask& T = p.task[tc.task];
         const int t = tc.m0 + quad * 32 + lane;
         Held h;
@@ -748,11 +792,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
             h.lrow[c] = (t + 1) / s - 1 - held_base(tc.m0, s);
           }
         }
-        epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel, &h);
-        fence_proxy_async_smem();
-        mbar_arrive(held_empty);
+        h.full = held_full;
+        h.empty = held_empty;
+        h.parity = it & 1;
+        h.abort_flag = abort_flag;
+        if (!epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel, fw, &h)) break;
       } else {
-        epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel);
+        epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel, fw);
       }
       tc_fence_before();
       mbar_arrive_cluster(buf ? lead_empty1 : lead_empty0);
@@ -811,8 +857,11 @@ cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pa
   if (p.total_tiles <= 0) return cudaSuccess;
   // the fused output launch with one or two coarse branches stages their held
   // rows in shared memory (the caller encodes tmOut[1 + c] for them)
+  // (and only with full 256-column tiles: every 64-column box of held rows then
+  // has the four epilogue warps that release it)
   const bool held = p.n_tasks == 1 && p.task[0].epi == kEpiFuse && p.task[0].n_coarse >= 1 &&
-                    p.task[0].n_coarse <= 2 && held_rows_fit(p.task[0].coarse_scale, p.task[0].n_coarse);
+                    p.task[0].n_coarse <= 2 && p.task[0].N % kPairBN == 0 &&
+                    held_rows_fit(p.task[0].coarse_scale, p.task[0].n_coarse);
   int pairs = (bn != 256) ? 0 : held ? max_active_pairs<true>() : max_active_pairs<false>();
   if (max_pairs > 0 && pairs > max_pairs) pairs = max_pairs;
   if (pairs > 0) {
