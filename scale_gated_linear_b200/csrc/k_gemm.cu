@@ -554,10 +554,10 @@ constexpr int kHeldBytes = 60 * 1024;
 
 template <bool kHeld>
 struct PairLayout {
-  static constexpr int kStages = kHeld ? 4 : 5;
+  static constexpr int kStages = kHeld ? 4 : 6;
   static constexpr int kThreadsT = kHeld ? 352 : 320;  // + warp 10: held-row loader
   static constexpr int kStagingOffset = kStages * kPairStageBytes;
-  static constexpr int kStagingBytesT = kHeld ? 8 * kStagerBytes : kStagingBytes;
+  static constexpr int kStagingBytesT = 8 * kStagerBytes;
   static constexpr int kHeldOffset = kStagingOffset + kStagingBytesT;
   static constexpr int kBarOffset = kHeldOffset + (kHeld ? kHeldBytes : 0);
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
@@ -762,7 +762,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
     const int quad = warp & 3;
     const uint32_t lead_empty0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     const uint32_t lead_empty1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
-    const Stager stg{smem + Lay::kStagingOffset + (warp - 2) * (kHeld ? 1 : 2) * kStagerBytes, lane, !kHeld};
+    const Stager stg{smem + Lay::kStagingOffset + (warp - 2) * kStagerBytes, lane, false};
     int sel = 0;
     if (lane == 0) prefetch_out_maps(p);
     for (uint32_t it = 0;; ++it) {
