@@ -17,7 +17,9 @@ norm of the GLA output.
 
 Prints one JSON line on rank 0. Timing: W untimed warm-up steps, then K timed
 steps, each bracketed by CUDA events on the launching stream with a 256 MiB
-write between steps to flush the 126 MB L2. The kernels of a forward are
+write between steps to flush the 126 MB L2, followed by a 256 MiB read so that
+the step does not pay for writing back the flush's own dirty lines. The kernels
+of a forward are
 launched so that each may start while the previous one finishes, and an event
 between two kernels takes that overlap away, so the timed steps record events
 only at the step boundaries and around the dominant kernel (for the roofline);
@@ -433,8 +435,12 @@ def run_ours(args) -> int:
         M = None if mask_kind == "none" else wl.make_mask(wk.B, wk.L, mask_kind, seed=wk.seed + rank).to(dev)
         O = torch.empty_like(X)
         ws = layer.alloc_workspace(wk.B, wk.L)
+        # L2 flush between steps: a 256 MiB write, then a 256 MiB read that evicts the
+        # write's dirty lines, so every timed step starts from a cold L2 that holds
+        # neither its inputs nor write-backs owed by the flush itself
         flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-        flush = lambda: flush_buf.fill_(1)
+        flush_rd = torch.ones(256 * 1024 * 1024 // 8, dtype=torch.int64, device=dev)
+        flush = lambda: (flush_buf.fill_(1), flush_rd.sum())
         names = layer.launch_names(wk.B, wk.L)
         n_ev = len(names) + 1
         stream = torch.cuda.current_stream()
@@ -490,7 +496,7 @@ def run_ours(args) -> int:
             res["io_bytes"] = Xh.numel() * 2
             del wsh
         layer.close()
-        del ws, flush_buf
+        del ws, flush_buf, flush_rd
         torch.cuda.empty_cache()
         return res
 
@@ -525,7 +531,7 @@ def run_ours(args) -> int:
                                + (f", {args.mask}-padding mask" if args.mask != "none" else "")
                                + (", head RMS norm" if w.head_norm else ""),
                    "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"sequence-sharded x{world}",
-                   "l2": "flushed between timed steps (256 MiB write)"},
+                   "l2": "flushed between timed steps (256 MiB write, then a 256 MiB read: cold and clean)"},
         "roofline": roof,
         "path_roofline": {"bound": "tensor", "achieved": path_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                           "frac": path_tf / peaks["bf16_tflops"], "flops_per_step": counts["total_flops"]},

@@ -13,6 +13,8 @@
 //   hold_fuse_kernel  O_t = sum_s w_{t,s} Y^(s)_{floor((t+1)/s)-1} (Sec. 3.3,
 //                     Eq. (11)) when no branch has scale 1.
 //   weight converters used once by msgla_create.
+#include <algorithm>
+
 #include "msgla_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -343,6 +345,71 @@ __global__ void __launch_bounds__(256) pool_rows_kernel(const PoolParams p) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) m[e] += x[r][e];
       put(j, s, i0, m, 1.f / static_cast<float>(max(1, __popc((vm >> i0) & ((1u << cnt) - 1u)))));
+    }
+  }
+  if (bad) atomicCAS(p.err, 0, kDevRange);
+}
+
+// Pooling only, with no mask, coarse scales that are powers of two dividing P,
+// and every sequence a whole number of P-row blocks: blocks are numbered flat
+// over the batch (block f starts at token f P, and its pooled row for scale s is
+// (f P + i0) / s), so the loop does no integer division. Thread (r, cg) of a CTA
+// of R x (d / 8) threads takes 8 columns of blocks f = R blockIdx.x + r, then
+// f + R gridDim.x, ..., U blocks' loads in flight per step.
+template <int P, int U>
+__global__ void __launch_bounds__(256) pool_rows_flat_kernel(const PoolParams p, int n_blocks, int R) {
+  griddep_wait();
+  griddep_launch();
+  const int groups = p.d >> 3;
+  const int cg = static_cast<int>(threadIdx.x) % groups, r = static_cast<int>(threadIdx.x) / groups;
+  if (r >= R) return;
+  const uint4* X4 = reinterpret_cast<const uint4*>(p.X) + cg;
+  const int fstep = R * static_cast<int>(gridDim.x);
+  bool bad = false;
+  for (int f0 = R * static_cast<int>(blockIdx.x) + r; f0 < n_blocks; f0 += U * fstep) {
+    uint4 raw[U][P];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int f = f0 + u * fstep;
+      if (f < n_blocks)
+#pragma unroll
+        for (int q = 0; q < P; ++q) raw[u][q] = __ldg(X4 + (static_cast<size_t>(f) * P + q) * groups);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int f = f0 + u * fstep;
+      if (f >= n_blocks) break;
+      float lv[P][8];
+#pragma unroll
+      for (int q = 0; q < P; ++q) bf16x8_to_f32(raw[u][q], lv[q]);
+#pragma unroll
+      for (int level = 0; (1 << level) < P; ++level) {
+        // lv[i] holds the sum of rows [i*width, (i+1)*width)
+        const int n = P >> level;
+        const int width = 2 << level;
+#pragma unroll
+        for (int i = 0; i < P / 2; ++i)
+          if (i < n / 2)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) lv[i][e] = lv[2 * i][e] + lv[2 * i + 1][e];
+        for (int j = 0; j < p.n_scales; ++j) {
+          if (p.scales[j] != width) continue;
+          const float inv = 1.f / static_cast<float>(width);  // exact: width is a power of two
+#pragma unroll
+          for (int i = 0; i < P / 2; ++i) {
+            if (i >= n / 2) break;
+            uint4 o;
+            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float a0 = lv[i][2 * e] * inv, a1 = lv[i][2 * e + 1] * inv;
+              bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
+              ow[e] = pack_half2(a0, a1);
+            }
+            reinterpret_cast<uint4*>(p.Xp[j] + (static_cast<size_t>(f) * (P / width) + i) * p.d)[cg] = o;
+          }
+        }
+      }
     }
   }
   if (bad) atomicCAS(p.err, 0, kDevRange);
@@ -742,6 +809,18 @@ cudaError_t launch_pool_rows(const PoolParams& p, cudaStream_t st) {
                     st, p);
 }
 
+template <int P, int U>
+cudaError_t launch_pool_flat(const PoolParams& p, cudaStream_t st) {
+  const int groups = p.d / 8;
+  const int R = 256 / groups;
+  const long long n_blocks = static_cast<long long>(p.B) * p.L / P;
+  const long long ctas = (n_blocks + static_cast<long long>(R) * U - 1) / (static_cast<long long>(R) * U);
+  const long long resident = (P == 8 ? 2LL : 3LL) * sm_count();  // CTAs of 256 threads per SM at its registers
+  const int grid = static_cast<int>(std::min<long long>(ctas, resident));
+  return launch_pdl(pool_rows_flat_kernel<P, U>, dim3(grid), dim3(R * groups), 0, st, p, static_cast<int>(n_blocks),
+                    R);
+}
+
 template <int P>
 cudaError_t launch_pool_only(const PoolParams& p, cudaStream_t st) {
   const size_t n = static_cast<size_t>(p.B) * ((p.L + P - 1) / P) * (p.d / 8);
@@ -754,6 +833,11 @@ cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st) {
   // the row-block kernels take P rows at a time, so every scale must divide P
   const int lcm = p.block_rows;
   if (!p.want_w) {
+    // flat kernel: no mask, power-of-two coarse scales, whole blocks, d <= 2048
+    const bool flat = !p.M && p.d <= 2048 && static_cast<long long>(p.B) * p.L < (1LL << 30);
+    if (flat && lcm <= 2 && p.L % 2 == 0) return launch_pool_flat<2, 4>(p, st);
+    if (flat && lcm == 4 && p.L % 4 == 0) return launch_pool_flat<4, 2>(p, st);
+    if (flat && lcm == 8 && p.L % 8 == 0) return launch_pool_flat<8, 1>(p, st);
     if (2 % lcm == 0) return launch_pool_only<2>(p, st);
     if (4 % lcm == 0) return launch_pool_only<4>(p, st);
     if (6 % lcm == 0) return launch_pool_only<6>(p, st);

@@ -140,6 +140,8 @@ cudaError_t launch_wait_started(const unsigned long long* started, unsigned long
 // (each returns the cudaError_t of the launch)
 // max_pairs > 0 caps the number of CTA pairs of the persistent grid.
 cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pairs = 0);
+// streaming multiprocessors of the current device
+int sm_count();
 cudaError_t launch_gla(const GlaParams& p, cudaStream_t st);
 // initial state of every segment from the state pass's end states (sequential over segments)
 cudaError_t launch_gla_scan(const GlaParams& p, int B, cudaStream_t st);
