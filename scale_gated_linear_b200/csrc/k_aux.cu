@@ -483,9 +483,18 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Nonzero if either half of a packed fp16 pair is inf or nan (exponent all ones).
-__device__ __forceinline__ uint32_t half2_nonfinite(uint32_t h) {
-  return ((h & 0x7c00u) == 0x7c00u) | ((h & 0x7c000000u) == 0x7c000000u);
+// log2(x) by the hardware approximation (absolute error about 2^-22 for x in (1, 2])
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Accumulates a packed fp16 pair's exponents into `acc` so that bit 15 or bit 31
+// of acc ends up set iff some half seen was inf or nan (exponent all ones: adding
+// one to the exponent field then carries into that half's sign position).
+__device__ __forceinline__ void half2_track_nonfinite(uint32_t& acc, uint32_t h) {
+  acc |= (h & 0x7c007c00u) + 0x04000400u;
 }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -635,23 +644,38 @@ __global__ void __launch_bounds__(kGateThreads, 3) gate_kernel(const __grid_cons
       }
     }
     // log alpha (base 2) into the blocked layout; D fragment: d0 = (gq, 2tq),
-    // d1 = (gq, 2tq+1), d2 = (gq+8, 2tq), d3 = (gq+8, 2tq+1)
-    const float scale = p.inv_normalizer * 1.4426950408889634f;  // 1/normalizer * log2(e)
+    // d1 = (gq, 2tq+1), d2 = (gq+8, 2tq), d3 = (gq+8, 2tq+1). With z2 = z log2(e),
+    // log2 alpha = (min(z2, 0) - log2(1 + 2^{-|z2|})) / normalizer, the base-2
+    // form of logsigmoid(z) / normalizer (the log argument lies in (1, 2]).
+    constexpr float kLog2e = 1.4426950408889634f;
+    const float inv_norm = p.inv_normalizer;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const int chl = warp * 16 + nt * 8 + 2 * tq;
-      const float bias0 = __ldg(P.bg + cbase + chl), bias1 = __ldg(P.bg + cbase + chl + 1);
+      const float bias0 = __ldg(P.bg + cbase + chl) * kLog2e, bias1 = __ldg(P.bg + cbase + chl + 1) * kLog2e;
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int row = mt * 16 + gq + ((e & 2) ? 8 : 0), ch = chl + (e & 1);
-          const float z = acc[mt][nt][e] + ((e & 1) ? bias1 : bias0);
-          // logsigmoid(z) = min(z, 0) - log(1 + e^{-|z|}); the log argument lies in (1, 2]
-          const float la = (fminf(z, 0.f) - __logf(1.f + __expf(-fabsf(z)))) * scale;
-          la_s[((ch >> 3) * (kChunk / 4) + (row >> 2)) * kGateBlk + (row & 3) * 8 + (ch & 7)] =
-              row < nrows ? la : 0.f;
+          const float z2 = fmaf(acc[mt][nt][e], kLog2e, (e & 1) ? bias1 : bias0);
+          const float la = (fminf(z2, 0.f) - lg2_approx(1.f + ex2_approx(-fabsf(z2)))) * inv_norm;
+          la_s[((ch >> 3) * (kChunk / 4) + (row >> 2)) * kGateBlk + (row & 3) * 8 + (ch & 7)] = la;
         }
+      }
+    }
+    if (nrows < kChunk) {
+      // rows past the end of the sequence contribute nothing to the sums
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int chl = warp * 16 + nt * 8 + 2 * tq;
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int row = mt * 16 + gq + ((e & 2) ? 8 : 0), ch = chl + (e & 1);
+            if (row >= nrows) la_s[((ch >> 3) * (kChunk / 4) + (row >> 2)) * kGateBlk + (row & 3) * 8 + (ch & 7)] = 0.f;
+          }
       }
     }
   }
@@ -695,7 +719,11 @@ __global__ void __launch_bounds__(kGateThreads, 3) gate_kernel(const __grid_cons
 #pragma unroll
   for (int e = 0; e < 8; ++e) pre[e] -= second ? 0.f : tot[e];
 
-  uint32_t over = 0;  // a scaled value left the fp16 range
+  // A scaled value can leave the fp16 range only where its factor exceeds 1: b
+  // does not increase along the chunk (log alpha <= 0), so in the first half
+  // (rows up to m's) Qs = q 2^{b-m} can grow and Ks cannot, and in the second
+  // half the reverse. Only the growing side is checked.
+  uint32_t over = 0;
   const int sw = rg & 7;  // (row >> 2) & 7 for all four rows of this thread
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
@@ -714,13 +742,13 @@ __global__ void __launch_bounds__(kGateThreads, 3) gate_kernel(const __grid_cons
       const float2 qf = __half22float2(qh[e]), kf = __half22float2(kh[e]);
       qw[e] = pack_half2(qf.x * ex2_approx(b0), qf.y * ex2_approx(b1));
       kw[e] = pack_half2(kf.x * ex2_approx(-b0), kf.y * ex2_approx(-b1));
-      over |= half2_nonfinite(qw[e]) | half2_nonfinite(kw[e]);
+      half2_track_nonfinite(over, second ? kw[e] : qw[e]);
     }
     const size_t go = (row_base + row) * ldk + cbase + cg * 8;
     *reinterpret_cast<uint4*>(P.qs + go) = qo;
     *reinterpret_cast<uint4*>(P.ks + go) = ko;
   }
-  if (over) atomicCAS(p.err, 0, kDevRange);
+  if (over & 0x80008000u) atomicCAS(p.err, 0, kDevRange);
   if (rg == 15) {
     const size_t gi = (static_cast<size_t>(b) * n_chunks + ci) * ldk + cbase + cg * 8;
     float* dst = second ? P.gamma : P.mid;

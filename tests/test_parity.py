@@ -246,6 +246,24 @@ def test_fp16_range_overflow_is_reported():
 
 
 @needs_gpu
+def test_gate_range_overflow_is_reported():
+    """A gate bias far below zero (log alpha near -200/16 per pooled step) makes
+    the decay-scaled queries and keys of the gate kernel leave the fp16 range on
+    both halves of a chunk: the kernel latches MSGLA_ERR_RANGE and the handle
+    stays usable."""
+    inp = gpu_inputs(SMALL, L=200)
+    strong = {k: v for k, v in inp.items()}
+    strong["branches"] = [dict(br) for br in inp["branches"]]
+    for br in strong["branches"]:
+        br["bg"] = torch.full_like(br["bg"], -200.0)
+    layer = _layer(SMALL, strong)
+    layer(inp["X"].cuda())
+    assert layer.sync_status() == -5
+    assert layer.sync_status() == 0
+    layer.close()
+
+
+@needs_gpu
 def test_forward_profiled_records_every_launch():
     inp = gpu_inputs(SMALL, L=100)
     layer = _layer(SMALL, inp)
