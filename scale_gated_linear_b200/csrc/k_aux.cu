@@ -149,8 +149,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_fuse_kernel(const PoolParam
 // in flight per lane), then forms the pooled rows of every coarse scale and the
 // partial fusion logits; the logits are reduced across the warp once per row at
 // the end. NS bounds the number of scales held in registers.
-template <int P, int GPL, int NS>
-__global__ void __launch_bounds__(256) pool_fuse_rows_kernel(const PoolParams p) {
+template <int P, int GPL, int NS, int MB>
+__global__ void __launch_bounds__(256, MB) pool_fuse_rows_kernel(const PoolParams p) {
   griddep_wait();
   griddep_launch();
   extern __shared__ float wf_s[];  // [n_scales][d] fp32
@@ -768,38 +768,46 @@ cudaError_t launch_gate_t(const GateParams& p, cudaStream_t st) {
   return launch_pdl(gate_kernel<RP>, dim3(p.total_blocks), dim3(kGateThreads), smem, st, p);
 }
 
-// one thread per 8 output columns of one row; flat grid over B*L*(d/8)
-__global__ void hold_fuse_kernel(const HoldFuseParams p) {
+// O_t = sum_s w_{t,s} Y^(s)_{floor((t+1)/s)-1} (Eq. (11) with the causal hold of
+// Sec. 3.3) when no branch has scale 1. One CTA per (sequence, tile of
+// kHoldRows rows, block of up to 256 column groups): thread (r, cg) takes 8
+// columns of rows t0 + r, t0 + r + R, ...; no division in the loop (the held
+// row index is a shift for power-of-two scales).
+constexpr int kHoldRows = 32;
+__global__ void __launch_bounds__(256) hold_fuse_kernel(const HoldFuseParams p, int CG, int R) {
   griddep_wait();
   griddep_launch();
-  const int groups = p.d / 8;
-  const size_t gid = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
-  if (gid >= static_cast<size_t>(p.B) * p.L * groups) return;
-  const int cg = static_cast<int>(gid % groups);
-  const size_t bt = gid / groups;
-  const int t = static_cast<int>(bt % p.L), b = static_cast<int>(bt / p.L);
-  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  const float* w = p.w + bt * p.n_scales;
-  for (int j = 0; j < p.n_scales; ++j) {
-    const int s = p.scales[j];
-    const int i = (t + 1) / s - 1;
-    if (i < 0) continue;
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p.Y[j] + (static_cast<size_t>(b) * p.rows[j] + i) * p.d) + cg);
-    const __half2* h = reinterpret_cast<const __half2*>(&u);
-    const float wj = w[j];
+  const int groups = p.d >> 3;
+  const int cgl = static_cast<int>(threadIdx.x) % CG, r = static_cast<int>(threadIdx.x) / CG;
+  const int cg = static_cast<int>(blockIdx.z) * CG + cgl;
+  if (r >= R || cg >= groups) return;
+  const int b = blockIdx.y;
+  const int t0 = blockIdx.x * kHoldRows, t1 = min(p.L, t0 + kHoldRows);
+  uint4* ob = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.L * p.d) + cg;
+  const float* wb = p.w + static_cast<size_t>(b) * p.L * p.n_scales;
+#pragma unroll 2
+  for (int t = t0 + r; t < t1; t += R) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float2 f = __half22float2(h[e]);
-      acc[2 * e] = fmaf(wj, f.x, acc[2 * e]);
-      acc[2 * e + 1] = fmaf(wj, f.y, acc[2 * e + 1]);
+    for (int j = 0; j < kMaxScales; ++j) {
+      if (j >= p.n_scales) break;
+      const int i = (p.shift[j] >= 0 ? ((t + 1) >> p.shift[j]) : (t + 1) / p.scales[j]) - 1;
+      if (i < 0) continue;
+      const uint4 u =
+          __ldg(reinterpret_cast<const uint4*>(p.Y[j] + (static_cast<size_t>(b) * p.rows[j] + i) * p.d) + cg);
+      const __half2* h = reinterpret_cast<const __half2*>(&u);
+      const float wj = __ldg(wb + static_cast<size_t>(t) * p.n_scales + j);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        acc[2 * e] = fmaf(wj, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(wj, f.y, acc[2 * e + 1]);
+      }
     }
+    ob[static_cast<size_t>(t) * groups] =
+        make_uint4(pack_bf162(acc[0], acc[1]), pack_bf162(acc[2], acc[3]), pack_bf162(acc[4], acc[5]),
+                   pack_bf162(acc[6], acc[7]));
   }
-  uint4 o;
-  o.x = pack_bf162(acc[0], acc[1]);
-  o.y = pack_bf162(acc[2], acc[3]);
-  o.z = pack_bf162(acc[4], acc[5]);
-  o.w = pack_bf162(acc[6], acc[7]);
-  reinterpret_cast<uint4*>(p.out + bt * p.d)[cg] = o;
 }
 
 __global__ void bf16_to_f16_rows_kernel(const __nv_bfloat16* src, int src_ld, int rows, int cols, __half* dst,
@@ -826,15 +834,17 @@ __global__ void bf16_copy_rows_kernel(const __nv_bfloat16* src, int src_ld, int 
 
 }  // namespace
 
+// MB: resident CTAs per SM the registers are fitted to (2 for 4-row blocks)
 template <int P, int GPL, int NS>
 cudaError_t launch_pool_rows(const PoolParams& p, cudaStream_t st) {
+  constexpr int MB = P == 4 ? 2 : 1;
   const int smem = p.n_scales * p.d * static_cast<int>(sizeof(float));
-  cudaError_t e =
-      cudaFuncSetAttribute(pool_fuse_rows_kernel<P, GPL, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(pool_fuse_rows_kernel<P, GPL, NS, MB>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const size_t warps = static_cast<size_t>(p.B) * ((p.L + P - 1) / P);
-  return launch_pdl(pool_fuse_rows_kernel<P, GPL, NS>, dim3(static_cast<unsigned>((warps + 7) / 8)), dim3(256), smem,
-                    st, p);
+  return launch_pdl(pool_fuse_rows_kernel<P, GPL, NS, MB>, dim3(static_cast<unsigned>((warps + 7) / 8)), dim3(256),
+                    smem, st, p);
 }
 
 template <int P, int U>
@@ -873,7 +883,7 @@ cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st) {
   }
   if (p.n_scales * p.d * 4 <= 160 * 1024) {
     if (4 % lcm == 0)
-      return p.n_scales <= 4 ? launch_pool_rows<4, 4, 4>(p, st) : launch_pool_rows<4, 4, 8>(p, st);
+      return p.n_scales <= 4 ? launch_pool_rows<4, 2, 4>(p, st) : launch_pool_rows<4, 2, 8>(p, st);
     if (6 % lcm == 0)
       return p.n_scales <= 4 ? launch_pool_rows<6, 2, 4>(p, st) : launch_pool_rows<6, 2, 8>(p, st);
     if (8 % lcm == 0)
@@ -899,8 +909,10 @@ cudaError_t launch_gate(const GateParams& p, cudaStream_t st) {
 
 cudaError_t launch_hold_fuse(const HoldFuseParams& p, cudaStream_t st) {
   if (p.B * p.L == 0) return cudaSuccess;
-  const size_t n = static_cast<size_t>(p.B) * p.L * (p.d / 8);
-  return launch_pdl(hold_fuse_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st, p);
+  const int groups = p.d / 8;
+  const int CG = std::min(groups, 256), R = 256 / CG;
+  const dim3 grid((p.L + kHoldRows - 1) / kHoldRows, p.B, (groups + CG - 1) / CG);
+  return launch_pdl(hold_fuse_kernel, grid, dim3(CG * R), 0, st, p, CG, R);
 }
 
 cudaError_t launch_bf16_to_f16_rows(const __nv_bfloat16* src, int src_ld, int rows, int cols, __half* dst,

@@ -767,6 +767,9 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     for (int j = 0; j < ns; ++j) {
       hp.Y[j] = static_cast<const __half*>(at(ws.br[j].Y));
       hp.scales[j] = h->br[j].scale;
+      hp.shift[j] = -1;
+      for (int k = 0; k < 31; ++k)
+        if ((1 << k) == hp.scales[j]) hp.shift[j] = k;
       hp.rows[j] = ws.br[j].rows;
     }
     hp.w = static_cast<const float*>(at(ws.w));

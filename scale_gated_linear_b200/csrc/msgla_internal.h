@@ -205,6 +205,7 @@ cudaError_t launch_head_norm(const HeadNormParams& p, cudaStream_t st);
 struct HoldFuseParams {
   const __half* Y[kMaxScales];  // [B, n_s, d]
   int scales[kMaxScales];
+  int shift[kMaxScales];        // log2(scale) for a power of two, else -1
   int rows[kMaxScales];
   const float* w;               // [B, L, n_scales]
   __nv_bfloat16* out;           // [B, L, d]
