@@ -785,7 +785,7 @@ __global__ void __launch_bounds__(256) hold_fuse_kernel(const HoldFuseParams p, 
   const int t0 = blockIdx.x * kHoldRows, t1 = min(p.L, t0 + kHoldRows);
   uint4* ob = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.L * p.d) + cg;
   const float* wb = p.w + static_cast<size_t>(b) * p.L * p.n_scales;
-#pragma unroll 2
+#pragma unroll 4
   for (int t = t0 + r; t < t1; t += R) {
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
