@@ -811,6 +811,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
     tc_fence_after();
     tmem_dealloc_pair(tmem, 2 * kPairBN);
   }
+  if (dyn && p.tile_exit && threadIdx.x == 0) {
+    // this CTA takes no more tiles and waits for nothing more; the last CTA to
+    // leave clears the counters for the next launch
+    __threadfence();
+    if (atomicAdd(p.tile_exit, 1u) + 1u == gridDim.x) {
+      atomicExch(p.tile_counter, 0u);
+      for (int i = 0; i < p.n_reset64; ++i) atomicExch(p.reset64 + i, 0ull);
+      atomicExch(p.tile_exit, 0u);
+    }
+  }
 }
 
 }  // namespace

@@ -401,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (threadIdx.x == 0 && p.done && !state_pass) {
+  if (threadIdx.x == 0 && p.done && !state_pass && T.signal_done) {
     // every o row of this CTA is stored (the barrier above orders the stores of
     // all its threads before this release)
     __threadfence();

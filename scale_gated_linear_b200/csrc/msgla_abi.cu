@@ -142,14 +142,12 @@ struct msgla_handle {
   int* d_err;  // device error word
   int test_skip_arrival;  // failure-detection tests (msgla_test_skip_arrival)
   // Coarse output projection overlapped with the GLA kernel: a second stream,
-  // fork/join events, and per-branch GLA completion counters (monotonic) with
-  // the host's running count of GLA CTAs launched against each.
+  // fork/join events, per-branch GLA completion counters and a GLA start counter
+  // (all zero when a forward begins: the overlapped GEMM's last CTA clears them).
   cudaStream_t side;
   cudaEvent_t ev_fork, ev_join;
   unsigned long long* d_gla_done;  // [MSGLA_MAX_SCALES] completion, then [1] start counter
-  unsigned long long gla_total[MSGLA_MAX_SCALES];
-  unsigned long long gla_started;
-  unsigned int* d_tiles;           // dynamic tile counter of the overlapped GEMM
+  unsigned int* d_tiles;           // [2] dynamic tile and exit counters of the overlapped GEMM
   // host-buffer forward: copy streams and events of its pipeline
   cudaStream_t copy_in, copy_out;
   cudaEvent_t ev_start, ev_in, ev_done;
@@ -374,9 +372,7 @@ int create_impl(msgla_handle* h, const msgla_weights* w) {
   if (w->bfuse) CUDA_TRY(cudaMemcpy(h->bfuse, w->bfuse, h->n_scales * 4, cudaMemcpyDeviceToDevice));
   if ((st = dmalloc_zero(&h->d_err, sizeof(int)))) return st;
   if ((st = dmalloc_zero(&h->d_gla_done, (MSGLA_MAX_SCALES + 1) * sizeof(unsigned long long)))) return st;
-  if ((st = dmalloc_zero(&h->d_tiles, sizeof(unsigned int)))) return st;
-  for (int j = 0; j < MSGLA_MAX_SCALES; ++j) h->gla_total[j] = 0;
-  h->gla_started = 0;
+  if ((st = dmalloc_zero(&h->d_tiles, 2 * sizeof(unsigned int)))) return st;
   CUDA_TRY(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
   CUDA_TRY(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
   CUDA_TRY(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
@@ -616,17 +612,14 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   long long gla_ctas = 0;
   const bool overlap = coarse_overlap(h, ws, B, &gla_ctas);
   if (overlap) {
-    // the second stream starts once the gates are done, alongside the GLA
+    // the second stream starts once the gates are done, alongside the GLA; the
+    // coarse branches' CTAs signal their stored outputs to it
     lp.done = h->d_gla_done;
     lp.started = h->d_gla_done + MSGLA_MAX_SCALES;
+    for (int j = 0; j < ns; ++j) lp.task[j].signal_done = j != h->main_index;
     CUDA_TRY(cudaEventRecord(h->ev_fork, st));
   }
   CUDA_TRY(launch_gla(lp, st));
-  if (overlap) {
-    for (int j = 0; j < ns; ++j)
-      h->gla_total[j] += static_cast<unsigned long long>(B) * lp.task[j].heads * lp.task[j].v_tiles;
-    h->gla_started += static_cast<unsigned long long>(gla_ctas);
-  }
   CUDA_TRY(rec->mark(st));
 
   // 4b. optional per-head RMS norm of the GLA output (in place)
@@ -681,7 +674,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (output store, scale %d)", b.scale);
     if (overlap) {
       t.dep = h->d_gla_done + j;
-      t.dep_target = h->gla_total[j];
+      t.dep_target = static_cast<unsigned long long>(B) * b.heads * (h->dvp / kGlaTile);  // its GLA CTAs
     }
     tiles += B * t.m_tiles * t.n_tiles;
   }
@@ -690,9 +683,13 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     gp.total_tiles = tiles;
     if (overlap) {
       CUDA_TRY(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
-      CUDA_TRY(launch_wait_started(h->d_gla_done + MSGLA_MAX_SCALES, h->gla_started, h->d_err, h->side));
-      CUDA_TRY(cudaMemsetAsync(h->d_tiles, 0, sizeof(unsigned int), h->side));
+      CUDA_TRY(launch_wait_started(h->d_gla_done + MSGLA_MAX_SCALES, static_cast<unsigned long long>(gla_ctas),
+                                   h->d_err, h->side));
+      // the GEMM's last CTA clears the tile, start and completion counters
       gp.tile_counter = h->d_tiles;
+      gp.tile_exit = h->d_tiles + 1;
+      gp.reset64 = h->d_gla_done;
+      gp.n_reset64 = MSGLA_MAX_SCALES + 1;
       CUDA_TRY(launch_gemm(gp, 256, h->side));
       rec->unmarked += 2;
       CUDA_TRY(cudaEventRecord(h->ev_join, h->side));

@@ -99,6 +99,13 @@ struct GemmParams {
   int* err;
   // non-null: CTA pairs take tiles dynamically from *tile_counter (zero at launch)
   unsigned int* tile_counter;
+  // with tile_counter: every CTA adds 1 to *tile_exit when it leaves; the last one
+  // sets *tile_counter, *tile_exit and reset64[0, n_reset64) (the counters its
+  // tasks waited on) back to zero, so every launch starts from zero and a captured
+  // launch replays with the same targets
+  unsigned int* tile_exit;
+  unsigned long long* reset64;
+  int n_reset64;
 };
 
 // Chunkwise GLA over one or more branches.
@@ -113,7 +120,8 @@ struct alignas(64) GlaTask {
   // sequence segments (long sequences): chunks [s*seg_chunks, (s+1)*seg_chunks)
   float* seg_state;    // [B, h, v_tiles, n_segs, dkp, 128]: end states, then initial states
   float* seg_decay;    // [B, h, v_tiles, n_segs, dkp]: product of the state factors
-  int rows, n_chunks, heads, dkp, dvp, v_tiles, cta_begin, seg_chunks, n_segs, pad_;
+  int rows, n_chunks, heads, dkp, dvp, v_tiles, cta_begin, seg_chunks, n_segs;
+  int signal_done;  // full pass: this task's CTAs add 1 to GlaParams::done[task] when stored
 };
 
 struct GlaParams {
@@ -124,9 +132,9 @@ struct GlaParams {
   int mode;          // 0: full pass; 1: state pass over segments 0..n_segs-2
   int skip_arrival;  // failure-detection tests: CTA 0 omits one barrier arrival
   int* err;
-  // full pass only: every CTA of task t adds 1 to done[t] once its outputs are
-  // stored (release), for a concurrent consumer, and 1 to *started when it
-  // begins (null: none)
+  // full pass only: every CTA of a task with signal_done adds 1 to done[t] once
+  // its outputs are stored (release), for a concurrent consumer, and every CTA
+  // adds 1 to *started when it begins (null: none)
   unsigned long long* done;
   unsigned long long* started;
 };

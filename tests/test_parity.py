@@ -282,6 +282,42 @@ def test_forward_profiled_records_every_launch():
     layer.close()
 
 
+@needs_gpu
+def test_forward_replays_as_cuda_graph():
+    """A captured forward (the coarse output projection on the handle's second
+    stream beside the GLA, waiting on the GLA's start and completion counters)
+    replays three times with outputs bit-identical to an eager forward, and an
+    eager forward after the replays still matches: every launch starts its
+    counters from zero and waits for per-launch targets."""
+    w = wl.WORKLOADS["msgla_340m"].replace(name="graph", L=300)
+    inp = gpu_inputs(w)
+    layer = _layer(w, inp)
+    X = inp["X"].cuda()
+    B, L = X.shape[:2]
+    assert "out_gemm_coarse" not in layer.launch_names(B, L)  # overlapped with the GLA
+    ws = layer.alloc_workspace(B, L)
+    ref = torch.empty_like(X)
+    layer.forward(X, out=ref, workspace=ws)
+    torch.cuda.synchronize()
+    layer.check_status()
+    O = torch.empty_like(X)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.forward(X, out=O, workspace=ws, stream=torch.cuda.current_stream())
+    for _ in range(3):
+        O.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        layer.check_status()
+        assert torch.equal(O, ref)
+    again = layer.forward(X, workspace=ws)
+    torch.cuda.synchronize()
+    layer.check_status()
+    assert torch.equal(again, ref)
+    del graph
+    layer.close()
+
+
 _SERIAL_CHILD = """
 import sys, numpy as np, torch
 sys.path.insert(0, sys.argv[1])
