@@ -123,7 +123,9 @@ int msgla_workspace_size(const msgla_handle* h, int B, int L, size_t* bytes);
  * a second stream owned by the handle, concurrently with the GLA kernel (forked
  * after the gates, joined back before the final output projection), so all of
  * the forward's work is still ordered before what follows it on `stream`; the
- * fork and join use events, so the forward can be captured into a CUDA graph.
+ * fork and join use events, so the forward can be captured into a CUDA graph
+ * and replayed any number of times (the cross-stream counters start from zero
+ * at every launch and are cleared by the launch that waited on them).
  * The environment variable MSGLA_SERIAL=1 (read once per process) keeps every
  * kernel on `stream`: needed under profilers that run kernels one at a time,
  * where the concurrent GEMM's bounded wait for the GLA CTAs would time out.
