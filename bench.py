@@ -476,7 +476,8 @@ def run_ours(args) -> int:
         dom_ms = [ev[k][i_dom].elapsed_time(ev[k][i_dom + 1]) for k in range(steps)]
         total_ms = max_over_ranks(sum(step_ms), world, dev)
         res = {"total_ms": total_ms, "step_ms": step_ms, "dominant": dom, "dominant_ms": dom_ms,
-               "profiled_ms": prof, "launches": launches, "clocks": clocks, "tokens_per_step": wk.B * wk.L}
+               "profiled_ms": prof, "launches": launches, "clocks": clocks, "tokens_per_step": wk.B * wk.L,
+               "workspace_bytes": int(ws.numel())}
         if e2e:
             wsh = layer.alloc_workspace(wk.B, wk.L, host_staging=True)
             Xh = inp["X"].pin_memory()
@@ -541,6 +542,8 @@ def run_ours(args) -> int:
                           "boundaries and the dominant kernel",
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
+        "memory": {"workspace_bytes": r["workspace_bytes"],
+                   "note": "device intermediates of one forward (the caller-owned workspace)"},
     }
     if "e2e_ms" in r:
         line["e2e"] = {"value": tokens / (r["e2e_ms"] / 1e3), "unit": UNIT,
@@ -551,7 +554,9 @@ def run_ours(args) -> int:
         g = measure(wl.WORKLOADS[BASELINE_WORKLOAD], max(3, args.steps // 2), args.warmup, e2e=False)
         g_ms = g["total_ms"] / max(3, args.steps // 2)
         line["gla_baseline"] = {"workload": BASELINE_WORKLOAD, "value": g["tokens_per_step"] / (g_ms * 1e-3),
-                                "unit": UNIT, "ms_per_step": g_ms, "time_ratio_msgla_over_gla": step_ms / g_ms}
+                                "unit": UNIT, "ms_per_step": g_ms, "time_ratio_msgla_over_gla": step_ms / g_ms,
+                                "workspace_bytes": g["workspace_bytes"],
+                                "workspace_ratio_msgla_over_gla": r["workspace_bytes"] / g["workspace_bytes"]}
     if cpu_line is not None:
         line["cpu_baseline"] = cpu_line
     if rank == 0:
