@@ -125,6 +125,24 @@ def test_wide_scale_set_small():
 
 
 @needs_gpu
+@pytest.mark.parametrize("L", [200, 201])
+def test_two_row_pooling(L):
+    """Scales {1, 2}: with an even length and no mask the pooling runs the flat
+    2-row kernel, with an odd one the per-block kernel; pooled rows and output
+    match the oracle either way."""
+    from scale_gated_linear_b200 import WS_POOLED
+    w = SMALL.replace(name="s12", scales=(1, 2), heads=(2, 1))
+    inp = gpu_inputs(w, L=L)
+    got, layer, ws = run_gpu(w, inp)
+    ref, inter = oracle_forward(w, inp, intermediates=True)
+    assert_parity(got, ref)
+    pooled = layer.workspace_tensor(ws, w.B, L, 1, WS_POOLED).float().cpu().numpy()
+    want = inter["branches"][1]["Xp"]
+    assert np.abs(pooled - want).max() <= 1e-3 * np.abs(want).max()
+    layer.close()
+
+
+@needs_gpu
 @pytest.mark.parametrize("scales,heads", [((1, 3), (2, 1)), ((2, 3), (1, 1)), ((1, 2, 6), (1, 1, 1)),
                                           ((1, 5), (1, 1)), ((2, 5), (1, 1)), ((3,), (2,))])
 def test_scale_sets_beyond_powers_of_two(scales, heads):
