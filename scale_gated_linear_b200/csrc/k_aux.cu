@@ -2,7 +2,11 @@
 //   pool_fuse_kernel  one pass over X: mean pooling of s adjacent rows for every
 //                     scale s > 1 (reading notes Sec. 3.1, Eq. (8)) and the
 //                     fusion weights w_t = softmax(W_fuse x_t + b_fuse) from the
-//                     unpooled rows (Sec. 3.3, Eq. (10)).
+//                     unpooled rows (Sec. 3.3, Eq. (10)); pool_fuse_rows_kernel
+//                     does both per row block when there is no scale-1 branch,
+//                     pool_rows_kernel and pool_rows_flat_kernel pool only (with
+//                     a scale-1 branch the fusion logits come from its
+//                     projection GEMM).
 //   gate_kernel       log alpha = logsigmoid(g W_g2^T + b_g) / normalizer (the
 //                     low-rank gate of Sec. 2.1), its cumulative sum b inside
 //                     each 128-row GLA chunk referenced to the chunk's 64th
