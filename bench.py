@@ -24,7 +24,9 @@ launched so that each may start while the previous one finishes, and an event
 between two kernels takes that overlap away, so the timed steps record events
 only at the step boundaries and around the dominant kernel (for the roofline);
 the dominant kernel and the per-kernel table (kernel_ms) come from separate
-forwards with an event at every kernel boundary.
+forwards with an event at every kernel boundary. The line also carries the
+forward's workspace bytes (`memory`) and, beside the single-scale GLA layer's
+throughput, its workspace bytes and the ratio of the two.
 """
 from __future__ import annotations
 

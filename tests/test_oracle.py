@@ -439,6 +439,27 @@ def test_half_life():
         assert abs(a ** i_half - 0.5) < 1e-12
 
 
+def test_coarse_gate_input_is_block_mean_of_row_projections():
+    """Eq. (8) is linear, so a coarse branch's low-rank gate input xbar_i W_g1^T
+    equals the mean over block i of x_j W_g1^T (a ragged tail block: over its
+    rows inside L). log alpha rebuilt that way from the unpooled rows, with the
+    sigmoid written out, agrees with the oracle's."""
+    rng = np.random.default_rng(41)
+    d, dk, dv, L = 8, 3, 5, 23  # 23 leaves ragged tail blocks at s = 2 and 4
+    scales, heads = (1, 2, 4), (1, 1, 1)
+    W = _rand_weights(rng, d, scales, heads, dk, dv, gate_bias=0.3)
+    X = rng.normal(size=(1, L, d))
+    _, inter = om.layer_forward(X, W, scales, heads, dk, dv, intermediates=True)
+    for j, s in enumerate(scales):
+        br = W["branches"][j]
+        g_rows = X[0] @ br["Wg1"].T
+        n = -(-L // s)
+        g = np.stack([g_rows[i * s:min(L, (i + 1) * s)].mean(axis=0) for i in range(n)])
+        z = g @ br["Wg2"].T + br["bg"]
+        la = np.log(1.0 / (1.0 + np.exp(-z))) / 16.0
+        np.testing.assert_allclose(inter["branches"][j]["log_alpha"][0], la, rtol=1e-10, atol=1e-14)
+
+
 def test_fusion_weights_simplex():
     rng = np.random.default_rng(7)
     X = rng.normal(size=(50, 16)) * 5
