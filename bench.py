@@ -47,7 +47,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MS-GLA layer fwd tokens/sec @d=1024,L=2048"
 UNIT = "tokens/s"
 WORKLOAD = "msgla_340m"
-BASELINE_WORKLOAD = "gla_340m"
+SINGLE_SCALE_WORKLOAD = "gla_340m"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -553,9 +553,9 @@ def run_ours(args) -> int:
     elif args.mask != "none":
         line["e2e"] = {"value": None, "unit": UNIT, "note": "not measured: the host-buffer entry point takes no mask"}
     if world == 1 and not args.no_gla_baseline and args.mask == "none" and not w.head_norm:
-        g = measure(wl.WORKLOADS[BASELINE_WORKLOAD], max(3, args.steps // 2), args.warmup, e2e=False)
+        g = measure(wl.WORKLOADS[SINGLE_SCALE_WORKLOAD], max(3, args.steps // 2), args.warmup, e2e=False)
         g_ms = g["total_ms"] / max(3, args.steps // 2)
-        line["gla_baseline"] = {"workload": BASELINE_WORKLOAD, "value": g["tokens_per_step"] / (g_ms * 1e-3),
+        line["gla_baseline"] = {"workload": SINGLE_SCALE_WORKLOAD, "value": g["tokens_per_step"] / (g_ms * 1e-3),
                                 "unit": UNIT, "ms_per_step": g_ms, "time_ratio_msgla_over_gla": step_ms / g_ms,
                                 "workspace_bytes": g["workspace_bytes"],
                                 "workspace_ratio_msgla_over_gla": r["workspace_bytes"] / g["workspace_bytes"]}
