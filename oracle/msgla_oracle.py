@@ -56,7 +56,8 @@ worked s = 4 hold table and pooling example of Sec. 3.1/3.3, a masked s = 4
 pooling example with an all-padding block, unit RMS per head and invariance to
 the value scale of the optional head normalisation, causality,
 half-life, the 11/16 update count and the simplex property of the fusion
-weights.
+weights. The gradients (``layer_backward``, for a backward pass that has no
+GPU counterpart yet) are pinned by central finite differences of the forward.
 """
 from __future__ import annotations
 
@@ -229,6 +230,117 @@ def layer_forward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: in
         for name in list(br):
             br[name] = np.stack(br[name]) if br[name] else None
     return O, inter
+
+
+# ---------------------------------------------------------------------------
+# gradients (the backward pass of training; pinned by finite differences)
+# ---------------------------------------------------------------------------
+def gla_recurrent_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, log_alpha: np.ndarray,
+                           do: np.ndarray, qk_scale: float = 1.0):
+    """Adjoints of ``gla_recurrent`` for the output adjoint do [n, d_v]:
+    returns dq, dk, dv, dlog_alpha.
+
+    The forward keeps every state S_t. Walking back from the last step, G holds
+    the adjoint of S_t: G_t = qk_scale q_t^T do_t + Diag(alpha_{t+1}) G_{t+1}.
+    Then dq_t = qk_scale S_t do_t^T, dk_t = G_t v_t^T, dv_t = k_t G_t, and
+    d alpha_t = rowsum(G_t * S_{t-1}) (elementwise), d log alpha_t = alpha_t *
+    d alpha_t."""
+    n, dk_ = q.shape
+    dv_ = v.shape[1]
+    alpha = np.exp(log_alpha)
+    S = np.zeros((n + 1, dk_, dv_), dtype=np.float64)
+    for t in range(n):
+        S[t + 1] = alpha[t][:, None] * S[t] + np.outer(k[t], v[t])
+    dq = np.zeros_like(q, dtype=np.float64)
+    dkk = np.zeros_like(k, dtype=np.float64)
+    dvv = np.zeros_like(v, dtype=np.float64)
+    dla = np.zeros_like(log_alpha, dtype=np.float64)
+    G = np.zeros((dk_, dv_), dtype=np.float64)
+    for t in range(n - 1, -1, -1):
+        G = G + qk_scale * np.outer(q[t], do[t])
+        dq[t] = qk_scale * (S[t + 1] @ do[t])
+        dkk[t] = G @ v[t]
+        dvv[t] = k[t] @ G
+        dla[t] = alpha[t] * (G * S[t]).sum(axis=1)
+        G = alpha[t][:, None] * G
+    return dq, dkk, dvv, dla
+
+
+def layer_backward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: int, dO: np.ndarray,
+                   gate_normalizer: float = 16.0, qk_scale: float = 1.0, mask: np.ndarray | None = None):
+    """Gradients of sum(O * dO), O = layer_forward(X, ...) with the per-head norm
+    off: returns dX [B, L, d] and a dict shaped like ``weights`` (``branches``
+    with Wq, Wk, Wv, Wg1, Wg2, bg, Wo each; ``Wfuse``, ``bfuse``).
+
+    The steps of the forward in reverse: the fusion softmax (dz = w * (dw -
+    sum_s w_s dw_s) with dw_{t,s} = dO_t . Yhat^(s)_t), the causal hold (dY_i
+    sums dYhat_t over the positions t that read row i), W_o, the GLA recurrence
+    per head (gla_recurrent_backward), the gate (d/du logsigmoid(u) =
+    sigmoid(-u)), the projections, and the pooling of Eq. (8) (each valid row of
+    block i receives dXbar_i / max(1, sum M))."""
+    X = np.asarray(X, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    B, L, d = X.shape
+    names = ("Wq", "Wk", "Wv", "Wg1", "Wg2", "bg", "Wo")
+    grads = {"branches": [{n_: np.zeros_like(np.asarray(br[n_], dtype=np.float64)) for n_ in names}
+                          for br in weights["branches"]],
+             "Wfuse": np.zeros_like(np.asarray(weights["Wfuse"], dtype=np.float64)),
+             "bfuse": np.zeros_like(np.asarray(weights["bfuse"], dtype=np.float64))}
+    dX = np.zeros_like(X)
+    for b in range(B):
+        M = None if mask is None else np.asarray(mask[b], dtype=np.float64)
+        w = fusion_weights(X[b], weights["Wfuse"], weights["bfuse"])
+        fwd = []
+        for j, (s, h) in enumerate(zip(scales, heads)):
+            br = weights["branches"][j]
+            Xp = pool(X[b], s, M)
+            q, k, v, la = branch_projections(Xp, br, gate_normalizer)
+            o = np.zeros((Xp.shape[0], h * d_v), dtype=np.float64)
+            for hh in range(h):
+                ck, cv = slice(hh * d_k, (hh + 1) * d_k), slice(hh * d_v, (hh + 1) * d_v)
+                o[:, cv] = gla_recurrent(q[:, ck], k[:, ck], v[:, cv], la[:, ck], qk_scale=qk_scale)
+            Y = o @ br["Wo"].T
+            fwd.append((Xp, q, k, v, la, o, Y, hold(Y, s, L)))
+        # fusion: O_t = sum_s w_{t,s} Yhat^(s)_t, w_t = softmax(z_t), z_t = W_fuse x_t + b_fuse
+        dw = np.stack([(dO[b] * f[7]).sum(axis=1) for f in fwd], axis=1)
+        dz = w * (dw - (w * dw).sum(axis=1, keepdims=True))
+        grads["Wfuse"] += dz.T @ X[b]
+        grads["bfuse"] += dz.sum(axis=0)
+        dX[b] += dz @ weights["Wfuse"]
+        for j, (s, h) in enumerate(zip(scales, heads)):
+            br, gb = weights["branches"][j], grads["branches"][j]
+            Xp, q, k, v, la, o, Y, _ = fwd[j]
+            dYhat = w[:, j:j + 1] * dO[b]
+            dY = np.zeros_like(Y)
+            for t in range(L):
+                i = hold_index(t, s)
+                if i >= 0:
+                    dY[i] += dYhat[t]
+            gb["Wo"] += dY.T @ o
+            do = dY @ br["Wo"]
+            dq, dk, dv, dla = (np.zeros_like(q), np.zeros_like(k), np.zeros_like(v), np.zeros_like(la))
+            for hh in range(h):
+                ck, cv = slice(hh * d_k, (hh + 1) * d_k), slice(hh * d_v, (hh + 1) * d_v)
+                dq[:, ck], dk[:, ck], dv[:, cv], dla[:, ck] = gla_recurrent_backward(
+                    q[:, ck], k[:, ck], v[:, cv], la[:, ck], do[:, cv], qk_scale=qk_scale)
+            g = Xp @ br["Wg1"].T
+            u = g @ br["Wg2"].T + br["bg"]
+            du = dla / gate_normalizer * np.exp(-np.logaddexp(0.0, u))  # sigmoid(-u)
+            gb["Wg2"] += du.T @ g
+            gb["bg"] += du.sum(axis=0)
+            dg = du @ br["Wg2"]
+            gb["Wg1"] += dg.T @ Xp
+            gb["Wq"] += dq.T @ Xp
+            gb["Wk"] += dk.T @ Xp
+            gb["Wv"] += dv.T @ Xp
+            dXp = dq @ br["Wq"] + dk @ br["Wk"] + dv @ br["Wv"] + dg @ br["Wg1"]
+            Mb = np.ones(L) if M is None else M
+            for i in range(Xp.shape[0]):
+                rows = [i * s + r for r in range(s) if i * s + r < L]
+                cnt = max(1.0, sum(Mb[r] for r in rows))
+                for r in rows:
+                    dX[b, r] += Mb[r] * dXp[i] / cnt
+    return dX, grads
 
 
 # ---------------------------------------------------------------------------

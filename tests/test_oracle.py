@@ -460,6 +460,73 @@ def test_coarse_gate_input_is_block_mean_of_row_projections():
         np.testing.assert_allclose(inter["branches"][j]["log_alpha"][0], la, rtol=1e-10, atol=1e-14)
 
 
+# --------------------------------------------------------------------------
+# gradients (layer_backward): central finite differences of the forward
+# --------------------------------------------------------------------------
+def _check_gradients(X, W, scales, heads, dk, dv, mask=None, qk_scale=1.0, seed=0, eps=1e-6, rtol=1e-6):
+    dO = np.random.default_rng(seed).normal(size=X.shape)
+    dX, g = om.layer_backward(X, W, scales, heads, dk, dv, dO, qk_scale=qk_scale, mask=mask)
+
+    def loss():
+        return float((om.layer_forward(X, W, scales, heads, dk, dv, qk_scale=qk_scale, mask=mask) * dO).sum())
+
+    def finite_difference(arr):
+        out = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            keep = arr[idx]
+            arr[idx] = keep + eps
+            up = loss()
+            arr[idx] = keep - eps
+            down = loss()
+            arr[idx] = keep
+            out[idx] = (up - down) / (2 * eps)
+        return out
+
+    # central differences carry about |loss| * 2^-52 / eps ~ 1e-8 of rounding noise;
+    # the 1e-7 floor is still ~1e-4 of the smallest gradient block checked
+    def close(name, got, want):
+        assert np.abs(got - want).max() <= rtol * np.abs(want).max() + 1e-7, name
+
+    close("X", dX, finite_difference(X))
+    for j, br in enumerate(W["branches"]):
+        for name in ("Wq", "Wk", "Wv", "Wg1", "Wg2", "bg", "Wo"):
+            close(f"{name} of branch {j}", g["branches"][j][name], finite_difference(br[name]))
+    close("Wfuse", g["Wfuse"], finite_difference(W["Wfuse"]))
+    close("bfuse", g["bfuse"], finite_difference(W["bfuse"]))
+
+
+def check_gradients_plain():
+    """Every gradient of layer_backward (input, all projections, gate factors
+    and bias, output projections, fusion weights and bias) against central
+    differences of layer_forward; ragged tail blocks at s = 2 and 4."""
+    rng = np.random.default_rng(51)
+    d, dk, dv, L = 5, 3, 2, 9
+    W = _rand_weights(rng, d, (1, 2, 4), (1, 1, 1), dk, dv, gate_bias=0.5)
+    W["bfuse"] = rng.normal(size=3)
+    X = rng.normal(size=(2, L, d))
+    _check_gradients(X, W, (1, 2, 4), (1, 1, 1), dk, dv, seed=52)
+
+
+def check_gradients_masked():
+    """The same with a padding mask in the pooling, qk_scale 0.7, two heads on
+    one branch and no scale-1 branch (scales 2 and 3)."""
+    rng = np.random.default_rng(53)
+    d, dk, dv, L = 4, 2, 3, 8
+    W = _rand_weights(rng, d, (2, 3), (2, 1), dk, dv, gate_bias=-0.3)
+    X = rng.normal(size=(2, L, d))
+    mask = np.ones((2, L))
+    mask[1, :3] = 0.0  # left padding of the second sequence
+    _check_gradients(X, W, (2, 3), (2, 1), dk, dv, mask=mask, qk_scale=0.7, seed=54)
+
+
+def test_gradients_match_finite_differences():
+    check_gradients_plain()
+
+
+def test_gradients_with_mask_scale_and_no_fine_branch():
+    check_gradients_masked()
+
+
 def test_fusion_weights_simplex():
     rng = np.random.default_rng(7)
     X = rng.normal(size=(50, 16)) * 5
@@ -585,6 +652,31 @@ def _mutant_decode_buffer_kept(cache, x, weights, scales, heads, d_k, d_v, **kw)
     return out
 
 
+_real_gla_backward = om.gla_recurrent_backward
+
+
+def _mutant_gla_backward_no_alpha(q, k, v, log_alpha, do, qk_scale=1.0):
+    dq, dk, dv, dla = _real_gla_backward(q, k, v, log_alpha, do, qk_scale)
+    return dq, dk, dv, dla / np.exp(log_alpha)          # d alpha instead of d log alpha
+
+
+def _mutant_gla_backward_no_carry(q, k, v, log_alpha, do, qk_scale=1.0):
+    n = q.shape[0]
+    out = [np.zeros_like(a, dtype=float) for a in (q, k, v, log_alpha)]
+    for t in range(n):                                  # drops the adjoint carried from later steps
+        g = [np.zeros_like(do)]
+        g[0][t] = do[t]
+        parts = _real_gla_backward(q[:t + 1], k[:t + 1], v[:t + 1], log_alpha[:t + 1], g[0][:t + 1], qk_scale)
+        for a, p in zip(out, parts):
+            a[t] += p[t]
+    return tuple(out)
+
+
+def _mutant_gla_backward_k_for_v(q, k, v, log_alpha, do, qk_scale=1.0):
+    dq, dk, dv, dla = _real_gla_backward(q, k, v, log_alpha, do, qk_scale)
+    return dq, dk[:, ::-1], dv, dla                     # key adjoint channels reversed
+
+
 def _mutant_softmax_wrong_axis(X, Wfuse, bfuse):
     z = X @ Wfuse.T + bfuse
     return np.exp(z) / np.exp(z).sum(axis=0, keepdims=True)
@@ -592,7 +684,8 @@ def _mutant_softmax_wrong_axis(X, Wfuse, bfuse):
 
 PINS = [check_hold_table, check_pool_example, check_pool_tail, check_pool_mask, check_gla_bruteforce,
         check_layer_bruteforce, check_constant_input_closed_form, check_head_norm_unit_rms,
-        check_head_norm_constant_row, check_decode_matches_parallel]
+        check_head_norm_constant_row, check_decode_matches_parallel, check_gradients_plain,
+        check_gradients_masked]
 
 
 @pytest.mark.parametrize("name,mutant", [
@@ -609,6 +702,9 @@ PINS = [check_hold_table, check_pool_example, check_pool_tail, check_pool_mask, 
     ("head_rmsnorm", _mutant_head_norm_no_weight),
     ("decode_step", _mutant_decode_one_step_late),
     ("decode_step", _mutant_decode_buffer_kept),
+    ("gla_recurrent_backward", _mutant_gla_backward_no_alpha),
+    ("gla_recurrent_backward", _mutant_gla_backward_no_carry),
+    ("gla_recurrent_backward", _mutant_gla_backward_k_for_v),
 ])
 def test_planted_mistake_is_caught(monkeypatch, name, mutant):
     monkeypatch.setattr(om, name, mutant)
