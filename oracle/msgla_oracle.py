@@ -266,18 +266,43 @@ def gla_recurrent_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, log_alph
     return dq, dkk, dvv, dla
 
 
+def _norm_weight(br: dict, h: int, d_v: int) -> np.ndarray:
+    """The branch's per-channel head-norm weight [h*d_v] (all ones when absent)."""
+    nw = br.get("norm_w")
+    return np.ones(h * d_v) if nw is None else np.asarray(nw, dtype=np.float64)
+
+
+def head_rmsnorm_backward(o: np.ndarray, weight: np.ndarray, eps: float, dy: np.ndarray):
+    """Adjoints of ``head_rmsnorm`` for dy [n, d_v]: returns do and dweight.
+    With r_t = sqrt(mean(o_t^2) + eps) and y_t = o_t / r_t * weight:
+    do_t = (dy_t * weight) / r_t - o_t * sum(dy_t * weight * o_t) / (d_v r_t^3),
+    dweight = sum_t dy_t * o_t / r_t."""
+    n, dv_ = o.shape
+    do = np.zeros_like(o, dtype=np.float64)
+    dweight = np.zeros_like(weight, dtype=np.float64)
+    for t in range(n):
+        r = np.sqrt(float(np.dot(o[t], o[t])) / dv_ + eps)
+        gw = dy[t] * weight
+        do[t] = gw / r - o[t] * float(np.dot(gw, o[t])) / (dv_ * r ** 3)
+        dweight += dy[t] * o[t] / r
+    return do, dweight
+
+
 def layer_backward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: int, dO: np.ndarray,
-                   gate_normalizer: float = 16.0, qk_scale: float = 1.0, mask: np.ndarray | None = None):
-    """Gradients of sum(O * dO), O = layer_forward(X, ...) with the per-head norm
-    off: returns dX [B, L, d] and a dict shaped like ``weights`` (``branches``
-    with Wq, Wk, Wv, Wg1, Wg2, bg, Wo each; ``Wfuse``, ``bfuse``).
+                   gate_normalizer: float = 16.0, qk_scale: float = 1.0, mask: np.ndarray | None = None,
+                   head_norm_eps: float | None = None):
+    """Gradients of sum(O * dO), O = layer_forward(X, ...) with the same
+    arguments: returns dX [B, L, d] and a dict shaped like ``weights``
+    (``branches`` with Wq, Wk, Wv, Wg1, Wg2, bg, Wo each, and norm_w when the
+    per-head norm is on; ``Wfuse``, ``bfuse``).
 
     The steps of the forward in reverse: the fusion softmax (dz = w * (dw -
     sum_s w_s dw_s) with dw_{t,s} = dO_t . Yhat^(s)_t), the causal hold (dY_i
     sums dYhat_t over the positions t that read row i), W_o, the GLA recurrence
     per head (gla_recurrent_backward), the gate (d/du logsigmoid(u) =
     sigmoid(-u)), the projections, and the pooling of Eq. (8) (each valid row of
-    block i receives dXbar_i / max(1, sum M))."""
+    block i receives dXbar_i / max(1, sum M)); with the per-head norm, its
+    adjoint (head_rmsnorm_backward) sits between W_o and the recurrence."""
     X = np.asarray(X, dtype=np.float64)
     dO = np.asarray(dO, dtype=np.float64)
     B, L, d = X.shape
@@ -295,21 +320,26 @@ def layer_backward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: i
             br = weights["branches"][j]
             Xp = pool(X[b], s, M)
             q, k, v, la = branch_projections(Xp, br, gate_normalizer)
-            o = np.zeros((Xp.shape[0], h * d_v), dtype=np.float64)
+            o_raw = np.zeros((Xp.shape[0], h * d_v), dtype=np.float64)
             for hh in range(h):
                 ck, cv = slice(hh * d_k, (hh + 1) * d_k), slice(hh * d_v, (hh + 1) * d_v)
-                o[:, cv] = gla_recurrent(q[:, ck], k[:, ck], v[:, cv], la[:, ck], qk_scale=qk_scale)
+                o_raw[:, cv] = gla_recurrent(q[:, ck], k[:, ck], v[:, cv], la[:, ck], qk_scale=qk_scale)
+            o = o_raw.copy()
+            if head_norm_eps is not None:
+                for hh in range(h):
+                    cv = slice(hh * d_v, (hh + 1) * d_v)
+                    o[:, cv] = head_rmsnorm(o_raw[:, cv], _norm_weight(br, h, d_v)[cv], head_norm_eps)
             Y = o @ br["Wo"].T
-            fwd.append((Xp, q, k, v, la, o, Y, hold(Y, s, L)))
+            fwd.append((Xp, q, k, v, la, o_raw, o, Y, hold(Y, s, L)))
         # fusion: O_t = sum_s w_{t,s} Yhat^(s)_t, w_t = softmax(z_t), z_t = W_fuse x_t + b_fuse
-        dw = np.stack([(dO[b] * f[7]).sum(axis=1) for f in fwd], axis=1)
+        dw = np.stack([(dO[b] * f[8]).sum(axis=1) for f in fwd], axis=1)
         dz = w * (dw - (w * dw).sum(axis=1, keepdims=True))
         grads["Wfuse"] += dz.T @ X[b]
         grads["bfuse"] += dz.sum(axis=0)
         dX[b] += dz @ weights["Wfuse"]
         for j, (s, h) in enumerate(zip(scales, heads)):
             br, gb = weights["branches"][j], grads["branches"][j]
-            Xp, q, k, v, la, o, Y, _ = fwd[j]
+            Xp, q, k, v, la, o_raw, o, Y, _ = fwd[j]
             dYhat = w[:, j:j + 1] * dO[b]
             dY = np.zeros_like(Y)
             for t in range(L):
@@ -318,6 +348,13 @@ def layer_backward(X: np.ndarray, weights: dict, scales, heads, d_k: int, d_v: i
                     dY[i] += dYhat[t]
             gb["Wo"] += dY.T @ o
             do = dY @ br["Wo"]
+            if head_norm_eps is not None:
+                nw = _norm_weight(br, h, d_v)
+                gb.setdefault("norm_w", np.zeros(h * d_v))
+                for hh in range(h):
+                    cv = slice(hh * d_v, (hh + 1) * d_v)
+                    do[:, cv], dnw = head_rmsnorm_backward(o_raw[:, cv], nw[cv], head_norm_eps, do[:, cv])
+                    gb["norm_w"][cv] += dnw
             dq, dk, dv, dla = (np.zeros_like(q), np.zeros_like(k), np.zeros_like(v), np.zeros_like(la))
             for hh in range(h):
                 ck, cv = slice(hh * d_k, (hh + 1) * d_k), slice(hh * d_v, (hh + 1) * d_v)

@@ -463,12 +463,15 @@ def test_coarse_gate_input_is_block_mean_of_row_projections():
 # --------------------------------------------------------------------------
 # gradients (layer_backward): central finite differences of the forward
 # --------------------------------------------------------------------------
-def _check_gradients(X, W, scales, heads, dk, dv, mask=None, qk_scale=1.0, seed=0, eps=1e-6, rtol=1e-6):
+def _check_gradients(X, W, scales, heads, dk, dv, mask=None, qk_scale=1.0, seed=0, eps=1e-6, rtol=1e-6,
+                     head_norm_eps=None):
     dO = np.random.default_rng(seed).normal(size=X.shape)
-    dX, g = om.layer_backward(X, W, scales, heads, dk, dv, dO, qk_scale=qk_scale, mask=mask)
+    dX, g = om.layer_backward(X, W, scales, heads, dk, dv, dO, qk_scale=qk_scale, mask=mask,
+                              head_norm_eps=head_norm_eps)
 
     def loss():
-        return float((om.layer_forward(X, W, scales, heads, dk, dv, qk_scale=qk_scale, mask=mask) * dO).sum())
+        return float((om.layer_forward(X, W, scales, heads, dk, dv, qk_scale=qk_scale, mask=mask,
+                                       head_norm_eps=head_norm_eps) * dO).sum())
 
     def finite_difference(arr):
         out = np.zeros_like(arr)
@@ -489,7 +492,7 @@ def _check_gradients(X, W, scales, heads, dk, dv, mask=None, qk_scale=1.0, seed=
 
     close("X", dX, finite_difference(X))
     for j, br in enumerate(W["branches"]):
-        for name in ("Wq", "Wk", "Wv", "Wg1", "Wg2", "bg", "Wo"):
+        for name in ("Wq", "Wk", "Wv", "Wg1", "Wg2", "bg", "Wo") + (("norm_w",) if head_norm_eps else ()):
             close(f"{name} of branch {j}", g["branches"][j][name], finite_difference(br[name]))
     close("Wfuse", g["Wfuse"], finite_difference(W["Wfuse"]))
     close("bfuse", g["bfuse"], finite_difference(W["bfuse"]))
@@ -519,8 +522,23 @@ def check_gradients_masked():
     _check_gradients(X, W, (2, 3), (2, 1), dk, dv, mask=mask, qk_scale=0.7, seed=54)
 
 
+def check_gradients_head_norm():
+    """The same with the optional per-head RMS norm (and its weight) on."""
+    rng = np.random.default_rng(55)
+    d, dk, dv, L = 4, 2, 3, 7
+    W = _rand_weights(rng, d, (1, 2), (1, 2), dk, dv)
+    for j, h in enumerate((1, 2)):
+        W["branches"][j]["norm_w"] = rng.normal(1.0, 0.3, size=h * dv)
+    X = rng.normal(size=(1, L, d))
+    _check_gradients(X, W, (1, 2), (1, 2), dk, dv, seed=56, head_norm_eps=1e-3)
+
+
 def test_gradients_match_finite_differences():
     check_gradients_plain()
+
+
+def test_gradients_with_head_norm():
+    check_gradients_head_norm()
 
 
 def test_gradients_with_mask_scale_and_no_fine_branch():
@@ -685,7 +703,7 @@ def _mutant_softmax_wrong_axis(X, Wfuse, bfuse):
 PINS = [check_hold_table, check_pool_example, check_pool_tail, check_pool_mask, check_gla_bruteforce,
         check_layer_bruteforce, check_constant_input_closed_form, check_head_norm_unit_rms,
         check_head_norm_constant_row, check_decode_matches_parallel, check_gradients_plain,
-        check_gradients_masked]
+        check_gradients_masked, check_gradients_head_norm]
 
 
 @pytest.mark.parametrize("name,mutant", [
