@@ -47,7 +47,8 @@ notes of this repository):
   unpooled row x_t whatever its mask.
 
 Every step is written token by token or row by row; numpy's matmul is used as
-a library primitive for the per-row projections only.
+a library primitive for the per-row projections only (and, in the gradients,
+for their transposed products: dW = dYᵀ X and dX = dY W).
 
 Parity pins (tests/test_oracle.py): brute-force quadratic form of the GLA
 recurrence, alpha = 1 reducing to causal (Q K^T) V, the single-scale layer
