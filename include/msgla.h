@@ -210,11 +210,18 @@ int msgla_sync_status(msgla_handle* h);
 
 /* Intermediate tensors inside the workspace of a forward with the same B and L
  * (for inspection by tests and tools; valid after the forward completes).
- * `which`: 0 pooled X (fp16 [B, n_s, d]; scales > 1 only), 1 q (fp16 [B, n_s, h*dkp]),
- * 2 k, 3 v (fp16 [B, n_s, h*dvp]), 4 gate low-rank g (f32 [B, n_s, rp]),
- * 5 o (fp16 [B, n_s, h*dvp]), 6 Y (fp16 [B, n_s, d]; branches whose output is
- * materialised), 7 fusion weights w (f32 [B, L, n_scales]; `scale_index` ignored).
- * dkp, dvp and rp are the padded widths reported in dims[2] (columns). Padding
+ * With b the cumulative sum of log alpha over the rows of a 128-row chunk (from
+ * its first row) and m its value at the chunk's row 63, per key channel:
+ * `which`: 0 pooled X (fp16 [B, n_s, d]; scales > 1 only),
+ * 1 Qs = q e^{b - m} (fp16 [B, n_s, h*dkp]), 2 Ks = k e^{m - b} (same shape),
+ * 3 v (fp16 [B, n_s, h*dvp]), 5 o (fp16 [B, n_s, h*dvp]), 6 Y (fp16 [B, n_s, d];
+ * branches whose output is materialised), 7 fusion weights w (f32 [B, L, n_scales]),
+ * 8 U = X Wu^T (f32 [B, L, ldu]): the fusion logits W_fuse x_t in columns
+ * 0..n_scales-1 and the low-rank gate input x_t W_g1^T of scale index j in columns
+ * 16 + j*rp .. (unpooled rows; a coarse branch uses their block means),
+ * 9 gamma = e^{b_last - m} and 10 mid = e^{m} (f32 [B, n_chunks, h*dkp], n_chunks =
+ * ceil(n_s / 128)). `scale_index` is ignored for 7 and 8. dkp, dvp and rp (the gate
+ * rank rounded up to 16) are padded widths; dims[2] reports the columns. Padding
  * columns hold zeros. A tensor that does not exist gives MSGLA_ERR_INVALID_ARG. */
 int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index, int which,
                            size_t* offset, int dims[3]);

@@ -15,7 +15,8 @@ import ctypes
 from typing import Optional, Sequence
 
 from . import _lib
-from ._lib import MSGLAError, WS_FUSION, WS_GATE, WS_K, WS_O, WS_POOLED, WS_Q, WS_V, WS_Y
+from ._lib import (MSGLAError, WS_FUSION, WS_GAMMA, WS_KS, WS_MID, WS_O, WS_POOLED, WS_QS, WS_U, WS_V,
+                   WS_Y)
 
 __all__ = ["MSGLA", "MSGLAError", "load_library"]
 
@@ -220,7 +221,7 @@ class MSGLA:
         off = ctypes.c_size_t()
         dims = (ctypes.c_int * 3)()
         _lib.check(self._lib.msgla_workspace_tensor(self._h, B, L, scale_index, which, ctypes.byref(off), dims))
-        dtype = torch.float32 if which in (WS_GATE, WS_FUSION) else torch.float16
+        dtype = torch.float32 if which in (WS_FUSION, WS_U, WS_GAMMA, WS_MID) else torch.float16
         esz = 4 if dtype == torch.float32 else 2
         n = dims[0] * dims[1] * dims[2]
         raw = workspace[off.value: off.value + n * esz]

@@ -18,7 +18,11 @@ STATUS = {0: "MSGLA_OK", -1: "MSGLA_ERR_INVALID_ARG", -2: "MSGLA_ERR_UNSUPPORTED
           -4: "MSGLA_ERR_DEVICE_TIMEOUT", -5: "MSGLA_ERR_RANGE", -6: "MSGLA_ERR_WORKSPACE"}
 
 # which-codes of msgla_workspace_tensor
-WS_POOLED, WS_Q, WS_K, WS_V, WS_GATE, WS_O, WS_Y, WS_FUSION = range(8)
+# msgla_workspace_tensor views: WS_QS / WS_KS are the decay-scaled queries and keys
+# (q e^{b-m}, k e^{m-b} per 128-row chunk), WS_U the gate inputs and fusion logits
+# of the unpooled rows, WS_GAMMA / WS_MID the per-chunk decays
+WS_POOLED, WS_QS, WS_KS, WS_V = 0, 1, 2, 3
+WS_O, WS_Y, WS_FUSION, WS_U, WS_GAMMA, WS_MID = 5, 6, 7, 8, 9, 10
 
 
 class Config(ctypes.Structure):

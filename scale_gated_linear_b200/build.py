@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmsgla.so")
-SOURCES = ["msgla_abi.cu", "k_gemm.cu", "k_gla.cu", "k_aux.cu", "k_decode.cu"]
+SOURCES = ["msgla_abi.cu", "k_gemm.cu", "k_gla.cu", "k_aux.cu", "k_pool.cu", "k_decode.cu"]
 HEADERS = ["msgla_internal.h", "sm100_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

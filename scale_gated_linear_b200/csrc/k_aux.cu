@@ -7,11 +7,11 @@
 //                     pool_rows_kernel and pool_rows_flat_kernel pool only (with
 //                     a scale-1 branch the fusion logits come from its
 //                     projection GEMM).
-//   gate_kernel       log alpha = logsigmoid(g W_g2^T + b_g) / normalizer (the
-//                     low-rank gate of Sec. 2.1), its cumulative sum b inside
-//                     each 128-row GLA chunk referenced to the chunk's 64th
-//                     row (m): Qs = q e^{b - m}, Ks = k e^{m - b}, and per chunk
-//                     gamma = e^{b_last - m}, mid = e^{m}.
+//   gate_kernel       the gate of Sec. 2.1 in the chunkwise GLA form: with b the
+//                     cumulative sum of log2 alpha over a 128-row chunk and m
+//                     its value at the chunk's row 63, the exponents d = b - m
+//                     per row and key channel (the projection scales q and k by
+//                     2^{+-d}), and per chunk gamma = 2^{b_127 - m}, mid = 2^{m}.
 //   head_norm_kernel  optional per-branch normalisation (Sec. 3.2), read as an
 //                     RMS norm of each head's GLA output row, in place.
 //   hold_fuse_kernel  O_t = sum_s w_{t,s} Y^(s)_{floor((t+1)/s)-1} (Sec. 3.3,
@@ -476,307 +476,189 @@ __global__ void __launch_bounds__(256) head_norm_kernel(const HeadNormParams p) 
   if (bad) atomicCAS(p.err, 0, kDevRange);
 }
 
-constexpr int kGateThreads = 256;
-constexpr int kGateChannels = 128;  // key channels per CTA
-
-// 2^x by the hardware approximation (relative error about 2^-22, far below the
-// fp16 rounding of the scaled q and k it feeds)
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// log2(x) by the hardware approximation (absolute error about 2^-22 for x in (1, 2])
-__device__ __forceinline__ float lg2_approx(float x) {
-  float y;
-  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Accumulates a packed fp16 pair's exponents into `acc` so that bit 15 or bit 31
-// of acc ends up set iff some half seen was inf or nan (exponent all ones: adding
-// one to the exponent field then carries into that half's sign position).
-__device__ __forceinline__ void half2_track_nonfinite(uint32_t& acc, uint32_t h) {
-  acc |= (h & 0x7c007c00u) + 0x04000400u;
-}
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-
-// tf32 split of an fp32 value: hi has the top 10 mantissa bits, lo the rest.
-__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-  uint32_t h;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
-  float r = x - __uint_as_float(h);
-  uint32_t l;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(l) : "f"(r));
-  hi = h;
-  lo = l;
-}
-
-__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-// One CTA per (branch, batch, head, 64-row half of a 128-row GLA chunk, 128 key
-// channels), 256 threads.
-//  0. cp.async stages the half chunk's low-rank gate rows g [64 x RP] and its q
-//     and k rows [64 x 128] (fp16; the 16-byte chunks of a row are XOR-swizzled
-//     by (row / 4) mod 8 so that phase 2 reads them without bank conflicts).
-//  1. z = g W_g2^T for the 64 x 128 block on tensor cores (mma.sync m16n8k8 tf32;
-//     each operand split into tf32 hi + lo parts, three products, so z keeps
-//     fp32-level accuracy), then log alpha = logsigmoid(z + b_g) / normalizer,
-//     kept in base-2 units (times log2 e) in shared memory; rows past the end of
-//     the sequence get 0.
-//  2. Thread (channel group cg of 8 channels, row group rg of 4 rows): the
-//     cumulative sum of log alpha over its 4 rows, the exclusive prefix over the
-//     16 row groups by a 16-lane shuffle scan, and Qs = q 2^{b - m},
-//     Ks = k 2^{m - b} stored 16 bytes at a time. With b_loc the cumulative sum
-//     from the half's first row and T its total: in the first half b - m =
-//     b_loc - T, in the second half b - m = b_loc (m is the first half's total),
-//     so each half needs only its own rows. Per chunk: gamma = e^{b_last - m},
-//     mid = e^{m}.
-constexpr int kGateBlk = 36;  // floats per (channel group, row group) block of log alpha: 4 x 8 + 4 padding
-
-template <int RP>
-struct GateSmem {
-  static constexpr int kQK = 2 * kChunk * kGateChannels * 2;              // q, k rows (fp16)
-  static constexpr int kLA = (kGateChannels / 8) * (kChunk / 4) * kGateBlk * 4;
-  static constexpr int kGS = RP + 4;                                      // padded g row (floats)
-  static constexpr int kG = kChunk * kGS * 4;
-  static constexpr int kBytes = kQK + kLA + kG;
-};
-
-template <int RP>
-__global__ void __launch_bounds__(kGateThreads, 3) gate_kernel(const __grid_constant__ GateParams p) {
-  griddep_wait();
-  griddep_launch();
-  using L = GateSmem<RP>;
-  extern __shared__ __align__(16) uint8_t gate_smem[];
-  __half* qk_s = reinterpret_cast<__half*>(gate_smem);
-  float* la_s = reinterpret_cast<float*>(gate_smem + L::kQK);
-  float* g_s = reinterpret_cast<float*>(gate_smem + L::kQK + L::kLA);
-  const int dkp = p.dkp;
-  const int cblocks = dkp / kGateChannels;
-  int bi = 0;
-#pragma unroll 1
-  for (int j = 1; j < p.n_branches; ++j)
-    if (static_cast<int>(blockIdx.x) >= p.br[j].block_begin) bi = j;
-  const GateBranch& P = p.br[bi];
-  int local = blockIdx.x - P.block_begin;
-  const int cb = local % cblocks;
-  local /= cblocks;
-  const int hc = local % P.n_halves;
-  const int head = (local / P.n_halves) % P.heads;
-  const int b = local / (P.n_halves * P.heads);
-  const int ci = hc >> 1, second = hc & 1;
-  const int n_chunks = (P.n_halves + 1) >> 1;
-  const int t0 = hc * kChunk;
-  const int nrows = min(kChunk, P.rows - t0);
-  const int ldk = P.heads * dkp;
-  const int cbase = head * dkp + cb * kGateChannels;  // first channel of this CTA
-  const size_t row_base = static_cast<size_t>(b) * P.rows + t0;
-  const int tid = threadIdx.x;
-
-  // ---- phase 0: g rows (group 0), then q and k rows (group 1)
-  constexpr int kGChunks = kChunk * RP / 4;
-  for (int i = tid; i < kGChunks; i += kGateThreads) {
-    const int row = i / (RP / 4), seg = i % (RP / 4);
-    float* dst = g_s + row * L::kGS + seg * 4;
-    if (row < nrows)
-      cp_async16(dst, P.g + (row_base + row) * RP + seg * 4);
-    else
-      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-#pragma unroll
-  for (int it = 0; it < 2 * kChunk * 16 / kGateThreads; ++it) {
-    const int flat = tid + it * kGateThreads;
-    const int tsel = flat >> 10, row = (flat >> 4) & (kChunk - 1), seg = flat & 15;
-    if (row < nrows) {
-      const __half* src = (tsel ? P.k : P.q) + (row_base + row) * ldk + cbase + seg * 8;
-      cp_async16(qk_s + (tsel * kChunk + row) * kGateChannels + ((seg ^ ((row >> 2) & 7)) * 8), src);
-    }
-  }
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 1;" ::: "memory");
-  __syncthreads();
-
-  // ---- phase 1: z = g W^T on tensor cores. Warp w owns channels [16w, 16w+16)
-  // (two n8 tiles) for all 64 rows (four m16 tiles); K = RP in steps of 8.
-  {
-    const int warp = tid >> 5, lane = tid & 31;
-    const int gq = lane >> 2, tq = lane & 3;
-    float acc[4][2][4];
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-#pragma unroll
-    for (int k8 = 0; k8 < RP / 8; ++k8) {
-      // B fragments: W[channel][k]; b0 = (k = tq, n = gq), b1 = (k = tq + 4, n = gq)
-      uint32_t bh[2][2], bl[2][2];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const float* wr = P.Wg2 + static_cast<size_t>(cbase + warp * 16 + nt * 8 + gq) * RP + k8 * 8;
-        split_tf32(__ldg(wr + tq), bh[nt][0], bl[nt][0]);
-        split_tf32(__ldg(wr + tq + 4), bh[nt][1], bl[nt][1]);
-      }
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        // A fragments: g[row][k]; a0 = (gq, tq), a1 = (gq + 8, tq), a2 = (gq, tq + 4), a3 = (gq + 8, tq + 4)
-        const float* g0 = g_s + (mt * 16 + gq) * L::kGS + k8 * 8;
-        const float* g1 = g0 + 8 * L::kGS;
-        uint32_t ah[4], al[4];
-        split_tf32(g0[tq], ah[0], al[0]);
-        split_tf32(g1[tq], ah[1], al[1]);
-        split_tf32(g0[tq + 4], ah[2], al[2]);
-        split_tf32(g1[tq + 4], ah[3], al[3]);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          mma_tf32(acc[mt][nt], al, bh[nt]);
-          mma_tf32(acc[mt][nt], ah, bl[nt]);
-          mma_tf32(acc[mt][nt], ah, bh[nt]);
-        }
-      }
-    }
-    // log alpha (base 2) into the blocked layout; D fragment: d0 = (gq, 2tq),
-    // d1 = (gq, 2tq+1), d2 = (gq+8, 2tq), d3 = (gq+8, 2tq+1). With z2 = z log2(e),
-    // log2 alpha = (min(z2, 0) - log2(1 + 2^{-|z2|})) / normalizer, the base-2
-    // form of logsigmoid(z) / normalizer (the log argument lies in (1, 2]).
-    constexpr float kLog2e = 1.4426950408889634f;
-    const float inv_norm = p.inv_normalizer;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int chl = warp * 16 + nt * 8 + 2 * tq;
-      const float bias0 = __ldg(P.bg + cbase + chl) * kLog2e, bias1 = __ldg(P.bg + cbase + chl + 1) * kLog2e;
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int row = mt * 16 + gq + ((e & 2) ? 8 : 0), ch = chl + (e & 1);
-          const float z2 = fmaf(acc[mt][nt][e], kLog2e, (e & 1) ? bias1 : bias0);
-          const float la = (fminf(z2, 0.f) - lg2_approx(1.f + ex2_approx(-fabsf(z2)))) * inv_norm;
-          la_s[((ch >> 3) * (kChunk / 4) + (row >> 2)) * kGateBlk + (row & 3) * 8 + (ch & 7)] = la;
-        }
-      }
-    }
-    if (nrows < kChunk) {
-      // rows past the end of the sequence contribute nothing to the sums
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int chl = warp * 16 + nt * 8 + 2 * tq;
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int row = mt * 16 + gq + ((e & 2) ? 8 : 0), ch = chl + (e & 1);
-            if (row >= nrows) la_s[((ch >> 3) * (kChunk / 4) + (row >> 2)) * kGateBlk + (row & 3) * 8 + (ch & 7)] = 0.f;
-          }
-      }
-    }
-  }
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
-
-  // ---- phase 2: warp w holds channel groups 2w (lanes 0-15) and 2w+1 (lanes
-  // 16-31); lane rg of a 16-lane segment holds rows [4rg, 4rg+4).
-  const int lane = tid & 31;
-  const int cg = 2 * (tid >> 5) + (lane >> 4), rg = lane & 15;
-  const float* blk = la_s + (cg * (kChunk / 4) + rg) * kGateBlk;
-  float c[4][8];
-  float run[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) run[e] = 0.f;
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const float4 x0 = *reinterpret_cast<const float4*>(blk + r * 8);
-    const float4 x1 = *reinterpret_cast<const float4*>(blk + r * 8 + 4);
-    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      run[e] += x[e];
-      c[r][e] = run[e];
-    }
-  }
-  // exclusive prefix over the row groups before this one, and the half's total
-  float pre[8], tot[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    float v = run[e];
-#pragma unroll
-    for (int off = 1; off < 16; off <<= 1) {
-      const float u = __shfl_up_sync(0xffffffffu, v, off, 16);
-      if (rg >= off) v += u;
-    }
-    pre[e] = v - run[e];
-    tot[e] = __shfl_sync(0xffffffffu, v, 15, 16);
-  }
-  // reference: b - m = b_loc - T in the first half, b_loc in the second
-#pragma unroll
-  for (int e = 0; e < 8; ++e) pre[e] -= second ? 0.f : tot[e];
-
-  // A scaled value can leave the fp16 range only where its factor exceeds 1: b
-  // does not increase along the chunk (log alpha <= 0), so in the first half
-  // (rows up to m's) Qs = q 2^{b-m} can grow and Ks cannot, and in the second
-  // half the reverse. Only the growing side is checked.
-  uint32_t over = 0;
-  const int sw = rg & 7;  // (row >> 2) & 7 for all four rows of this thread
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int row = 4 * rg + r;
-    if (row >= nrows) break;
-    const uint4 qv = *reinterpret_cast<const uint4*>(qk_s + row * kGateChannels + ((cg ^ sw) * 8));
-    const uint4 kv = *reinterpret_cast<const uint4*>(qk_s + (kChunk + row) * kGateChannels + ((cg ^ sw) * 8));
-    const __half2* qh = reinterpret_cast<const __half2*>(&qv);
-    const __half2* kh = reinterpret_cast<const __half2*>(&kv);
-    uint4 qo, ko;
-    uint32_t* qw = reinterpret_cast<uint32_t*>(&qo);
-    uint32_t* kw = reinterpret_cast<uint32_t*>(&ko);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float b0 = pre[2 * e] + c[r][2 * e], b1 = pre[2 * e + 1] + c[r][2 * e + 1];
-      const float2 qf = __half22float2(qh[e]), kf = __half22float2(kh[e]);
-      qw[e] = pack_half2(qf.x * ex2_approx(b0), qf.y * ex2_approx(b1));
-      kw[e] = pack_half2(kf.x * ex2_approx(-b0), kf.y * ex2_approx(-b1));
-      half2_track_nonfinite(over, second ? kw[e] : qw[e]);
-    }
-    const size_t go = (row_base + row) * ldk + cbase + cg * 8;
-    *reinterpret_cast<uint4*>(P.qs + go) = qo;
-    *reinterpret_cast<uint4*>(P.ks + go) = ko;
-  }
-  if (over & 0x80008000u) atomicCAS(p.err, 0, kDevRange);
-  if (rg == 15) {
-    const size_t gi = (static_cast<size_t>(b) * n_chunks + ci) * ldk + cbase + cg * 8;
-    float* dst = second ? P.gamma : P.mid;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) dst[gi + e] = exp2f(tot[e]);
-    if (!second && hc + 1 >= P.n_halves)  // chunk without a second half: b_last = m
-#pragma unroll
-      for (int e = 0; e < 8; ++e) P.gamma[gi + e] = 1.f;
-  }
-}
-
-template <int RP>
-cudaError_t launch_gate_t(const GateParams& p, cudaStream_t st) {
-  const int smem = GateSmem<RP>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(gate_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(gate_kernel<RP>, dim3(p.total_blocks), dim3(kGateThreads), smem, st, p);
-}
-
 // O_t = sum_s w_{t,s} Y^(s)_{floor((t+1)/s)-1} (Eq. (11) with the causal hold of
 // Sec. 3.3) when no branch has scale 1. One CTA per (sequence, tile of
 // kHoldRows rows, block of up to 256 column groups): thread (r, cg) takes 8
 // columns of rows t0 + r, t0 + r + R, ...; no division in the loop (the held
 // row index is a shift for power-of-two scales).
+// Packed fp32 pairs (two IEEE fp32 operations per instruction, round to nearest).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// One item per (branch, sequence, half of a 128-row chunk, block of 256 key
+// channels), a CTA of 128 threads; thread t owns channels c0 + 2t, c0 + 2t + 1.
+//  1. The half's 64 gate inputs g (rank RP) go to shared memory: a scale-1
+//     row's are its columns of U, a coarse row's the mean of its block's valid
+//     unpooled rows' columns (Eq. (8), pooling being linear).
+//  2. Per row z2 = log2(e) (g W_g2[c]^T + b_g[c]) (packed fp32 pairs over the
+//     rank) and l = log2 alpha = (min(z2, 0) - log2(1 + 2^{-|z2|})) /
+//     normalizer: logsigmoid in base 2 with the hardware 2^x and log2
+//     approximations (relative errors near 2^-22).
+//  3. The first half walks its rows backwards: d(r) = b(r) - m = -(sum of l over
+//     rows r+1..63), and its total is m (mid = 2^m); the second half walks
+//     forwards: d(r) = sum of l over rows 64..r, its total giving gamma =
+//     2^{b_127 - m}. The projection GEMM scales q and k of the row by 2^{+-d}.
+//     Rows past the sequence's end add nothing (a chunk without a second half
+//     gets gamma = 1).
+constexpr int kGateThreads = 128;
+constexpr int kGateRows = 64;
+constexpr int kGateChannels = 2 * kGateThreads;
+
+template <int RP>
+__device__ __forceinline__ void gate_item(const GateParams& p, int item, float* gs);
+
+// Persistent over the items (a grid of whole waves): CTA x takes items x,
+// x + gridDim.x, ...
+template <int RP>
+__global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constant__ GateParams p) {
+  __shared__ __align__(16) float gs[kGateRows * RP];
+  griddep_wait();
+  griddep_launch();
+#pragma unroll 1
+  for (int item = blockIdx.x; item < p.total_blocks; item += gridDim.x) {
+    gate_item<RP>(p, item, gs);
+    __syncthreads();  // the next item overwrites gs
+  }
+}
+
+template <int RP>
+__device__ __forceinline__ void gate_item(const GateParams& p, int item, float* gs) {
+  int bi = 0;
+#pragma unroll 1
+  for (int j = 1; j < p.n_branches; ++j)
+    if (item >= p.br[j].block_begin) bi = j;
+  const GateBranch& P = p.br[bi];
+  int local = item - P.block_begin;
+  const int cblk = local % P.cblocks;
+  local /= P.cblocks;
+  const int half = local & 1;
+  local >>= 1;
+  const int chunk = local % P.n_chunks;
+  const int b = local / P.n_chunks;
+  const int r0 = chunk * 2 * kGateRows + half * kGateRows;  // first pooled row of the half
+  const int nr = min(kGateRows, P.rows - r0);               // its rows inside the sequence
+  const int tid = threadIdx.x;
+  const size_t ubase = static_cast<size_t>(b) * p.L;
+  // 1. gate inputs of the half's rows
+  for (int idx = tid; idx < kGateRows * RP / 4; idx += kGateThreads) {
+    const int row = idx / (RP / 4), k4 = idx % (RP / 4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row < nr) {
+      const int t0 = (r0 + row) * P.scale, t1 = min(t0 + P.scale, p.L);
+      float cnt = 0.f;
+      for (int t = t0; t < t1; ++t) {
+        if (p.mask && !__ldg(p.mask + ubase + t)) continue;
+        const float4 x = __ldg(reinterpret_cast<const float4*>(p.u + (ubase + t) * p.ldu + P.ucol) + k4);
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
+        cnt += 1.f;
+      }
+      if (P.scale > 1) {
+        const float inv = 1.f / fmaxf(cnt, 1.f);
+        acc.x *= inv;
+        acc.y *= inv;
+        acc.z *= inv;
+        acc.w *= inv;
+      }
+    }
+    *reinterpret_cast<float4*>(gs + row * RP + 4 * k4) = acc;
+  }
+  __syncthreads();
+  const int c0 = cblk * kGateChannels + 2 * tid;
+  if (c0 >= P.ldk || nr <= 0) return;
+  // 2. this thread's two rows of W_g2 and biases, in log2 units, as pairs over the rank
+  constexpr float kLog2e = 1.4426950408889634f;
+  uint64_t w0[RP / 2], w1[RP / 2];
+  {
+    const float4* a = reinterpret_cast<const float4*>(P.Wg2 + static_cast<size_t>(c0) * RP);
+#pragma unroll
+    for (int j = 0; j < RP / 4; ++j) {
+      const float4 x = __ldg(a + j), y = __ldg(a + RP / 4 + j);
+      w0[2 * j] = f2_pack(x.x * kLog2e, x.y * kLog2e);
+      w0[2 * j + 1] = f2_pack(x.z * kLog2e, x.w * kLog2e);
+      w1[2 * j] = f2_pack(y.x * kLog2e, y.y * kLog2e);
+      w1[2 * j + 1] = f2_pack(y.z * kLog2e, y.w * kLog2e);
+    }
+  }
+  const float2 bb = __ldg(reinterpret_cast<const float2*>(P.bg + c0));
+  const float bias0 = bb.x * kLog2e, bias1 = bb.y * kLog2e;
+  const float inv_norm = p.inv_normalizer;
+  // log2 alpha of row r for both channels (two packed partial sums per channel)
+  auto log2_alpha = [&](const float* g_row, float& l0, float& l1) {
+    const uint64_t zero = f2_pack(0.f, 0.f);
+    uint64_t a0 = zero, b0 = zero, a1 = zero, b1 = zero;
+    const float4* g4 = reinterpret_cast<const float4*>(g_row);
+#pragma unroll
+    for (int j = 0; j < RP / 4; ++j) {
+      const float4 g = g4[j];
+      const uint64_t g01 = f2_pack(g.x, g.y), g23 = f2_pack(g.z, g.w);
+      a0 = f2_fma(g01, w0[2 * j], a0);
+      b0 = f2_fma(g23, w0[2 * j + 1], b0);
+      a1 = f2_fma(g01, w1[2 * j], a1);
+      b1 = f2_fma(g23, w1[2 * j + 1], b1);
+    }
+    const float2 pa0 = f2_unpack(a0), pb0 = f2_unpack(b0), pa1 = f2_unpack(a1), pb1 = f2_unpack(b1);
+    const float z0 = bias0 + ((pa0.x + pa0.y) + (pb0.x + pb0.y));
+    const float z1 = bias1 + ((pa1.x + pa1.y) + (pb1.x + pb1.y));
+    l0 = fminf(z0, 0.f) - lg2_approx(1.f + ex2_approx(-fabsf(z0)));
+    l1 = fminf(z1, 0.f) - lg2_approx(1.f + ex2_approx(-fabsf(z1)));
+  };
+  // Rows go in batches of kBatch, walked by a pointer stepping one row (backwards
+  // in the first half): first the batch's log2 alpha (independent of each
+  // other), then in row order d (first half: the sum of the rows after it,
+  // negated, taken before its own l is added; second half: the running sum
+  // including l), stored as soon as it is known.
+  constexpr int kBatch = 8;
+  const long long step = (half == 0 ? -1 : 1) * static_cast<long long>(P.ldk / 2);
+  const int first = half == 0 ? nr - 1 : 0;
+  float2* dp = reinterpret_cast<float2*>(P.d + (static_cast<size_t>(b) * P.rows + r0 + first) * P.ldk + c0);
+  const float* gp = gs + first * RP;
+  const int gstep = half == 0 ? -RP : RP;
+  float acc0 = 0.f, acc1 = 0.f;
+  const float sgn = half == 0 ? -inv_norm : inv_norm;
+#pragma unroll 1
+  for (int r = 0; r < nr; r += kBatch) {
+    const int n = min(kBatch, nr - r);
+    float l0[kBatch], l1[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i)
+      if (i < n) log2_alpha(gp + i * gstep, l0[i], l1[i]);
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      if (i >= n) break;
+      const float a0 = acc0 + l0[i], a1 = acc1 + l1[i];
+      dp[i * step] = make_float2((half == 0 ? acc0 : a0) * sgn, (half == 0 ? acc1 : a1) * sgn);
+      acc0 = a0;
+      acc1 = a1;
+    }
+    dp += kBatch * step;
+    gp += kBatch * gstep;
+  }
+  const size_t gi = (static_cast<size_t>(b) * P.n_chunks + chunk) * P.ldk + c0;
+  if (half == 0) {
+    *reinterpret_cast<float2*>(P.mid + gi) = make_float2(ex2_approx(acc0 * inv_norm), ex2_approx(acc1 * inv_norm));
+    if (P.rows - r0 <= kGateRows)  // no second half: b_127 = m
+      *reinterpret_cast<float2*>(P.gamma + gi) = make_float2(1.f, 1.f);
+  } else {
+    *reinterpret_cast<float2*>(P.gamma + gi) = make_float2(ex2_approx(acc0 * inv_norm), ex2_approx(acc1 * inv_norm));
+  }
+}
+
 constexpr int kHoldRows = 32;
 __global__ void __launch_bounds__(256) hold_fuse_kernel(const HoldFuseParams p, int CG, int R) {
   griddep_wait();
@@ -905,10 +787,23 @@ cudaError_t launch_head_norm(const HeadNormParams& p, cudaStream_t st) {
   return launch_pdl(head_norm_kernel, dim3(static_cast<unsigned>((p.total_warps + 7) / 8)), dim3(256), 0, st, p);
 }
 
+
+// whole waves of resident CTAs, no more than there are items
+template <int RP>
+cudaError_t launch_gate_t(const GateParams& p, cudaStream_t st) {
+  static int per_sm = 0;
+  if (per_sm == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gate_kernel<RP>, kGateThreads, 0) !=
+                          cudaSuccess || per_sm < 1))
+    per_sm = 1;
+  const int grid = std::min(p.total_blocks, per_sm * sm_count());
+  return launch_pdl(gate_kernel<RP>, dim3(grid), dim3(kGateThreads), 0, st, p);
+}
+
 cudaError_t launch_gate(const GateParams& p, cudaStream_t st) {
   if (p.total_blocks <= 0) return cudaSuccess;
-  if (p.dkp % kGateChannels) return cudaErrorInvalidValue;
-  return p.rp == 16 ? launch_gate_t<16>(p, st) : launch_gate_t<32>(p, st);
+  if (p.rp == 16) return launch_gate_t<16>(p, st);
+  if (p.rp == 32) return launch_gate_t<32>(p, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_hold_fuse(const HoldFuseParams& p, cudaStream_t st) {

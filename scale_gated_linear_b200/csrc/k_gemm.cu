@@ -20,6 +20,12 @@
 //   kEpiFuse      the scale-1 branch's Y^(1) fused with the causal hold of the
 //                 coarse branches and the fusion softmax weights (Eq. (11)):
 //                 O_t = w_{t,1} Y^(1)_t + sum_s w_{t,s} Y^(s)_{floor((t+1)/s)-1}
+//   kEpiProjGate  the forward's projection: q|k tiles pair W_q and W_k rows of the
+//                 same 128 key channels and leave as the decay-scaled Qs = q 2^d,
+//                 Ks = k 2^-d of the chunkwise GLA (d: the gate exponents of
+//                 Sec. 2.1, launch_gate); v tiles leave as fp16
+//   kEpiStoreF32  the low-rank gate inputs and fusion logits of the unpooled rows
+//                 (fp32), optionally with the fusion weights of Eq. (10)
 #include "msgla_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -58,8 +64,12 @@ __device__ __forceinline__ void add_scaled_f16x32(float (&acc)[32], const __half
   }
 }
 
+// n0: the tile's first output column (for a q|k tile of kEpiProjGate its first
+// key channel, for its v tiles the first v column); brow0 / brow1: the first B
+// row of the tile's column halves (CTA rank 0 / 1 of a pair, or the two
+// 128-row B loads of a single-CTA 256-column tile).
 struct TileCoord {
-  int task, b, m0, n0, n_eff, kblocks;
+  int task, b, m0, n0, n_eff, kblocks, qk, brow0, brow1;
 };
 
 __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int tile, int bn, int bm = kGemmBM) {
@@ -75,10 +85,30 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int tile, 
   c.task = ti;
   c.b = local / (T.n_tiles * T.m_tiles);
   c.m0 = m_tile * bm;
-  c.n0 = n_tile * bn;
-  const int n_rem = T.N - c.n0;
-  c.n_eff = n_rem >= bn ? bn : ((n_rem + 15) / 16) * 16;
   c.kblocks = (T.K + kGemmBK - 1) / kGemmBK;
+  c.qk = 0;
+  if (T.epi == kEpiProjGate && n_tile < T.n_qk) {
+    // 128 key channels of one head: W_q rows, then W_k rows of the same channels
+    const int per_head = T.dkp / 128;
+    c.qk = 1;
+    c.n0 = (n_tile / per_head) * T.dkp + (n_tile % per_head) * 128;
+    c.n_eff = 256;
+    c.brow0 = c.n0;
+    c.brow1 = T.nq + c.n0;
+    return c;
+  }
+  int n_cols = T.N, b_first = 0;
+  if (T.epi == kEpiProjGate) {  // v tiles
+    c.n0 = (n_tile - T.n_qk) * bn;
+    n_cols = T.nv;
+    b_first = T.nq + T.nk;
+  } else {
+    c.n0 = n_tile * bn;
+  }
+  const int n_rem = n_cols - c.n0;
+  c.n_eff = n_rem >= bn ? bn : ((n_rem + 15) / 16) * 16;
+  c.brow0 = b_first + c.n0;
+  c.brow1 = c.brow0 + (c.n_eff >> 1);
   return c;
 }
 
@@ -87,7 +117,7 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int tile, 
 // hides behind the MMAs.
 __device__ __forceinline__ bool row_is_padded(const GemmParams& p, const TileCoord& tc, int quad, int lane) {
   const GemmTask& T = p.task[tc.task];
-  if (T.epi != kEpiProj || !T.mask) return false;
+  if ((T.epi != kEpiProj && T.epi != kEpiProjGate) || !T.mask) return false;
   const int row = tc.m0 + quad * 32 + lane;
   return row < T.rows && !__ldg(T.mask + static_cast<size_t>(tc.b) * T.rows + row);
 }
@@ -238,7 +268,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, const TileCoo
       d1[j] = base1 ? __ldg(base1 + (c0 >> 3) + j) : make_uint4(0, 0, 0, 0);
     }
   };
-  const int n_f16 = T.epi == kEpiProj ? T.nq + T.nk + T.nv : T.N;
+  const int n_f16 = T.epi == kEpiProj ? T.nq + T.nk + T.nv : T.epi == kEpiProjGate ? T.nv : T.N;
   // one 32-column chunk (tile columns [c0, c0 + 32), values v); `half` places it
   // in the current staging buffer, `last` = no chunk of this tile follows
   auto chunk = [&](int c0, uint32_t (&v)[32], int half, bool last) __attribute__((always_inline)) {
@@ -274,7 +304,13 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, const TileCoo
     const CUtensorMap* map = &T.tmOut[0];
     int dcol = col64;
     uint32_t pk[16];
-    if (T.epi == kEpiProj) {
+    if (T.epi == kEpiProjGate) {  // a v tile
+      map = &T.tmOut[2];
+      if (padded)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0u;
+      pack_f16x32(pk, v);
+    } else if (T.epi == kEpiProj) {
       if (col64 >= T.nq + T.nk) {
         map = &T.tmOut[2];
         dcol = col64 - T.nq - T.nk;
@@ -383,6 +419,56 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, const TileCoo
   return true;
 }
 
+// Columns [c_lo, c_hi) of a kEpiStoreF32 tile: fp32 rows stored directly (the
+// gate inputs and fusion logits, 64 to 272 columns per row); the thread holding
+// column 0 of a row also forms the fusion weights w = softmax(z + b_fuse) from
+// the logits in columns 0..n_scales-1 when T.w is set (Eq. (10)).
+__device__ __forceinline__ void epilogue_f32(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
+                                             int lane, int c_lo, int c_hi) {
+  const GemmTask& T = p.task[tc.task];
+  const int row = tc.m0 + quad * 32 + lane;
+  const bool valid = row < T.rows;
+  const size_t grow = static_cast<size_t>(tc.b) * T.rows + row;
+#pragma unroll 1
+  for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(tmem_addr(tacc, quad * 32, c0), v);
+    tmem_wait_ld(v);
+    if (!valid) continue;
+    const int col = tc.n0 + c0;
+    if (col == 0 && T.w) {
+      float zz[kMaxScales];
+      float zmax = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kMaxScales; ++j) {
+        zz[j] = j < T.n_scales ? __uint_as_float(v[j]) + __ldg(T.bfuse + j) : -INFINITY;
+        zmax = fmaxf(zmax, zz[j]);
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxScales; ++j) {
+        zz[j] = j < T.n_scales ? __expf(zz[j] - zmax) : 0.f;
+        sum += zz[j];
+      }
+      const float inv = 1.f / sum;
+#pragma unroll
+      for (int j = 0; j < kMaxScales; ++j)
+        if (j < T.n_scales) T.w[grow * T.n_scales + j] = zz[j] * inv;
+    }
+    float* dst = T.f32 + grow * T.ldf + col;
+    if (col + 32 <= T.N) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        reinterpret_cast<float4*>(dst)[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                        __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col + j < T.N) dst[j] = __uint_as_float(v[j]);
+    }
+  }
+}
+
 // Two epilogue warps share each TMEM lane quadrant and split the tile's columns
 // at a multiple of 64 (one staging step).
 __device__ __forceinline__ void epi_columns(int warp, int n_eff, int& lo, int& hi) {
@@ -392,10 +478,97 @@ __device__ __forceinline__ void epi_columns(int warp, int n_eff, int& lo, int& h
   hi = second ? n_eff : mid;
 }
 
+// ---------------------------------------------------------------- gated projection
+// Pulls this thread's 64 gate exponents of a q|k tile (two 128-byte lines) into
+// L2 while the tile's accumulator is still being computed.
+__device__ __forceinline__ void prefetch_gate_exponents(const GemmParams& p, const TileCoord& tc, int quad, int lane,
+                                                        int ch) {
+  const GemmTask& T = p.task[tc.task];
+  const int row = tc.m0 + quad * 32 + lane;
+  if (row >= T.rows) return;
+  const float* a = T.gd + (static_cast<size_t>(tc.b) * T.rows + row) * T.nq + tc.n0 + 64 * ch;
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(a + 32));
+}
+
+// Epilogue of a q|k tile of the gated projection (kEpiProjGate; MS-GLA reading
+// notes, Sec. 2.1). The accumulator holds q (columns 0..127) and k (128..255) of
+// the 128 key channels c0.. of one head for the CTA's 128 rows, which are one
+// 128-row chunk of the GLA kernel. The thread of chunk row r and channel half ch
+// takes channels c0 + 64 ch .., 32 at a time: with the gate exponents d = b - m
+// of its row (b the cumulative sum of log2 alpha over the chunk's rows, m its
+// value at row 63; launch_gate) it stores Qs = q 2^d and Ks = k 2^-d (fp16), the
+// operands of the chunkwise GLA kernel, as two 32 x 32 boxes through the warp's
+// staging buffer (Qs in its first 2 KB, Ks in the second; 64-byte swizzle, maps
+// tmQK). Only the side whose factor can exceed 1 is checked for the fp16 range
+// (b does not increase along the chunk: Qs in rows 0..63, Ks in rows 64..127);
+// an overflow latches kDevRange.
+__device__ __forceinline__ void epilogue_qk(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
+                                            int lane, int ch, bool padded, const Stager& stg) {
+  const GemmTask& T = p.task[tc.task];
+  const int lrow = quad * 32 + lane;
+  const int row = tc.m0 + lrow;
+  const bool valid = row < T.rows;
+  const int grow_side = lrow < 64 ? 0 : 1;
+  const float4* gd = reinterpret_cast<const float4*>(T.gd + (static_cast<size_t>(tc.b) * T.rows + row) * T.nq +
+                                                     tc.n0 + 64 * ch);
+  uint8_t* buf = stg.at(0);
+  uint32_t over = 0;
+#pragma unroll
+  for (int grp = 0; grp < 2; ++grp) {
+    float4 dn[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dn[j] = valid ? __ldg(gd + 8 * grp + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float d[32];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      d[4 * j] = dn[j].x;
+      d[4 * j + 1] = dn[j].y;
+      d[4 * j + 2] = dn[j].z;
+      d[4 * j + 3] = dn[j].w;
+    }
+    const int cb = tc.n0 + 64 * ch + 32 * grp;  // first key channel of this group
+    stg.acquire();  // the previous group's stores have read the buffer
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      uint32_t a[32];
+      tmem_ld32(tmem_addr(tacc, quad * 32, which * 128 + 64 * ch + 32 * grp), a);
+      tmem_wait_ld(a);
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float d0 = d[2 * e], d1 = d[2 * e + 1];
+        const float s0 = ex2_approx(which ? -d0 : d0), s1 = ex2_approx(which ? -d1 : d1);
+        const float v0 = padded ? 0.f : __uint_as_float(a[2 * e]) * s0;
+        const float v1 = padded ? 0.f : __uint_as_float(a[2 * e + 1]) * s1;
+        pk[e] = pack_half2(v0, v1);
+        if (which == grow_side) half2_track_nonfinite(over, pk[e]);
+      }
+      // 64-byte rows, 16-byte chunk j of row r at chunk j ^ ((r >> 1) & 3)
+      uint8_t* rowp = buf + which * 2048 + lane * 64;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        st_shared_v4(smem_u32(rowp + ((j ^ ((lane >> 1) & 3)) << 4)), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2],
+                     pk[4 * j + 3]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(&T.tmQK[0], buf, cb, tc.m0 + quad * 32, tc.b);
+      tma_store_3d(&T.tmQK[1], buf + 2048, cb, tc.m0 + quad * 32, tc.b);
+      bulk_commit();
+    }
+  }
+  if (over & 0x80008000u) atomicCAS(p.err, 0, kDevRange);
+}
+
 // Prefetch the output tensor maps of every task (epilogue warps).
 __device__ __forceinline__ void prefetch_out_maps(const GemmParams& p) {
-  for (int t = 0; t < p.n_tasks; ++t)
+  for (int t = 0; t < p.n_tasks; ++t) {
     for (int m = 0; m < 3; ++m) prefetch_tmap(&p.task[t].tmOut[m]);
+    if (p.task[t].epi == kEpiProjGate)
+      for (int m = 0; m < 2; ++m) prefetch_tmap(&p.task[t].tmQK[m]);
+  }
 }
 
 // Producer side of a per-task input dependency (GemmTask::dep): before the first
@@ -471,7 +644,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         // B tensor maps carry a 128-row box: BN / 128 loads fill the stage's B slot
 #pragma unroll
         for (int h = 0; h < BN / 128; ++h)
-          tma_load_2d(&T.tmB, &full_bar[s], sb + h * 128 * kGemmBK * 2, kb * kGemmBK, tc.n0 + h * 128);
+          tma_load_2d(&T.tmB, &full_bar[s], sb + h * 128 * kGemmBK * 2, kb * kGemmBK,
+                      h == 0 ? tc.brow0 : (tc.qk ? tc.brow1 : tc.brow0 + h * 128));
       }
     }
   } else if (warp == 1 && lane == 0) {
@@ -517,9 +691,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       epi_columns(warp, tc.n_eff, lo, hi);
       FuseW fw;
       fuse_weights(p, tc, quad, lane, lo, fw);
+      if (tc.qk) prefetch_gate_exponents(p, tc, quad, lane, (warp - 2) >= 4 ? 1 : 0);
       if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      epilogue_tile(p, tc, tmem + buf * BN, quad, lane, lo, hi, padded, stg, sel, fw);
+      if (tc.qk) {
+        epilogue_qk(p, tc, tmem + buf * BN, quad, lane, (warp - 2) >= 4 ? 1 : 0, padded, stg);
+      } else if (p.task[tc.task].epi == kEpiStoreF32) {
+        epilogue_f32(p, tc, tmem + buf * BN, quad, lane, lo, hi);
+      } else {
+        epilogue_tile(p, tc, tmem + buf * BN, quad, lane, lo, hi, padded, stg, sel, fw);
+      }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
     }
@@ -560,7 +741,7 @@ struct PairLayout {
   static constexpr int kStagingBytesT = 8 * kStagerBytes;
   static constexpr int kHeldOffset = kStagingOffset + kStagingBytesT;
   static constexpr int kBarOffset = kHeldOffset + (kHeld ? kHeldBytes : 0);
-  static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
+  static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + 1024 B alignment slack
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -684,7 +865,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
       const GemmTask& T = p.task[tc.task];
       if (!task_ready(T, tc.task, ready, abort_flag, p.err)) break;
       const int arow = tc.m0 + 128 * static_cast<int>(rank);
-      const int brow = tc.n0 + static_cast<int>(rank) * (tc.n_eff >> 1);
+      const int brow = rank ? tc.brow1 : tc.brow0;
       for (int kb = 0; kb < tc.kblocks; ++kb, ++kbg) {
         const uint32_t s = kbg % kStagesT;
         if (kbg >= kStagesT && !mbar_wait(&empty_bar[s], ((kbg / kStagesT) - 1) & 1, abort_flag, p.err)) {
@@ -777,6 +958,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
       epi_columns(warp, tc.n_eff, lo, hi);
       FuseW fw;
       fuse_weights(p, tc, quad, lane, lo, fw);
+      if (!kHeld && tc.qk) prefetch_gate_exponents(p, tc, quad, lane, (warp - 2) >= 4 ? 1 : 0);
       if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
       if (kHeld) {
@@ -797,6 +979,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
         h.parity = it & 1;
         h.abort_flag = abort_flag;
         if (!epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel, fw, &h)) break;
+      } else if (!kHeld && tc.qk) {
+        epilogue_qk(p, tc, tmem + buf * kPairBN, quad, lane, (warp - 2) >= 4 ? 1 : 0, padded, stg);
+      } else if (p.task[tc.task].epi == kEpiStoreF32) {
+        epilogue_f32(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi);
       } else {
         epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel, fw);
       }
@@ -865,6 +1051,7 @@ int max_active_pairs() {
 
 cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pairs) {
   if (p.total_tiles <= 0) return cudaSuccess;
+  if (bn != 256) return cudaErrorInvalidValue;
   // the fused output launch with one or two coarse branches stages their held
   // rows in shared memory (the caller encodes tmOut[1 + c] for them)
   // (and only with full 256-column tiles: every 64-column box of held rows then
@@ -872,7 +1059,7 @@ cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pa
   const bool held = p.n_tasks == 1 && p.task[0].epi == kEpiFuse && p.task[0].n_coarse >= 1 &&
                     p.task[0].n_coarse <= 2 && p.task[0].N % kPairBN == 0 &&
                     held_rows_fit(p.task[0].coarse_scale, p.task[0].n_coarse);
-  int pairs = (bn != 256) ? 0 : held ? max_active_pairs<true>() : max_active_pairs<false>();
+  int pairs = held ? max_active_pairs<true>() : max_active_pairs<false>();
   if (max_pairs > 0 && pairs > max_pairs) pairs = max_pairs;
   if (pairs > 0) {
     // re-tile every task in 256 x 256 pair tiles
@@ -884,7 +1071,7 @@ cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pa
       const int end = (t + 1 < p.n_tasks) ? p.task[t + 1].tile_begin : p.total_tiles;
       const int batches = (end - p.task[t].tile_begin) / (p.task[t].m_tiles * p.task[t].n_tiles);
       T.m_tiles = (T.rows + kPairBM - 1) / kPairBM;
-      T.n_tiles = (T.N + kPairBN - 1) / kPairBN;
+      T.n_tiles = T.epi == kEpiProjGate ? T.n_qk + (T.nv + kPairBN - 1) / kPairBN : (T.N + kPairBN - 1) / kPairBN;
       T.tile_begin = tiles;
       tiles += batches * T.m_tiles * T.n_tiles;
     }
@@ -898,20 +1085,11 @@ cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pa
   }
   int grid = p.total_tiles < sm_count() ? p.total_tiles : sm_count();
   if (max_pairs > 0 && grid > 2 * max_pairs) grid = 2 * max_pairs;
-  if (bn == 256) {
-    const int smem = GemmLayout<256>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(gemm_kernel<256>, dim3(grid), dim3(kThreads), smem, st, p);
-  } else if (bn == 128) {
-    const int smem = GemmLayout<128>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(gemm_kernel<128>, dim3(grid), dim3(kThreads), smem, st, p);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  const int smem = GemmLayout<256>::kSmemBytes;
+  auto kern = gemm_kernel<256>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, p);
 }
 
 }  // namespace msgla

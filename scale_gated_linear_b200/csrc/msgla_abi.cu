@@ -106,6 +106,20 @@ bool encode_out_3d(CUtensorMap* m, bool bf16, void* base, uint64_t inner, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp16 [batch][rows][inner] with a {32, 32, 1} box and 64B swizzle (32-column
+// TMA stores of the gated projection's Qs and Ks).
+bool encode_out_3d_32(CUtensorMap* m, void* base, uint64_t inner, uint64_t rows, uint64_t batch) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DeviceGuard {
   int prev = -1;
   bool ok = false;
@@ -137,6 +151,11 @@ struct msgla_handle {
   int sm_count;  // streaming multiprocessors of the device
   int nzp, ldz;  // fusion-logit rows in the scale-1 packed weights (16) and z row stride
   Branch br[MSGLA_MAX_SCALES];
+  // gate inputs and fusion logits of the unpooled rows in one GEMM:
+  // U = X Wu^T with Wu [ldu, d] bf16 = [W_fuse (rows 0..n_scales-1, zero to 16);
+  // W_g1 of scale index j at rows 16 + j rp ..], ldu = 16 + n_scales rp
+  __nv_bfloat16* Wu;
+  int ldu;
   __nv_bfloat16* Wfuse;
   float* bfuse;
   int* d_err;  // device error word
@@ -159,13 +178,13 @@ struct Region {
   size_t off = 0, bytes = 0;
 };
 struct BranchWs {
-  int rows, n_chunks, n_halves, seg_chunks, n_segs;
+  int rows, n_chunks, seg_chunks, n_segs;
   Region seg_state, seg_decay;
-  Region Xp, q, k, qs, ks, v, g, gamma, mid, o, Y;
+  Region Xp, qs, ks, v, gd, gamma, mid, o, Y;
 };
 struct Workspace {
   BranchWs br[MSGLA_MAX_SCALES];
-  Region w, z;
+  Region w, u;
   size_t total = 0;
 };
 
@@ -210,17 +229,14 @@ Workspace layout(const msgla_handle* h, int B, int L) {
     BranchWs& w = ws.br[j];
     w.rows = ceil_div(L, b.scale);
     w.n_chunks = ceil_div(w.rows, kGlaChunk);
-    w.n_halves = ceil_div(w.rows, kChunk);
     w.seg_chunks = std::max(1, std::min(seg_chunks, w.n_chunks));
     w.n_segs = std::max(1, ceil_div(w.n_chunks, w.seg_chunks));
     const size_t n = BB * w.rows;
     if (b.scale > 1) add(w.Xp, cur, n * d * 2);
-    add(w.q, cur, n * b.heads * h->dkp * 2);
-    add(w.k, cur, n * b.heads * h->dkp * 2);
     add(w.qs, cur, n * b.heads * h->dkp * 2);
     add(w.ks, cur, n * b.heads * h->dkp * 2);
     add(w.v, cur, n * b.heads * h->dvp * 2);
-    add(w.g, cur, n * h->rp * 4);
+    add(w.gd, cur, n * b.heads * h->dkp * 4);
     add(w.gamma, cur, BB * w.n_chunks * b.heads * h->dkp * 4);
     add(w.mid, cur, BB * w.n_chunks * b.heads * h->dkp * 4);
     add(w.o, cur, n * b.heads * h->dvp * 2);
@@ -232,7 +248,7 @@ Workspace layout(const msgla_handle* h, int B, int L) {
     }
   }
   add(ws.w, cur, BB * L * h->n_scales * 4);
-  if (h->main_index >= 0) add(ws.z, cur, BB * L * h->ldz * 4);
+  add(ws.u, cur, BB * L * h->ldu * 4);
   ws.total = cur;
   return ws;
 }
@@ -283,6 +299,7 @@ void free_handle(msgla_handle* h) {
     cudaFree(h->br[j].Wop);
     cudaFree(h->br[j].normw);
   }
+  cudaFree(h->Wu);
   cudaFree(h->Wfuse);
   cudaFree(h->bfuse);
   cudaFree(h->d_err);
@@ -366,6 +383,12 @@ int create_impl(msgla_handle* h, const msgla_weights* w) {
     }
   }
   if (!w->Wfuse) return fail(MSGLA_ERR_INVALID_ARG, "Wfuse is NULL");
+  // gate inputs and fusion logits of the unpooled rows (one bf16 GEMM over X)
+  if ((st = dmalloc_zero(&h->Wu, static_cast<size_t>(h->ldu) * d * 2))) return st;
+  CUDA_TRY(launch_bf16_copy_rows(static_cast<const __nv_bfloat16*>(w->Wfuse), d, h->n_scales, d, h->Wu, d, 0));
+  for (int j = 0; j < h->n_scales; ++j)
+    CUDA_TRY(launch_bf16_copy_rows(static_cast<const __nv_bfloat16*>(w->Wg1[j]), d, r, d,
+                                   h->Wu + static_cast<size_t>(16 + j * h->rp) * d, d, 0));
   if ((st = dmalloc_zero(&h->Wfuse, static_cast<size_t>(h->n_scales) * d * 2))) return st;
   if ((st = dmalloc_zero(&h->bfuse, static_cast<size_t>(h->n_scales) * 4))) return st;
   CUDA_TRY(cudaMemcpy(h->Wfuse, w->Wfuse, static_cast<size_t>(h->n_scales) * d * 2, cudaMemcpyDeviceToDevice));
@@ -427,6 +450,18 @@ bool coarse_overlap(const msgla_handle* h, const Workspace& ws, int B, long long
   return h->sm_count - ctas >= 2;
 }
 
+// Pooling and the gate inputs in one pass over X (k_pool.cu): every coarse scale
+// a power of two up to 8 (pooled blocks inside the 128-row tiles) and U at most
+// 256 columns wide (one TMA box of Wu).
+bool fused_pool(const msgla_handle* h) {
+  if (h->ldu > 256) return false;
+  for (int j = 0; j < h->n_scales; ++j) {
+    const int s = h->br[j].scale;
+    if (s != 1 && s != 2 && s != 4 && s != 8) return false;
+  }
+  return true;
+}
+
 int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* wsp, size_t ws_bytes,
                  cudaStream_t st, Recorder* rec = nullptr, const uint8_t* M = nullptr) {
   Recorder none;
@@ -445,33 +480,137 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   auto at = [&](const Region& r) { return static_cast<void*>(base + r.off); };
   const int ns = h->n_scales;
 
-  // 1. pooling + fusion weights
-  PoolParams pp{};
-  pp.X = static_cast<const __nv_bfloat16*>(X);
-  pp.M = M;
-  pp.B = B;
-  pp.L = L;
-  pp.d = d;
-  pp.n_scales = ns;
-  for (int j = 0; j < ns; ++j) {
-    pp.scales[j] = h->br[j].scale;
-    pp.Xp[j] = h->br[j].scale > 1 ? static_cast<__half*>(at(ws.br[j].Xp)) : nullptr;
+  static thread_local GemmParams gp;
+  // 1-2. gate inputs and fusion logits of the unpooled rows, U = X Wu^T (fp32
+  // [B, L, ldu]): every branch's low-rank gate input is a column block of U (a
+  // coarse branch's is the mean over its pooled block, pooling being linear),
+  // and the fusion logits z_t = W_fuse x_t of Eq. (10) are its first columns;
+  // without a scale-1 branch the fusion weights too. Pooled rows of the coarse
+  // branches (Eq. (8)). One pass over X when every coarse scale is a power of two
+  // up to 8 (pool_u); otherwise a GEMM for U and a pooling kernel.
+  if (fused_pool(h)) {
+    PoolUParams q{};
+    if (!encode_3d(&q.tmX, true, X, d, L, B, 128) || !encode_2d(&q.tmW, true, h->Wu, d, h->ldu, h->ldu))
+      return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (pooling and gate inputs)");
+    q.X = static_cast<const __nv_bfloat16*>(X);
+    q.M = M;
+    q.U = static_cast<float*>(at(ws.u));
+    q.w = h->main_index < 0 ? static_cast<float*>(at(ws.w)) : nullptr;
+    q.bfuse = h->bfuse;
+    q.B = B;
+    q.L = L;
+    q.d = d;
+    q.m_tiles = ceil_div(L, 128);
+    q.ldu = h->ldu;
+    // TMEM: U in [0, ldu rounded up to a power of two), then two 64-column
+    // buffers of pooled sums
+    q.pool_col = 32;
+    while (q.pool_col < h->ldu) q.pool_col *= 2;
+    q.tmem_cols = 32;
+    while (q.tmem_cols < q.pool_col + 64 * kPoolUBufs) q.tmem_cols *= 2;
+    const int stage_bytes = 128 * 128 + h->ldu * 128;
+    q.stages = std::min(kPoolUMaxStages, (192 * 1024 - 32 * 1024) / stage_bytes);
+    q.n_scales = ns;
+    for (int l = 0; l < 4; ++l) q.lvl_branch[l] = -1;
+    int slot = 0;
+    for (int l = 1; l <= 3; ++l) {
+      for (int j = 0; j < ns; ++j) {
+        if (h->br[j].scale != (1 << l)) continue;
+        q.lvl_branch[l] = q.n_coarse;
+        q.slot_base[l] = slot;
+        slot += 128 >> l;
+        q.rows[q.n_coarse] = ws.br[j].rows;
+        q.Xp[q.n_coarse] = static_cast<__half*>(at(ws.br[j].Xp));
+        ++q.n_coarse;
+      }
+    }
+    q.err = h->d_err;
+    CUDA_TRY(launch_pool_u(q, st));
+    CUDA_TRY(rec->mark(st));
+  } else {
+    memset(&gp, 0, sizeof(gp));
+    gp.err = h->d_err;
+    GemmTask& t = gp.task[0];
+    if (!encode_3d(&t.tmA, true, X, d, L, B, kGemmBM) || !encode_2d(&t.tmB, true, h->Wu, d, h->ldu, 128))
+      return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (gate inputs)");
+    t.rows = L;
+    t.m_tiles = ceil_div(L, kGemmBM);
+    t.n_tiles = ceil_div(h->ldu, 256);
+    t.N = h->ldu;
+    t.K = d;
+    t.tile_begin = 0;
+    t.ab_bf16 = 1;
+    t.epi = kEpiStoreF32;
+    t.f32 = static_cast<float*>(at(ws.u));
+    t.ldf = h->ldu;
+    t.n_scales = ns;
+    t.bfuse = h->bfuse;
+    t.w = h->main_index < 0 ? static_cast<float*>(at(ws.w)) : nullptr;
+    gp.n_tasks = 1;
+    gp.total_tiles = B * t.m_tiles * t.n_tiles;
+    CUDA_TRY(launch_gemm(gp, 256, st));
+    CUDA_TRY(rec->mark(st));
+    PoolParams pp{};
+    pp.X = static_cast<const __nv_bfloat16*>(X);
+    pp.M = M;
+    pp.B = B;
+    pp.L = L;
+    pp.d = d;
+    pp.n_scales = ns;
+    for (int j = 0; j < ns; ++j) {
+      pp.scales[j] = h->br[j].scale;
+      pp.Xp[j] = h->br[j].scale > 1 ? static_cast<__half*>(at(ws.br[j].Xp)) : nullptr;
+    }
+    pp.Wfuse = h->Wfuse;
+    pp.bfuse = h->bfuse;
+    pp.w = static_cast<float*>(at(ws.w));
+    pp.block_rows = h->pool_rows;
+    pp.want_w = 0;
+    pp.err = h->d_err;
+    if (h->pool_rows > 1) {
+      CUDA_TRY(launch_pool_fuse(pp, st));
+      CUDA_TRY(rec->mark(st));
+    }
   }
-  pp.Wfuse = h->Wfuse;
-  pp.bfuse = h->bfuse;
-  pp.w = static_cast<float*>(at(ws.w));
-  pp.block_rows = h->pool_rows;
-  pp.want_w = h->main_index < 0 ? 1 : 0;
-  pp.err = h->d_err;
-  // nothing to pool and no fusion weights to form: single-scale layer
-  const bool need_pool = pp.want_w || h->pool_rows > 1;
-  if (need_pool) {
-    CUDA_TRY(launch_pool_fuse(pp, st));
+
+  // 3. the gate (one launch over all branches): exponents d = b - m per pooled
+  // row and key channel (b the cumulative sum of log2 alpha over a 128-row
+  // chunk, m its value at row 63) and the chunk decays gamma, mid
+  {
+    GateParams g{};
+    int blocks = 0;
+    for (int j = 0; j < ns; ++j) {
+      const Branch& b = h->br[j];
+      const BranchWs& bw = ws.br[j];
+      GateBranch& q = g.br[j];
+      q.Wg2 = b.Wg2p;
+      q.bg = b.bgp;
+      q.d = static_cast<float*>(at(bw.gd));
+      q.gamma = static_cast<float*>(at(bw.gamma));
+      q.mid = static_cast<float*>(at(bw.mid));
+      q.rows = bw.rows;
+      q.n_chunks = bw.n_chunks;
+      q.ldk = b.heads * h->dkp;
+      q.cblocks = ceil_div(q.ldk, 256);
+      q.ucol = 16 + j * h->rp;
+      q.scale = b.scale;
+      q.block_begin = blocks;
+      blocks += B * bw.n_chunks * 2 * q.cblocks;
+    }
+    g.u = static_cast<const float*>(at(ws.u));
+    g.mask = M;
+    g.n_branches = ns;
+    g.total_blocks = blocks;
+    g.L = L;
+    g.ldu = h->ldu;
+    g.rp = h->rp;
+    g.inv_normalizer = 1.f / c.gate_normalizer;
+    g.err = h->d_err;
+    CUDA_TRY(launch_gate(g, st));
     CUDA_TRY(rec->mark(st));
   }
 
-  // 2. projections (grouped over branches)
-  static thread_local GemmParams gp;
+  // 4. projections (grouped over branches): Qs = q 2^d, Ks = k 2^-d and v (fp16)
   memset(&gp, 0, sizeof(gp));
   gp.err = h->d_err;
   int tiles = 0;
@@ -484,27 +623,23 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
         !encode_2d(&t.tmB, bf, b.Bproj, d, b.np, 128))
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (projection, scale %d)", b.scale);
     t.rows = bw.rows;
-    t.m_tiles = ceil_div(bw.rows, kGemmBM);
-    t.n_tiles = ceil_div(b.np, 256);
-    t.N = b.np;
-    t.K = d;
-    t.tile_begin = tiles;
-    t.ab_bf16 = bf ? 1 : 0;
-    t.epi = kEpiProj;
     t.nq = t.nk = b.heads * h->dkp;
     t.nv = b.heads * h->dvp;
     t.ng = h->rp;
-    t.nz = (j == h->main_index) ? h->n_scales : 0;
-    t.ldz = h->ldz;
-    t.z = (j == h->main_index) ? static_cast<float*>(at(ws.z)) : nullptr;
-    t.q = static_cast<__half*>(at(bw.q));
-    t.k = static_cast<__half*>(at(bw.k));
-    t.v = static_cast<__half*>(at(bw.v));
-    t.g = static_cast<float*>(at(bw.g));
+    t.n_qk = b.heads * (h->dkp / 128);
+    t.m_tiles = ceil_div(bw.rows, kGemmBM);
+    t.N = t.nq + t.nk + t.nv;
+    t.n_tiles = t.n_qk + ceil_div(t.nv, 256);
+    t.K = d;
+    t.tile_begin = tiles;
+    t.ab_bf16 = bf ? 1 : 0;
+    t.epi = kEpiProjGate;
+    t.dkp = h->dkp;
+    t.gd = static_cast<const float*>(at(bw.gd));
     t.mask = bf ? M : nullptr;
-    if (!encode_out_3d(&t.tmOut[0], false, t.q, t.nq, bw.rows, B) ||
-        !encode_out_3d(&t.tmOut[1], false, t.k, t.nk, bw.rows, B) ||
-        !encode_out_3d(&t.tmOut[2], false, t.v, t.nv, bw.rows, B))
+    if (!encode_out_3d_32(&t.tmQK[0], at(bw.qs), t.nq, bw.rows, B) ||
+        !encode_out_3d_32(&t.tmQK[1], at(bw.ks), t.nk, bw.rows, B) ||
+        !encode_out_3d(&t.tmOut[2], false, at(bw.v), t.nv, bw.rows, B))
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (projection outputs, scale %d)", b.scale);
     tiles += B * t.m_tiles * t.n_tiles;
   }
@@ -513,40 +648,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   CUDA_TRY(launch_gemm(gp, 256, st));
   CUDA_TRY(rec->mark(st));
 
-  // 3. gates (one launch over all branches)
-  {
-    GateParams g{};
-    int blocks = 0;
-    for (int j = 0; j < ns; ++j) {
-      const Branch& b = h->br[j];
-      const BranchWs& bw = ws.br[j];
-      GateBranch& q = g.br[j];
-      q.q = static_cast<const __half*>(at(bw.q));
-      q.k = static_cast<const __half*>(at(bw.k));
-      q.g = static_cast<const float*>(at(bw.g));
-      q.Wg2 = b.Wg2p;
-      q.bg = b.bgp;
-      q.qs = static_cast<__half*>(at(bw.qs));
-      q.ks = static_cast<__half*>(at(bw.ks));
-      q.gamma = static_cast<float*>(at(bw.gamma));
-      q.mid = static_cast<float*>(at(bw.mid));
-      q.rows = bw.rows;
-      q.heads = b.heads;
-      q.n_halves = bw.n_halves;
-      q.block_begin = blocks;
-      blocks += B * b.heads * bw.n_halves * (h->dkp / 128);
-    }
-    g.n_branches = ns;
-    g.total_blocks = blocks;
-    g.dkp = h->dkp;
-    g.rp = h->rp;
-    g.inv_normalizer = 1.f / c.gate_normalizer;
-    g.err = h->d_err;
-    CUDA_TRY(launch_gate(g, st));
-    CUDA_TRY(rec->mark(st));
-  }
-
-  // 4. chunkwise GLA (grouped over branches; longest sequences first). Long
+  // 5. chunkwise GLA (grouped over branches; longest sequences first). Long
   // sequences with few CTAs run as segments: a state pass over all but the last
   // segment, a scan for the segments' initial states, then the full pass.
   static thread_local GlaParams lp;
@@ -622,7 +724,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   CUDA_TRY(launch_gla(lp, st));
   CUDA_TRY(rec->mark(st));
 
-  // 4b. optional per-head RMS norm of the GLA output (in place)
+  // 5b. optional per-head RMS norm of the GLA output (in place)
   if (c.head_norm) {
     HeadNormParams np{};
     long long warps = 0;
@@ -645,7 +747,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     CUDA_TRY(rec->mark(st));
   }
 
-  // 5. coarse branches: Y^(s) = o W_o^T (fp16). Overlapped with the GLA, the
+  // 6. coarse branches: Y^(s) = o W_o^T (fp16). Overlapped with the GLA, the
   // branches with the fewest chunks (largest scale) come first: their GLA CTAs
   // finish first.
   memset(&gp, 0, sizeof(gp));
@@ -700,7 +802,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     }
   }
 
-  // 6. scale-1 branch fused with hold + fusion, or the stand-alone hold + fusion
+  // 7. scale-1 branch fused with hold + fusion, or the stand-alone hold + fusion
   if (h->main_index >= 0) {
     memset(&gp, 0, sizeof(gp));
     gp.err = h->d_err;
@@ -722,8 +824,8 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.out = static_cast<__nv_bfloat16*>(O);
     if (!encode_out_3d(&t.tmOut[0], true, O, d, L, B))
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (layer output)");
-    t.zf = static_cast<const float*>(at(ws.z));
-    t.ldz = h->ldz;
+    t.zf = static_cast<const float*>(at(ws.u));  // fusion logits: columns 0.. of U
+    t.ldz = h->ldu;
     t.bfuse = h->bfuse;
     t.w = static_cast<float*>(at(ws.w));
     t.n_scales = ns;
@@ -1072,6 +1174,7 @@ int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weight
   h->d_tiles = nullptr;
   h->copy_in = h->copy_out = nullptr;
   h->ev_start = h->ev_in = h->ev_done = nullptr;
+  h->Wu = nullptr;
   h->Wfuse = nullptr;
   h->bfuse = nullptr;
   h->d_err = nullptr;
@@ -1086,6 +1189,7 @@ int msgla_create(msgla_handle** out, const msgla_config* cfg, const msgla_weight
   h->sm_count = prop.multiProcessorCount;
   h->nzp = 16;
   h->ldz = cfg->n_scales <= 4 ? 4 : 8;
+  h->ldu = 16 + cfg->n_scales * h->rp;
   int lcm = 1;
   for (int j = 0; j < h->n_scales; ++j) {
     h->br[j].scale = cfg->scales[j];
@@ -1297,11 +1401,11 @@ int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index,
   if (st) return st;
   if (B == 0 || L == 0) return fail(MSGLA_ERR_INVALID_ARG, "empty input has no workspace");
   const Workspace ws = layout(h, B, L);
-  if (which == 7) {
-    *offset = ws.w.off;
+  if (which == 7 || which == 8) {
+    *offset = which == 7 ? ws.w.off : ws.u.off;
     dims[0] = B;
     dims[1] = L;
-    dims[2] = h->n_scales;
+    dims[2] = which == 7 ? h->n_scales : h->ldu;
     return MSGLA_OK;
   }
   if (scale_index < 0 || scale_index >= h->n_scales) return fail(MSGLA_ERR_INVALID_ARG, "scale_index out of range");
@@ -1311,19 +1415,20 @@ int msgla_workspace_tensor(const msgla_handle* h, int B, int L, int scale_index,
   int cols = 0;
   switch (which) {
     case 0: r = &bw.Xp; cols = h->cfg.d; break;
-    case 1: r = &bw.q; cols = b.heads * h->dkp; break;
-    case 2: r = &bw.k; cols = b.heads * h->dkp; break;
+    case 1: r = &bw.qs; cols = b.heads * h->dkp; break;
+    case 2: r = &bw.ks; cols = b.heads * h->dkp; break;
     case 3: r = &bw.v; cols = b.heads * h->dvp; break;
-    case 4: r = &bw.g; cols = h->rp; break;
     case 5: r = &bw.o; cols = b.heads * h->dvp; break;
     case 6: r = &bw.Y; cols = h->cfg.d; break;
+    case 9: r = &bw.gamma; cols = b.heads * h->dkp; break;
+    case 10: r = &bw.mid; cols = b.heads * h->dkp; break;
     default: return fail(MSGLA_ERR_INVALID_ARG, "which=%d unknown", which);
   }
   if (r->bytes == 0) return fail(MSGLA_ERR_INVALID_ARG, "tensor %d does not exist for scale index %d", which,
                                  scale_index);
   *offset = r->off;
   dims[0] = B;
-  dims[1] = bw.rows;
+  dims[1] = (which == 9 || which == 10) ? bw.n_chunks : bw.rows;
   dims[2] = cols;
   return MSGLA_OK;
 }
@@ -1388,9 +1493,14 @@ int msgla_launch_plan(const msgla_handle* h, int B, int L, char* names, size_t l
     out += n;
   };
   if (B > 0 && L > 0) {
-    if (h->main_index < 0 || h->pool_rows > 1) add_name("pool_fuse");
-    add_name("proj_gemm");
+    if (fused_pool(h)) {
+      add_name("pool_u");
+    } else {
+      add_name("gate_inputs");
+      if (h->pool_rows > 1) add_name("pool");
+    }
     add_name("gate");
+    add_name("proj_gemm");
     const Workspace ws = layout(h, B, L);
     bool segmented = false;
     for (int j = 0; j < h->n_scales; ++j) segmented |= ws.br[j].n_segs > 1;

@@ -33,7 +33,6 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // Fixed tile constants.
 constexpr int kGemmBM = 128;     // GEMM rows per tile (tcgen05 M)
 constexpr int kGemmBK = 64;      // GEMM K per stage (one 128-byte swizzle atom of 16-bit data)
-constexpr int kChunk = 64;       // rows per gate block (half of a GLA chunk)
 constexpr int kGlaChunk = 128;   // chunk length of the chunkwise GLA kernel
 constexpr int kGlaTile = 128;    // value columns per GLA CTA (tcgen05 M of the output MMA)
 constexpr int kMaxTasks = 8;     // GEMM tasks per grouped launch
@@ -43,6 +42,8 @@ enum EpiKind : int {
   kEpiProj = 0,      // split columns into q | k | v (fp16) | g (fp32)
   kEpiStoreF16 = 1,  // plain fp16 store
   kEpiFuse = 2,      // O = w_main * acc + sum_coarse w_s * held Y_s  (bf16)
+  kEpiProjGate = 3,  // q|k tiles -> decay-scaled Qs | Ks (fp16) from the gate exponents; v tiles fp16
+  kEpiStoreF32 = 4,  // plain fp32 store (gate inputs and fusion logits), optionally the fusion weights
 };
 
 // One GEMM D[rows x N] = A[rows x K] * B[N x K]^T per batch, tiled 128 x BN.
@@ -53,6 +54,8 @@ struct alignas(64) GemmTask {
   // of 32 rows x 64 columns staged per epilogue warp): kEpiProj q, k, v;
   // kEpiStoreF16 y; kEpiFuse out
   CUtensorMap tmOut[3];
+  // kEpiProjGate: Qs and Ks, 3D {nq, rows, B}, box {32, 32, 1}, 64B swizzle
+  CUtensorMap tmQK[2];
   int rows, m_tiles, n_tiles, N, K, tile_begin, ab_bf16, epi;
   // kEpiProj (columns: q | k | v | g (ng) | fusion logits z (nz, scale-1 branch))
   int nq, nk, nv, ng, nz, ldz;
@@ -79,6 +82,17 @@ struct alignas(64) GemmTask {
   int coarse_index[kMaxScales];
   int coarse_rows[kMaxScales];
   const __half* coarse_y[kMaxScales];
+  // kEpiProjGate. Tiles [0, n_qk) of a batch row tile are q|k tiles: 128 key
+  // channels c0.. of one head, the B rows of W_q (CTA rank 0 / columns 0..127)
+  // and of W_k (rank 1 / columns 128..255) for the same channels, so that one
+  // load of the gate exponents d scales both. Tiles from n_qk on cover the v
+  // columns. Outputs: Qs = q 2^d (tmQK[0]), Ks = k 2^-d (tmQK[1]), v (tmOut[2]).
+  int n_qk, dkp;
+  const float* gd;        // [B, rows, nq] gate exponents d = b - m (launch_gate)
+  // kEpiStoreF32: D -> f32 [B, rows, ldf]; with w set, also the fusion weights
+  // w = softmax(D[:, 0:n_scales] + bfuse) (columns 0.. hold the fusion logits)
+  float* f32;
+  int ldf, pad3_;
 };
 
 // Rows of one 64-column box of held coarse rows staged by the fused output GEMM
@@ -170,22 +184,51 @@ struct PoolParams {
 };
 cudaError_t launch_pool_fuse(const PoolParams& p, cudaStream_t st);
 
-// gates: log alpha, chunk-local cumulative sums, scaled q/k and chunk decays
+
+// One pass over X per 128-row tile (k_pool.cu): U = X Wu^T (the fusion logits
+// and every branch's gate input, fp32 [B, L, ldu]), the pooled rows of every
+// coarse scale (powers of two dividing 128) and, with w set, the fusion weights.
+constexpr int kPoolUMaxStages = 8;
+constexpr int kPoolUBufs = 4;  // TMEM buffers of pooled sums (64 columns each)
+struct PoolUParams {
+  CUtensorMap tmX;       // X: 3D {d, L, B}, box {64, 128, 1}, bf16, 128B swizzle
+  CUtensorMap tmW;       // Wu: 2D {d, ldu}, box {64, ldu}, bf16, 128B swizzle
+  const __nv_bfloat16* X;  // [B, L, d] (the tensor map's memory; bulk L2 prefetch)
+  const uint8_t* M;      // [B, L] valid-token mask of the pooling, or null
+  float* U;              // [B, L, ldu]
+  float* w;              // [B, L, n_scales] fusion weights, or null
+  const float* bfuse;    // [n_scales]
+  int B, L, d, m_tiles, ldu, tmem_cols, pool_col, stages, n_scales;
+  int n_coarse;          // coarse branches (scales 2, 4, 8)
+  int lvl_branch[4];     // coarse branch of scale 2^l (l = 1..3), or -1
+  int slot_base[4];      // first pooling slot (TMEM lane) of scale 2^l
+  int rows[kMaxScales];  // pooled rows of each coarse branch
+  __half* Xp[kMaxScales];
+  int* err;
+};
+int pool_u_smem_bytes(int ldu, int stages);
+cudaError_t launch_pool_u(const PoolUParams& p, cudaStream_t st);
+
+// The gate of Sec. 2.1 per pooled row and key channel, in the form the chunkwise
+// GLA kernel takes: with l = log2 alpha = log2(e) logsigmoid(z) / normalizer,
+// z = g W_g2^T + b_g (g: the row's low-rank gate input, a coarse branch's the
+// mean over its block of the unpooled rows' inputs), b the cumulative sum of l
+// over the rows of a 128-row chunk and m = b at its row 63: the exponents
+// d = b - m (the projection stores Qs = q 2^d, Ks = k 2^-d), and per chunk
+// gamma = 2^{b_127 - m}, mid = 2^{m}.
 struct GateBranch {
-  const __half* q;   // [B, n_s, h*dkp]
-  const __half* k;
-  const float* g;    // [B, n_s, rp]
-  const float* Wg2;  // [h*dkp, rp]
-  const float* bg;   // [h*dkp]
-  __half* qs;        // q * exp(b - m)
-  __half* ks;        // k * exp(m - b)
-  float* gamma;      // [B, n_chunks, h*dkp] = exp(b_last - m)
-  float* mid;        // [B, n_chunks, h*dkp] = exp(m)
-  int rows, heads, n_halves, block_begin;
+  const float* Wg2;  // [ldk, rp]
+  const float* bg;   // [ldk]
+  float* d;          // [B, rows, ldk]
+  float* gamma;      // [B, n_chunks, ldk]
+  float* mid;        // [B, n_chunks, ldk]
+  int rows, n_chunks, ldk, cblocks, ucol, scale, block_begin;
 };
 struct GateParams {
   GateBranch br[kMaxScales];
-  int n_branches, total_blocks, dkp, rp;
+  const float* u;        // [B, L, ldu] gate inputs of the unpooled rows
+  const uint8_t* mask;   // [B, L] valid-token mask of the pooled means, or null
+  int n_branches, total_blocks, L, ldu, rp;
   float inv_normalizer;
   int* err;
 };

@@ -172,6 +172,10 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // All committed bulk stores of this thread are complete.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Bulk prefetch of [ptr, ptr + bytes) into L2 (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -375,6 +379,27 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mas
 // next kernel start launching.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------- special functions
+// 2^x and log2(x) by the hardware approximations (ex2.approx: relative error
+// about 2^-22; lg2.approx: absolute error about 2^-22 for x in (1, 2]), far
+// below the fp16 rounding of the decay-scaled queries and keys they feed.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Accumulates a packed fp16 pair's exponents into `acc` so that bit 15 or bit 31
+// of acc ends up set iff some half seen was inf or nan (exponent all ones: adding
+// one to the exponent field then carries into that half's sign position).
+__device__ __forceinline__ void half2_track_nonfinite(uint32_t& acc, uint32_t h) {
+  acc |= (h & 0x7c007c00u) + 0x04000400u;
+}
 
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {

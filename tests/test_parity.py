@@ -51,11 +51,30 @@ def test_tiny_workload():
     layer.close()
 
 
+def chunk_scaled(q, k, log_alpha, chunk=128):
+    """Decay-scaled queries and keys of the chunkwise GLA form: within each
+    chunk of `chunk` rows, b = cumulative sum of log alpha from the chunk's first
+    row, m = b at the chunk's row 63 (its last row if shorter); Qs = q e^{b-m},
+    Ks = k e^{m-b}, gamma = e^{b_last - m}, mid = e^{m} per chunk and channel."""
+    n = q.shape[0]
+    Qs, Ks = np.zeros_like(q), np.zeros_like(k)
+    gamma, mid = [], []
+    for c0 in range(0, n, chunk):
+        b = np.cumsum(log_alpha[c0:c0 + chunk], axis=0)
+        m = b[min(63, b.shape[0] - 1)]
+        Qs[c0:c0 + chunk] = q[c0:c0 + chunk] * np.exp(b - m)
+        Ks[c0:c0 + chunk] = k[c0:c0 + chunk] * np.exp(m - b)
+        gamma.append(np.exp(b[-1] - m))
+        mid.append(np.exp(m))
+    return Qs, Ks, np.array(gamma), np.array(mid)
+
+
 @needs_gpu
 def test_intermediate_stages():
-    """Pooled rows, q/k/v, the low-rank gate, the GLA output and the fusion
-    weights each match the oracle's intermediates (several chunks, ragged tail)."""
-    from scale_gated_linear_b200 import WS_FUSION, WS_GATE, WS_O, WS_POOLED, WS_Q, WS_K, WS_V
+    """Pooled rows, the gate inputs and fusion logits, the decay-scaled queries and
+    keys with their chunk decays, v, the GLA output and the fusion weights each
+    match the oracle's intermediates (several chunks, ragged tail)."""
+    from scale_gated_linear_b200 import WS_FUSION, WS_GAMMA, WS_KS, WS_MID, WS_O, WS_POOLED, WS_QS, WS_U, WS_V
     w = wl.WORKLOADS["msgla_340m"].replace(name="mid")
     B, L = 2, 300
     inp = gpu_inputs(w, B=B, L=L)
@@ -68,20 +87,38 @@ def test_intermediate_stages():
         d = np.abs(a - b).max() / np.abs(b).max()
         assert d <= tol, f"{name}: {d:.3e}"
 
+    def heads_only(t, h, width):
+        pad = t.shape[-1] // h
+        return np.concatenate([t[..., x * pad:x * pad + width] for x in range(h)], axis=-1)
+
     close("w", layer.workspace_tensor(ws, B, L, 0, WS_FUSION).cpu().numpy(), inter["w"], 1e-5)
+    U = layer.workspace_tensor(ws, B, L, 0, WS_U).cpu().numpy()
+    ns = len(w.scales)
+    close("fusion logits", U[:, :, :ns], f["X"] @ f["Wfuse"].T, 2e-3)
+    rp = -(-w.gate_rank // 16) * 16
     for j, (s, h) in enumerate(zip(w.scales, w.heads)):
         bi = inter["branches"][j]
         if s > 1:
             close(f"pooled s={s}", layer.workspace_tensor(ws, B, L, j, WS_POOLED).float().cpu().numpy(), bi["Xp"],
                   1e-3)
-        for name, which, width, ref_t, tol in (("q", WS_Q, w.d_k, bi["q"], 2e-3), ("k", WS_K, w.d_k, bi["k"], 2e-3),
-                                               ("v", WS_V, w.d_v, bi["v"], 2e-3), ("o", WS_O, w.d_v, bi["o"], 4e-3)):
-            t = layer.workspace_tensor(ws, B, L, j, which).float().cpu().numpy()
-            pad = t.shape[2] // h
-            t = np.concatenate([t[:, :, x * pad:x * pad + width] for x in range(h)], axis=2)
+        # the branch's gate input: block means of the unpooled rows' columns
+        gu = U[:, :, 16 + j * rp:16 + j * rp + w.gate_rank]
+        n = bi["Xp"].shape[1]
+        gp = np.stack([gu[:, i * s:min(L, i * s + s)].mean(axis=1) for i in range(n)], axis=1)
+        close(f"g s={s}", gp, bi["Xp"] @ f["branches"][j]["Wg1"].T, 2e-3)
+        qs = heads_only(layer.workspace_tensor(ws, B, L, j, WS_QS).float().cpu().numpy(), h, w.d_k)
+        ks = heads_only(layer.workspace_tensor(ws, B, L, j, WS_KS).float().cpu().numpy(), h, w.d_k)
+        gam = heads_only(layer.workspace_tensor(ws, B, L, j, WS_GAMMA).cpu().numpy(), h, w.d_k)
+        mid = heads_only(layer.workspace_tensor(ws, B, L, j, WS_MID).cpu().numpy(), h, w.d_k)
+        for b in range(B):
+            Qr, Kr, Gr, Mr = chunk_scaled(bi["q"][b], bi["k"][b], bi["log_alpha"][b])
+            close(f"Qs s={s} b={b}", qs[b], Qr, 2e-3)
+            close(f"Ks s={s} b={b}", ks[b], Kr, 2e-3)
+            close(f"gamma s={s} b={b}", gam[b], Gr, 1e-4)
+            close(f"mid s={s} b={b}", mid[b], Mr, 1e-4)
+        for name, which, width, ref_t, tol in (("v", WS_V, w.d_v, bi["v"], 2e-3), ("o", WS_O, w.d_v, bi["o"], 4e-3)):
+            t = heads_only(layer.workspace_tensor(ws, B, L, j, which).float().cpu().numpy(), h, width)
             close(f"{name} s={s}", t, ref_t, tol)
-        g = layer.workspace_tensor(ws, B, L, j, WS_GATE).cpu().numpy()[:, :, :w.gate_rank]
-        close(f"g s={s}", g, bi["Xp"] @ f["branches"][j]["Wg1"].T, 2e-3)
     layer.close()
 
 
@@ -266,9 +303,9 @@ def test_fp16_range_overflow_is_reported():
 @needs_gpu
 def test_gate_range_overflow_is_reported():
     """A gate bias far below zero (log alpha near -200/16 per pooled step) makes
-    the decay-scaled queries and keys of the gate kernel leave the fp16 range on
-    both halves of a chunk: the kernel latches MSGLA_ERR_RANGE and the handle
-    stays usable."""
+    the decay-scaled queries and keys formed in the projection's epilogue leave
+    the fp16 range on both halves of a chunk: the kernel latches MSGLA_ERR_RANGE
+    and the handle stays usable."""
     inp = gpu_inputs(SMALL, L=200)
     strong = {k: v for k, v in inp.items()}
     strong["branches"] = [dict(br) for br in inp["branches"]]
@@ -295,7 +332,7 @@ def test_forward_profiled_records_every_launch():
     # the GLA, after a one-warp wait for the GLA CTAs to start (no plan entries,
     # counted as launches)
     assert n == len(names) + 2
-    assert names == ["pool_fuse", "proj_gemm", "gate", "gla", "out_gemm_fused"]
+    assert names == ["pool_u", "gate", "proj_gemm", "gla", "out_gemm_fused"]
     assert all(ev[i].elapsed_time(ev[i + 1]) >= 0 for i in range(len(names)))
     layer.close()
 
@@ -371,10 +408,10 @@ def test_serial_switch_runs_one_stream_with_identical_output(tmp_path):
                        text=True, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     names = r.stdout.strip().splitlines()[-1].split(",")
-    assert names == ["pool_fuse", "proj_gemm", "gate", "gla", "out_gemm_coarse", "out_gemm_fused"]
+    assert names == ["pool_u", "gate", "proj_gemm", "gla", "out_gemm_coarse", "out_gemm_fused"]
     inp = gpu_inputs(SMALL, L=100)
     got, layer, _ = run_gpu(SMALL, inp)
-    assert layer.launch_names(2, 100) == ["pool_fuse", "proj_gemm", "gate", "gla", "out_gemm_fused"]
+    assert layer.launch_names(2, 100) == ["pool_u", "gate", "proj_gemm", "gla", "out_gemm_fused"]
     layer.close()
     np.testing.assert_array_equal(np.load(out), got)
 
