@@ -527,6 +527,7 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
   __shared__ __align__(16) float gs[kGateRows * RP];
   griddep_wait();
   griddep_launch();
+  if (p.clear && blockIdx.x == 0 && threadIdx.x == 0) *p.clear = 0ull;
 #pragma unroll 1
   for (int item = blockIdx.x; item < p.total_blocks; item += gridDim.x) {
     gate_item<RP>(p, item, gs);

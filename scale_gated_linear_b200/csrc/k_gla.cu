@@ -407,6 +407,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
     __threadfence();
     atomicAdd(p.done + ti, 1ull);
   }
+  if (threadIdx.x == 0 && p.exited && !state_pass) {
+    __threadfence();
+    atomicAdd(p.exited, 1ull);
+  }
 }
 
 // Initial state of every segment: S'_init(s+1) = G_s * S'_init(s) + A_s with
@@ -435,19 +439,20 @@ __global__ void gla_scan_kernel(const __grid_constant__ GlaParams p, int B) {
   }
 }
 
-__global__ void wait_started_kernel(const unsigned long long* started, unsigned long long target, int* err) {
+__global__ void wait_started_kernel(const unsigned long long* started, const unsigned long long* exited,
+                                    unsigned long long target, int* err) {
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    wait_count(started, target, &abort_flag, err);
+    if (!wait_count_quiet(started, target)) wait_count(exited, target, &abort_flag, err);
   }
 }
 
 }  // namespace
 
-cudaError_t launch_wait_started(const unsigned long long* started, unsigned long long target, int* err,
-                                cudaStream_t st) {
-  wait_started_kernel<<<1, 32, 0, st>>>(started, target, err);
+cudaError_t launch_wait_started(const unsigned long long* started, const unsigned long long* exited,
+                                unsigned long long target, int* err, cudaStream_t st) {
+  wait_started_kernel<<<1, 32, 0, st>>>(started, exited, target, err);
   return cudaGetLastError();
 }
 

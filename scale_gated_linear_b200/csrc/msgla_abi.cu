@@ -165,7 +165,7 @@ struct msgla_handle {
   // (all zero when a forward begins: the overlapped GEMM's last CTA clears them).
   cudaStream_t side;
   cudaEvent_t ev_fork, ev_join;
-  unsigned long long* d_gla_done;  // [MSGLA_MAX_SCALES] completion, then [1] start counter
+  unsigned long long* d_gla_done;  // [MSGLA_MAX_SCALES] completion, then the start and exit counters
   unsigned int* d_tiles;           // [2] dynamic tile and exit counters of the overlapped GEMM
   // host-buffer forward: copy streams and events of its pipeline
   cudaStream_t copy_in, copy_out;
@@ -394,7 +394,7 @@ int create_impl(msgla_handle* h, const msgla_weights* w) {
   CUDA_TRY(cudaMemcpy(h->Wfuse, w->Wfuse, static_cast<size_t>(h->n_scales) * d * 2, cudaMemcpyDeviceToDevice));
   if (w->bfuse) CUDA_TRY(cudaMemcpy(h->bfuse, w->bfuse, h->n_scales * 4, cudaMemcpyDeviceToDevice));
   if ((st = dmalloc_zero(&h->d_err, sizeof(int)))) return st;
-  if ((st = dmalloc_zero(&h->d_gla_done, (MSGLA_MAX_SCALES + 1) * sizeof(unsigned long long)))) return st;
+  if ((st = dmalloc_zero(&h->d_gla_done, (MSGLA_MAX_SCALES + 2) * sizeof(unsigned long long)))) return st;
   if ((st = dmalloc_zero(&h->d_tiles, 2 * sizeof(unsigned int)))) return st;
   CUDA_TRY(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
   CUDA_TRY(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
@@ -606,6 +606,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     g.rp = h->rp;
     g.inv_normalizer = 1.f / c.gate_normalizer;
     g.err = h->d_err;
+    g.clear = h->d_gla_done + MSGLA_MAX_SCALES + 1;  // GLA exit counter
     CUDA_TRY(launch_gate(g, st));
     CUDA_TRY(rec->mark(st));
   }
@@ -718,6 +719,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     // coarse branches' CTAs signal their stored outputs to it
     lp.done = h->d_gla_done;
     lp.started = h->d_gla_done + MSGLA_MAX_SCALES;
+    lp.exited = h->d_gla_done + MSGLA_MAX_SCALES + 1;
     for (int j = 0; j < ns; ++j) lp.task[j].signal_done = j != h->main_index;
     CUDA_TRY(cudaEventRecord(h->ev_fork, st));
   }
@@ -785,9 +787,12 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     gp.total_tiles = tiles;
     if (overlap) {
       CUDA_TRY(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
-      CUDA_TRY(launch_wait_started(h->d_gla_done + MSGLA_MAX_SCALES, static_cast<unsigned long long>(gla_ctas),
+      CUDA_TRY(launch_wait_started(h->d_gla_done + MSGLA_MAX_SCALES, h->d_gla_done + MSGLA_MAX_SCALES + 1,
+                                   static_cast<unsigned long long>(gla_ctas),
                                    h->d_err, h->side));
-      // the GEMM's last CTA clears the tile, start and completion counters
+      // the GEMM's last CTA clears the tile, start and completion counters (the
+      // scale-1 GLA CTAs may still be running then: their exit counter is
+      // cleared by the next forward's gate kernel instead)
       gp.tile_counter = h->d_tiles;
       gp.tile_exit = h->d_tiles + 1;
       gp.reset64 = h->d_gla_done;
@@ -1310,6 +1315,13 @@ int msgla_forward_profiled(msgla_handle* h, const void* X, const void* M, int B,
   if (!X || !O) return fail(MSGLA_ERR_INVALID_ARG, "X or O is NULL");
   if (reinterpret_cast<uintptr_t>(X) % 16 || reinterpret_cast<uintptr_t>(O) % 16)
     return fail(MSGLA_ERR_INVALID_ARG, "X and O must be 16-byte aligned");
+  const size_t nbytes = static_cast<size_t>(B) * L * h->cfg.d * 2;
+  const uint8_t* x0 = static_cast<const uint8_t*>(X);
+  const uint8_t* o0 = static_cast<const uint8_t*>(O);
+  if (x0 < o0 + nbytes && o0 < x0 + nbytes) return fail(MSGLA_ERR_INVALID_ARG, "O overlaps X");
+  const uint8_t* m0 = static_cast<const uint8_t*>(M);
+  if (m0 && m0 < o0 + nbytes && o0 < m0 + static_cast<size_t>(B) * L)
+    return fail(MSGLA_ERR_INVALID_ARG, "O overlaps M");
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(MSGLA_ERR_CUDA, "cudaSetDevice(%d) failed", h->device);
   Recorder rec;

@@ -147,16 +147,21 @@ struct GlaParams {
   int skip_arrival;  // failure-detection tests: CTA 0 omits one barrier arrival
   int* err;
   // full pass only: every CTA of a task with signal_done adds 1 to done[t] once
-  // its outputs are stored (release), for a concurrent consumer, and every CTA
-  // adds 1 to *started when it begins (null: none)
+  // its outputs are stored (release), for a concurrent consumer; every CTA adds
+  // 1 to *started when it begins and to *exited when it leaves (null: none)
   unsigned long long* done;
   unsigned long long* started;
+  unsigned long long* exited;
 };
-// Wait (one warp, bounded) until *started reaches target: ordered on a stream
-// before a kernel that may only take SMs once every CTA of a running GLA launch
-// is resident.
-cudaError_t launch_wait_started(const unsigned long long* started, unsigned long long target, int* err,
-                                cudaStream_t st);
+// One warp on a second stream, ordered before a kernel that may only take SMs
+// once every CTA of a running GLA launch is resident: waits (bounded) until
+// *started reaches target. If that bound runs out -- some GLA CTAs could not be
+// resident at once, as on a GPU shared with other work -- it waits instead
+// (bounded) until every GLA CTA has left (*exited reaches target), which
+// degrades the overlap to the serial order; only if that too runs out does it
+// latch kDevTimeout.
+cudaError_t launch_wait_started(const unsigned long long* started, const unsigned long long* exited,
+                                unsigned long long target, int* err, cudaStream_t st);
 
 // ---------------------------------------------------------------- launchers
 // (each returns the cudaError_t of the launch)
@@ -231,6 +236,9 @@ struct GateParams {
   int n_branches, total_blocks, L, ldu, rp;
   float inv_normalizer;
   int* err;
+  // set to zero before the forward's GLA launch (the GLA exit counter of the
+  // overlapped coarse projection; null: none)
+  unsigned long long* clear;
 };
 cudaError_t launch_gate(const GateParams& p, cudaStream_t st);
 

@@ -135,6 +135,22 @@ __device__ __forceinline__ bool wait_count(const unsigned long long* c, unsigned
     __nanosleep(256);
   }
 }
+// wait_count without the error latch: false once the bound runs out (the caller
+// decides what that means).
+__device__ __forceinline__ bool wait_count_quiet(const unsigned long long* c, unsigned long long target) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(c) : "memory");
+    if (v >= target) return true;
+    if ((it & 15u) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (it == 0 || now < t0) t0 = now;
+      if (now - t0 > kWaitTimeoutNs) return false;
+    }
+    __nanosleep(256);
+  }
+}
 // Orders this thread's earlier generic-proxy accesses (such as the acquire
 // above) before its later async-proxy (TMA) accesses of global memory.
 __device__ __forceinline__ void fence_proxy_async_global() {

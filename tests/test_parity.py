@@ -416,6 +416,34 @@ def test_serial_switch_runs_one_stream_with_identical_output(tmp_path):
     np.testing.assert_array_equal(np.load(out), got)
 
 
+@needs_gpu
+def test_forward_profiled_rejects_aliased_output():
+    """The profiled forward checks its buffers like msgla_forward_masked: an
+    output that overlaps the input or the mask is an invalid argument (no kernel
+    is launched), and the handle stays usable."""
+    from scale_gated_linear_b200 import MSGLAError
+    inp = gpu_inputs(SMALL, L=100)
+    layer = _layer(SMALL, inp)
+    X = inp["X"].cuda()
+    B, L, d = X.shape
+    ws = layer.alloc_workspace(B, L)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(layer.launch_names(B, L)) + 1)]
+    with pytest.raises(MSGLAError) as e:
+        layer.forward_profiled(X, X, ws, ev)  # O is X
+    assert e.value.status == -1
+    # a mask placed inside the output buffer
+    O = torch.empty_like(X)
+    M = O.view(torch.uint8).view(-1)[: B * L].view(B, L)
+    with pytest.raises(MSGLAError) as e:
+        layer.forward_profiled(X, O, ws, ev, mask=M)
+    assert e.value.status == -1
+    n = layer.forward_profiled(X, O, ws, ev)
+    torch.cuda.synchronize()
+    layer.check_status()
+    assert n >= len(ev) - 1
+    layer.close()
+
+
 # ----------------------------------------------------------------- full sizes
 @needs_gpu
 def test_340m_layer_full_size_sampled_rows():
@@ -439,25 +467,46 @@ def test_gla_340m_full_size_sampled_row():
 
 
 @needs_gpu
-def test_long_32k_full_launch_prefix():
-    """L = 32768 in one launch; by causality its first 4096 outputs equal the
-    oracle run on the 4096-position prefix."""
+def test_long_32k_full_sequence():
+    """L = 32768 (B = 1) in the launch the bench times (sequence segments, state
+    pass and scan): every one of the 32768 positions against the oracle, and the
+    last 4096 on their own (they depend on the whole carried state)."""
     w = wl.WORKLOADS["long_32k"]
     inp = gpu_inputs(w)
     got, layer, _ = run_gpu(w, inp)
-    assert_parity(got[:, :4096], oracle_forward(w, inp, rows=4096))
-    assert np.isfinite(got).all()
+    assert "gla_state" in layer.launch_names(w.B, w.L)
+    ref = oracle_forward(w, inp)
+    assert_parity(got, ref)
+    assert_parity(got[:, -4096:], ref[:, -4096:])
     layer.close()
 
 
 @needs_gpu
 @pytest.mark.parametrize("name", ["wide_8k", "wide_8k_no_fine"])
-def test_wide_8k_full_launch_prefix(name):
+def test_wide_8k_full_row(name):
+    """The wide scale set (d = 2048, B = 4, L = 8192) and its no-fine-branch
+    ablation in the launch the bench times: batch row 0 against the oracle at
+    all 8192 positions, and the other rows finite."""
     w = wl.WORKLOADS[name]
     inp = gpu_inputs(w)
     got, layer, _ = run_gpu(w, inp)
-    assert_parity(got[0:1, :1024], oracle_forward(w, inp, rows=1024, batch=slice(0, 1)))
+    ref = oracle_forward(w, inp, batch=slice(0, 1))
+    assert_parity(got[0:1], ref)
+    assert_parity(got[0:1, -1024:], ref[:, -1024:])
     assert np.isfinite(got).all()
+    layer.close()
+
+
+@needs_gpu
+def test_overlap_plan_falls_back_to_serial_when_gla_fills_the_gpu():
+    """The coarse output projection runs beside the GLA kernel only when the GLA
+    CTAs (one per SM) leave SMs free; at B = 10 (160 CTAs of the 340M-shaped
+    layer) they do not, and the plan runs it on the caller's stream."""
+    w = wl.WORKLOADS["msgla_340m"]
+    inp = gpu_inputs(w, B=1, L=64)
+    layer = _layer(w, inp)
+    assert "out_gemm_coarse" not in layer.launch_names(8, 2048)  # 128 GLA CTAs
+    assert "out_gemm_coarse" in layer.launch_names(10, 2048)     # 160 GLA CTAs
     layer.close()
 
 
