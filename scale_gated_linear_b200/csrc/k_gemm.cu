@@ -36,6 +36,7 @@ constexpr int kStages = 3;
 constexpr int kThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr int kEpiThreads = 256;
 constexpr int kStagerBytes = 32 * 128;              // one epilogue warp's staging buffer
+constexpr int kGdBoxBytes = 32 * 32 * 4;            // gate exponents of 32 rows x 32 channels (fp32)
 constexpr int kStagingBytes = 8 * 2 * kStagerBytes;  // eight epilogue warps, two buffers each
 
 template <int BN>
@@ -479,16 +480,21 @@ __device__ __forceinline__ void epi_columns(int warp, int n_eff, int& lo, int& h
 }
 
 // ---------------------------------------------------------------- gated projection
-// Pulls this thread's 64 gate exponents of a q|k tile (two 128-byte lines) into
-// L2 while the tile's accumulator is still being computed.
-__device__ __forceinline__ void prefetch_gate_exponents(const GemmParams& p, const TileCoord& tc, int quad, int lane,
-                                                        int ch) {
+// Gate exponents of a q|k tile for one epilogue warp: 32 rows (its TMEM lane
+// quadrant) x 32 key channels (group grp of its channel half) of d, fp32, loaded
+// by TMA into the warp's 4 KB buffer (128-byte swizzle: 16-byte chunk j of row r
+// at chunk j ^ (r & 7)); lane 0 issues it, gd_full completes when it lands.
+struct GateExp {
+  uint8_t* buf;
+  uint64_t* full;
+  uint32_t* phase;  // loads issued so far by this warp (parity of the next wait)
+};
+__device__ __forceinline__ void issue_gate_exponents(const GemmParams& p, const TileCoord& tc, int quad, int lane,
+                                                     int ch, int grp, const GateExp& ge) {
+  if (lane != 0) return;
   const GemmTask& T = p.task[tc.task];
-  const int row = tc.m0 + quad * 32 + lane;
-  if (row >= T.rows) return;
-  const float* a = T.gd + (static_cast<size_t>(tc.b) * T.rows + row) * T.nq + tc.n0 + 64 * ch;
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(a + 32));
+  mbar_arrive_expect_tx(ge.full, kGdBoxBytes);
+  tma_load_2d(&T.tmD, ge.full, ge.buf, tc.n0 + 64 * ch + 32 * grp, tc.b * T.rows + tc.m0 + quad * 32);
 }
 
 // Epilogue of a q|k tile of the gated projection (kEpiProjGate; MS-GLA reading
@@ -500,32 +506,40 @@ __device__ __forceinline__ void prefetch_gate_exponents(const GemmParams& p, con
 // value at row 63; launch_gate) it stores Qs = q 2^d and Ks = k 2^-d (fp16), the
 // operands of the chunkwise GLA kernel, as two 32 x 32 boxes through the warp's
 // staging buffer (Qs in its first 2 KB, Ks in the second; 64-byte swizzle, maps
-// tmQK). Only the side whose factor can exceed 1 is checked for the fp16 range
-// (b does not increase along the chunk: Qs in rows 0..63, Ks in rows 64..127);
-// an overflow latches kDevRange.
-__device__ __forceinline__ void epilogue_qk(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
-                                            int lane, int ch, bool padded, const Stager& stg) {
+// tmQK). The exponents of group 0 were requested before the accumulator wait
+// (issue_gate_exponents); those of group 1 are requested as soon as group 0's
+// are in registers. Only the side whose factor can exceed 1 is checked for the
+// fp16 range (b does not increase along the chunk: Qs in rows 0..63, Ks in rows
+// 64..127); an overflow latches kDevRange. Returns false if a bounded wait gave up.
+__device__ __forceinline__ bool epilogue_qk(const GemmParams& p, const TileCoord& tc, uint32_t tacc, int quad,
+                                            int lane, int ch, bool padded, const Stager& stg, const GateExp& ge,
+                                            volatile int* abort_flag) {
   const GemmTask& T = p.task[tc.task];
   const int lrow = quad * 32 + lane;
-  const int row = tc.m0 + lrow;
-  const bool valid = row < T.rows;
   const int grow_side = lrow < 64 ? 0 : 1;
-  const float4* gd = reinterpret_cast<const float4*>(T.gd + (static_cast<size_t>(tc.b) * T.rows + row) * T.nq +
-                                                     tc.n0 + 64 * ch);
   uint8_t* buf = stg.at(0);
   uint32_t over = 0;
 #pragma unroll
   for (int grp = 0; grp < 2; ++grp) {
-    float4 dn[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) dn[j] = valid ? __ldg(gd + 8 * grp + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!mbar_wait(ge.full, *ge.phase & 1, abort_flag, p.err)) return false;
+    ++*ge.phase;
     float d[32];
+    {
+      const uint8_t* row = ge.buf + lane * 128;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      d[4 * j] = dn[j].x;
-      d[4 * j + 1] = dn[j].y;
-      d[4 * j + 2] = dn[j].z;
-      d[4 * j + 3] = dn[j].w;
+      for (int j = 0; j < 8; ++j) {
+        const float4 x = *reinterpret_cast<const float4*>(row + ((j ^ (lane & 7)) << 4));
+        d[4 * j] = x.x;
+        d[4 * j + 1] = x.y;
+        d[4 * j + 2] = x.z;
+        d[4 * j + 3] = x.w;
+      }
+    }
+    if (grp == 0) {
+      // the buffer is read: the next 32 channels' exponents may land in it
+      fence_proxy_async_smem();
+      __syncwarp();
+      issue_gate_exponents(p, tc, quad, lane, ch, 1, ge);
     }
     const int cb = tc.n0 + 64 * ch + 32 * grp;  // first key channel of this group
     stg.acquire();  // the previous group's stores have read the buffer
@@ -560,14 +574,17 @@ __device__ __forceinline__ void epilogue_qk(const GemmParams& p, const TileCoord
     }
   }
   if (over & 0x80008000u) atomicCAS(p.err, 0, kDevRange);
+  return true;
 }
 
 // Prefetch the output tensor maps of every task (epilogue warps).
 __device__ __forceinline__ void prefetch_out_maps(const GemmParams& p) {
   for (int t = 0; t < p.n_tasks; ++t) {
     for (int m = 0; m < 3; ++m) prefetch_tmap(&p.task[t].tmOut[m]);
-    if (p.task[t].epi == kEpiProjGate)
+    if (p.task[t].epi == kEpiProjGate) {
       for (int m = 0; m < 2; ++m) prefetch_tmap(&p.task[t].tmQK[m]);
+      prefetch_tmap(&p.task[t].tmD);
+    }
   }
 }
 
@@ -591,8 +608,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   uint64_t* empty_bar = full_bar + kStages;
   uint64_t* acc_full = empty_bar + kStages;  // [2]
   uint64_t* acc_empty = acc_full + 2;        // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* gd_full = acc_empty + 2;         // [8] per epilogue warp: its gate exponents landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gd_full + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert((2 * kStages + 12) * 8 + 8 <= 256, "barrier region");
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
@@ -604,6 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], kEpiThreads);
     }
+    for (int w = 0; w < 8; ++w) mbar_init(&gd_full[w], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -679,7 +699,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   } else if (warp >= 2) {
     // ---------------- epilogue: one accumulator row per thread
     const int quad = warp & 3;
+    // one staging buffer per warp; the second 4 KB of its slot holds gate exponents
     const Stager stg{smem + Lay::kStagingOffset + (warp - 2) * 2 * kStagerBytes, lane};
+    uint32_t gd_phase = 0;
+    const GateExp ge{smem + Lay::kStagingOffset + (warp - 2) * 2 * kStagerBytes + kStagerBytes, &gd_full[warp - 2],
+                     &gd_phase};
     int sel = 0;
     if (lane == 0) prefetch_out_maps(p);
     uint32_t it = 0;
@@ -691,11 +715,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       epi_columns(warp, tc.n_eff, lo, hi);
       FuseW fw;
       fuse_weights(p, tc, quad, lane, lo, fw);
-      if (tc.qk) prefetch_gate_exponents(p, tc, quad, lane, (warp - 2) >= 4 ? 1 : 0);
+      if (tc.qk) issue_gate_exponents(p, tc, quad, lane, (warp - 2) >= 4 ? 1 : 0, 0, ge);
       if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
       if (tc.qk) {
-        epilogue_qk(p, tc, tmem + buf * BN, quad, lane, (warp - 2) >= 4 ? 1 : 0, padded, stg);
+        if (!epilogue_qk(p, tc, tmem + buf * BN, quad, lane, (warp - 2) >= 4 ? 1 : 0, padded, stg, ge, abort_flag))
+          break;
       } else if (p.task[tc.task].epi == kEpiStoreF32) {
         epilogue_f32(p, tc, tmem + buf * BN, quad, lane, lo, hi);
       } else {
@@ -735,13 +760,16 @@ constexpr int kHeldBytes = 60 * 1024;
 
 template <bool kHeld>
 struct PairLayout {
-  static constexpr int kStages = kHeld ? 4 : 6;
+  static constexpr int kStages = kHeld ? 4 : 5;
   static constexpr int kThreadsT = kHeld ? 352 : 320;  // + warp 10: held-row loader
   static constexpr int kStagingOffset = kStages * kPairStageBytes;
   static constexpr int kStagingBytesT = 8 * kStagerBytes;
   static constexpr int kHeldOffset = kStagingOffset + kStagingBytesT;
-  static constexpr int kBarOffset = kHeldOffset + (kHeld ? kHeldBytes : 0);
-  static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + 1024 B alignment slack
+  // !kHeld: one 4 KB buffer per epilogue warp for the gate exponents of a q|k
+  // tile (32 rows x 32 channels fp32, 128-byte swizzle), filled by TMA
+  static constexpr int kGdOffset = kHeldOffset + (kHeld ? kHeldBytes : 0);
+  static constexpr int kBarOffset = kGdOffset + (kHeld ? 0 : 8 * kGdBoxBytes);
+  static constexpr int kSmemBytes = kBarOffset + 512 + 1024;  // barriers + 1024 B alignment slack
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -761,7 +789,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
   using Lay = PairLayout<kHeld>;
   constexpr int kStagesT = Lay::kStages;
   constexpr int kHeldBars = kHeld ? 4 : 1;
-  static_assert((2 * kStagesT + 4 + 2 * kHeldBars + 2 * kTileRing) * 8 + 4 * kTileRing + 8 <= 256, "barrier region");
+  static_assert((2 * kStagesT + 4 + 2 * kHeldBars + 2 * kTileRing + 8) * 8 + 4 * kTileRing + 8 <= 512, "barrier region");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Lay::kBarOffset);
@@ -772,7 +800,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
   uint64_t* held_empty = held_full + kHeldBars;  // kHeld [4]: the epilogue warps are done with box j
   uint64_t* tile_full = held_empty + kHeldBars;  // [kTileRing] dynamic tiles
   uint64_t* tile_empty = tile_full + kTileRing;  // [kTileRing] (used in the leader)
-  volatile int* tile_slot = reinterpret_cast<volatile int*>(tile_empty + kTileRing);  // [kTileRing]
+  uint64_t* gd_full = tile_empty + kTileRing;    // [8] per epilogue warp: its gate exponents landed
+  volatile int* tile_slot = reinterpret_cast<volatile int*>(gd_full + 8);  // [kTileRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(tile_slot) + kTileRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* held_smem = smem + Lay::kHeldOffset;
@@ -798,6 +827,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
       mbar_init(&tile_full[r], 1);
       mbar_init(&tile_empty[r], kTileConsumers);
     }
+    for (int w = 0; w < 8; ++w) mbar_init(&gd_full[w], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -944,6 +974,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
     const uint32_t lead_empty0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     const uint32_t lead_empty1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
     const Stager stg{smem + Lay::kStagingOffset + (warp - 2) * kStagerBytes, lane, false};
+    uint32_t gd_phase = 0;
+    const GateExp ge{smem + Lay::kGdOffset + (warp - 2) * kGdBoxBytes, &gd_full[warp - 2], &gd_phase};
     int sel = 0;
     if (lane == 0) prefetch_out_maps(p);
     for (uint32_t it = 0;; ++it) {
@@ -958,7 +990,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
       epi_columns(warp, tc.n_eff, lo, hi);
       FuseW fw;
       fuse_weights(p, tc, quad, lane, lo, fw);
-      if (!kHeld && tc.qk) prefetch_gate_exponents(p, tc, quad, lane, (warp - 2) >= 4 ? 1 : 0);
+      if (!kHeld && tc.qk) issue_gate_exponents(p, tc, quad, lane, (warp - 2) >= 4 ? 1 : 0, 0, ge);
       if (!mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
       if (kHeld) {
@@ -980,7 +1012,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
         h.abort_flag = abort_flag;
         if (!epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel, fw, &h)) break;
       } else if (!kHeld && tc.qk) {
-        epilogue_qk(p, tc, tmem + buf * kPairBN, quad, lane, (warp - 2) >= 4 ? 1 : 0, padded, stg);
+        if (!epilogue_qk(p, tc, tmem + buf * kPairBN, quad, lane, (warp - 2) >= 4 ? 1 : 0, padded, stg, ge,
+                         abort_flag))
+          break;
       } else if (p.task[tc.task].epi == kEpiStoreF32) {
         epilogue_f32(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi);
       } else {

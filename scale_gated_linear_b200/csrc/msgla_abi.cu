@@ -120,6 +120,20 @@ bool encode_out_3d_32(CUtensorMap* m, void* base, uint64_t inner, uint64_t rows,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 row-major [rows][inner] with a {32, 32} box and 128B swizzle (the gate
+// exponents one epilogue warp of the gated projection reads).
+bool encode_f32_2d_32(CUtensorMap* m, void* base, uint64_t inner, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DeviceGuard {
   int prev = -1;
   bool ok = false;
@@ -638,7 +652,8 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.dkp = h->dkp;
     t.gd = static_cast<const float*>(at(bw.gd));
     t.mask = bf ? M : nullptr;
-    if (!encode_out_3d_32(&t.tmQK[0], at(bw.qs), t.nq, bw.rows, B) ||
+    if (!encode_f32_2d_32(&t.tmD, at(bw.gd), t.nq, static_cast<uint64_t>(B) * bw.rows) ||
+        !encode_out_3d_32(&t.tmQK[0], at(bw.qs), t.nq, bw.rows, B) ||
         !encode_out_3d_32(&t.tmQK[1], at(bw.ks), t.nk, bw.rows, B) ||
         !encode_out_3d(&t.tmOut[2], false, at(bw.v), t.nv, bw.rows, B))
       return fail(MSGLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (projection outputs, scale %d)", b.scale);

@@ -54,8 +54,10 @@ struct alignas(64) GemmTask {
   // of 32 rows x 64 columns staged per epilogue warp): kEpiProj q, k, v;
   // kEpiStoreF16 y; kEpiFuse out
   CUtensorMap tmOut[3];
-  // kEpiProjGate: Qs and Ks, 3D {nq, rows, B}, box {32, 32, 1}, 64B swizzle
+  // kEpiProjGate: Qs and Ks, 3D {nq, rows, B}, box {32, 32, 1}, 64B swizzle;
+  // the gate exponents d, 2D {nq, B * rows} fp32, box {32, 32}, 128B swizzle
   CUtensorMap tmQK[2];
+  CUtensorMap tmD;
   int rows, m_tiles, n_tiles, N, K, tile_begin, ab_bf16, epi;
   // kEpiProj (columns: q | k | v | g (ng) | fusion logits z (nz, scale-1 branch))
   int nq, nk, nv, ng, nz, ldz;
