@@ -18,6 +18,7 @@
 //                     Eq. (11)) when no branch has scale 1.
 //   weight converters used once by msgla_create.
 #include <algorithm>
+#include <type_traits>
 
 #include "msgla_internal.h"
 #include "sm100_ptx.cuh"
@@ -623,33 +624,49 @@ __device__ __forceinline__ void gate_item(const GateParams& p, int item, float* 
   // in the first half): first the batch's log2 alpha (independent of each
   // other), then in row order d (first half: the sum of the rows after it,
   // negated, taken before its own l is added; second half: the running sum
-  // including l), stored as soon as it is known.
-  constexpr int kBatch = 8;
-  const long long step = (half == 0 ? -1 : 1) * static_cast<long long>(P.ldk / 2);
+  // including l), stored as soon as it is known. Full batches run without
+  // bounds checks; the rows of a last, short batch one at a time.
+  const int rstride = P.ldk / 2;  // float2 per row
   const int first = half == 0 ? nr - 1 : 0;
   float2* dp = reinterpret_cast<float2*>(P.d + (static_cast<size_t>(b) * P.rows + r0 + first) * P.ldk + c0);
   const float* gp = gs + first * RP;
-  const int gstep = half == 0 ? -RP : RP;
   float acc0 = 0.f, acc1 = 0.f;
-  const float sgn = half == 0 ? -inv_norm : inv_norm;
+  auto walk = [&](auto dir) {
+    constexpr int kDir = decltype(dir)::value;  // -1: first half (backwards), +1: second half
+    constexpr int kBatch = 8;
+    const float sgn = kDir < 0 ? -inv_norm : inv_norm;
+    const int nfull = nr / kBatch;
 #pragma unroll 1
-  for (int r = 0; r < nr; r += kBatch) {
-    const int n = min(kBatch, nr - r);
-    float l0[kBatch], l1[kBatch];
+    for (int bt = 0; bt < nfull; ++bt) {
+      float l0[kBatch], l1[kBatch];
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i)
-      if (i < n) log2_alpha(gp + i * gstep, l0[i], l1[i]);
+      for (int i = 0; i < kBatch; ++i) log2_alpha(gp + kDir * i * RP, l0[i], l1[i]);
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      if (i >= n) break;
-      const float a0 = acc0 + l0[i], a1 = acc1 + l1[i];
-      dp[i * step] = make_float2((half == 0 ? acc0 : a0) * sgn, (half == 0 ? acc1 : a1) * sgn);
+      for (int i = 0; i < kBatch; ++i) {
+        const float a0 = acc0 + l0[i], a1 = acc1 + l1[i];
+        dp[kDir * i * rstride] = kDir < 0 ? make_float2(acc0 * sgn, acc1 * sgn) : make_float2(a0 * sgn, a1 * sgn);
+        acc0 = a0;
+        acc1 = a1;
+      }
+      dp += kDir * kBatch * rstride;
+      gp += kDir * kBatch * RP;
+    }
+#pragma unroll 1
+    for (int r = nfull * kBatch; r < nr; ++r) {
+      float l0, l1;
+      log2_alpha(gp, l0, l1);
+      const float a0 = acc0 + l0, a1 = acc1 + l1;
+      *dp = kDir < 0 ? make_float2(acc0 * sgn, acc1 * sgn) : make_float2(a0 * sgn, a1 * sgn);
       acc0 = a0;
       acc1 = a1;
+      dp += kDir * rstride;
+      gp += kDir * RP;
     }
-    dp += kBatch * step;
-    gp += kBatch * gstep;
-  }
+  };
+  if (half == 0)
+    walk(std::integral_constant<int, -1>());
+  else
+    walk(std::integral_constant<int, 1>());
   const size_t gi = (static_cast<size_t>(b) * P.n_chunks + chunk) * P.ldk + c0;
   if (half == 0) {
     *reinterpret_cast<float2*>(P.mid + gi) = make_float2(ex2_approx(acc0 * inv_norm), ex2_approx(acc1 * inv_norm));
