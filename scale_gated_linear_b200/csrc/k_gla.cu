@@ -8,25 +8,30 @@
 // Chunks hold C = 128 rows. With b_i the cumulative log forget gate from the
 // chunk's first row and m = b at its 64th row (the reference point), the gate
 // kernel supplies Qs = q e^{b - m}, Ks = k e^{m - b}, gamma = e^{b_last - m} and
-// mid = e^{m} per chunk and key channel. TMEM holds the scaled state
-// S' = Diag(e^{m_c}) S_{c-1} on entry to chunk c; per chunk:
-//   A     = Qs Ks^T, masked to j <= i            (scores, fp32 in TMEM)
-//   o     = Qs S' + A V                          (S' in shared memory as fp16,
-//                                                 A converted to fp16 in TMEM)
-//   S'   += Ks^T V
-//   S'   <- Diag(gamma_c mid_{c+1}) S'           (epilogue, in TMEM)
-// so every exponent stays within half a chunk's decay and every MMA is
-// M = 128, N = 128.
+// mid = e^{m} per chunk and key channel. TMEM holds the transposed scaled state
+// T = S'^T, S' = Diag(e^{m_c}) S_{c-1}, on entry to chunk c (value columns on
+// the TMEM lanes, key channels on the columns); per chunk:
+//   [A | o] = Qs [Ks ; T]^T                 one N = 256 product: the scores
+//                                            A = Qs Ks^T (masked to j <= i) and
+//                                            o = Qs S', reading Qs once
+//   T      += V^T Ks                         per 128-channel half of d_k
+//   o      += A V                            (A converted to fp16 in TMEM)
+//   T      <- T Diag(gamma_c mid_{c+1})      (epilogue, in TMEM)
+// so every exponent stays within half a chunk's decay. The tensor cores read
+// their shared-memory operands at about 64 bytes per clock, which bounds the
+// chunk loop; the fused product and the transposed state keep those reads at
+// 352 KB per chunk (Qs 64, [Ks ; T] 128, V^T 2 x 32, Ks 64, V 32).
 //
 // One CTA = (batch, branch, head, 128-column value tile), looping over chunks:
 //   warp 0        TMA loads of Qs, Ks (128 x dkp) and V (128 x 128)
 //   warp 1        TMEM allocation (512 columns) + tcgen05.mma issue
 //   warps 4..7    score epilogue (mask, fp16 back into TMEM) and the o store
 //                 (staged in the V buffer once A V is done, TMA tile stores)
-//   warps 8..15   state epilogue: S' <- factor * S' in TMEM and its fp16 copy
-//                 for the next chunk's Qs S' product (d_k rows 0..127 / 128..255)
-// TMEM columns: [0,256) S' (two 128-lane halves of d_k), [256,384) o,
-// [384,512) A (fp32; its fp16 form occupies [384,448)).
+//   warps 8..15   state epilogue: T <- T * factor in TMEM and its fp16 copy,
+//                 which sits right after each Ks atom in shared memory so that
+//                 [Ks ; T] is one K-major operand (d_k half 0 / half 1)
+// TMEM columns: [0,256) T (d_k channels), [256,384) A (fp32; its fp16 form
+// occupies [256,320)), [384,512) o.
 #include "msgla_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -37,18 +42,22 @@ constexpr int kThreads = 512;
 constexpr int kC = kGlaChunk;                 // 128 rows per chunk
 constexpr int kAtom = kC * 128;               // 128 rows x 128 bytes = 16 KB (64 16-bit columns)
 constexpr int kOffQ = 0;                      // Qs: up to 4 atoms (d_k <= 256)
-constexpr int kOffK = kOffQ + 4 * kAtom;      // Ks: up to 4 atoms
-constexpr int kOffV = kOffK + 4 * kAtom;      // V: 2 atoms (128 value columns)
-constexpr int kOffS = kOffV + 2 * kAtom;      // S' fp16: 2 MN blocks x 256 rows x 128 B
-constexpr int kOffBar = kOffS + 2 * 256 * 128;
-constexpr int kSmemBytes = kOffBar + 256 + 1024;
+constexpr int kOffKT = kOffQ + 4 * kAtom;     // per 64-channel block ka: Ks atom, then the T atom
+constexpr int kOffV = kOffKT + 8 * kAtom;     // V: 2 atoms (128 value columns)
+constexpr int kOffBar = kOffV + 2 * kAtom;
+constexpr int kOffF = kOffBar + 256;          // the chunk's 256 state factors
+constexpr int kSmemBytes = kOffF + 256 * 4 + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-constexpr uint32_t kColS = 0, kColO = 256, kColA = 384;
+constexpr uint32_t kColS = 0, kColA = 256, kColO = 384;
 
+// Ks, T and the state epilogue are split by 128-channel half h of d_k (the
+// barrier + h), so the refill of a Ks half and the epilogue of a state half
+// start as soon as that half's update has completed.
 enum {
-  B_Q_FULL = 0, B_Q_EMPTY, B_K_FULL, B_K_EMPTY, B_V_FULL, B_V_EMPTY,
-  B_A_FULL, B_A_READY, B_O_FULL, B_O_EMPTY, B_S_FULL, B_S_DONE, B_COUNT
+  B_Q_FULL = 0, B_Q_EMPTY, B_K_FULL, B_K_FULL1, B_K_EMPTY, B_K_EMPTY1, B_V_FULL, B_V_EMPTY,
+  B_A_FULL, B_A_READY, B_O_FULL, B_O_EMPTY, B_S_FULL, B_S_FULL1, B_S_DONE, B_S_DONE1,
+  B_F_READY, B_F_READY1, B_F_FREE, B_F_FREE1, B_COUNT
 };
 
 // D[tmem] (+)= A[tmem] * B[smem]^T (A K-major in TMEM, 16-bit pairs per column)
@@ -83,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
   const int head = (local / T.v_tiles) % T.heads;
   const int b = local / (T.v_tiles * T.heads);
   const int dkp = T.dkp;
-  const int n_half = dkp / 128;  // 1 or 2 state halves
+  const int n_half = dkp / 128;  // 1 or 2 halves of d_k
   const int nch_all = T.n_chunks;
   const int c_begin = seg * T.seg_chunks;
   const int nch = min(T.seg_chunks, nch_all - c_begin);  // chunks of this CTA
@@ -96,7 +105,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
     for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], 1);
     mbar_init(&bar[B_A_READY], 128);
     mbar_init(&bar[B_O_EMPTY], 128);
-    mbar_init(&bar[B_S_DONE], 128 * n_half);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bar[B_S_DONE + h], 128);
+      mbar_init(&bar[B_F_READY + h], 128);
+      mbar_init(&bar[B_F_FREE + h], 128);
+    }
     // full pass: the four output warps release V once their staged o tile is read
     mbar_init(&bar[B_V_EMPTY], state_pass ? 1 : 4);
     *abort_flag = 0;
@@ -130,10 +143,15 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
           for (int ka = 0; ka < dkp / 64; ++ka)
             tma_load_3d(&T.tmQ, &bar[B_Q_FULL], smem + kOffQ + ka * kAtom, head * dkp + ka * 64, row, b);
         }
-        if (c > 0 && !mbar_wait(&bar[B_K_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(&bar[B_K_FULL], qk_bytes);
-        for (int ka = 0; ka < dkp / 64; ++ka)
-          tma_load_3d(&T.tmK, &bar[B_K_FULL], smem + kOffK + ka * kAtom, head * dkp + ka * 64, row, b);
+        bool ok = true;
+        for (int h = 0; h < n_half && ok; ++h) {
+          if (c > 0 && !mbar_wait(&bar[B_K_EMPTY + h], (c - 1) & 1, abort_flag, p.err)) ok = false;
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bar[B_K_FULL + h], 2 * kAtom);
+          for (int ka = 2 * h; ka < 2 * h + 2; ++ka)
+            tma_load_3d(&T.tmK, &bar[B_K_FULL + h], smem + kOffKT + ka * 2 * kAtom, head * dkp + ka * 64, row, b);
+        }
+        if (!ok) break;
         if (c > 0 && !mbar_wait(&bar[B_V_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(&bar[B_V_FULL], 2 * kAtom);
         for (int mb = 0; mb < 2; ++mb)
@@ -143,68 +161,63 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer. Per chunk: Qs S', S' update, A V, then the
-      // scores of the next chunk.
-      const uint32_t id_kk = idesc_f16(128, 128, 0, 0, 0);  // K-major x K-major
-      const uint32_t id_km = idesc_f16(128, 128, 0, 0, 1);  // K-major (smem or TMEM) x MN-major
-      const uint32_t id_mm = idesc_f16(128, 128, 0, 1, 1);  // MN-major x MN-major
-      const uint32_t sQ = sbase + kOffQ, sK = sbase + kOffK, sV = sbase + kOffV, sS = sbase + kOffS;
-      const uint32_t lbo_s = static_cast<uint32_t>(dkp) * 128;
+      // ---------------- MMA issuer
+      const uint32_t id_fused = idesc_f16(128, 256, 0, 0, 0);  // [A | o] = Qs [Ks ; T]^T
+      const uint32_t id_score = idesc_f16(128, 128, 0, 0, 0);  // A = Qs Ks^T (no state yet)
+      const uint32_t id_mm = idesc_f16(128, 128, 0, 1, 1);     // T += V^T Ks: both MN-major
+      const uint32_t id_km = idesc_f16(128, 128, 0, 0, 1);     // o += A V: A in TMEM, V MN-major
+      const uint32_t sQ = sbase + kOffQ, sKT = sbase + kOffKT, sV = sbase + kOffV;
       const uint32_t sd0 = has_init ? 1u : 0u;  // state-epilogue completions before chunk 0
+      // T += V^T Ks for the channels of half h (K = chunk rows j); releases that
+      // Ks half and hands the half to the state epilogue
+      auto state_update = [&](int h, bool acc) {
+        for (int ks = 0; ks < kC / 16; ++ks)
+          umma_f16(tmem + kColS + h * 128, sdesc_sw128(sV + ks * 2048, kAtom, 1024),
+                   sdesc_sw128(sKT + h * 4 * kAtom + ks * 2048, 2 * kAtom, 1024), id_mm, (acc || ks > 0) ? 1u : 0u);
+        umma_commit(&bar[B_K_EMPTY + h]);
+        umma_commit(&bar[B_S_FULL + h]);
+      };
       for (int c = 0; c < nch && state_pass; ++c) {
-        // state pass: S' += Ks^T V and the state epilogue only
+        // state pass: the state update and the state epilogue only
         const uint32_t ph = c & 1;
-        if (!mbar_wait(&bar[B_K_FULL], ph, abort_flag, p.err)) break;
         if (!mbar_wait(&bar[B_V_FULL], ph, abort_flag, p.err)) break;
-        if (c > 0 && !mbar_wait(&bar[B_S_DONE], (c - 1) & 1, abort_flag, p.err)) break;
-        tc_fence_after();
-        for (int h = 0; h < n_half; ++h)
-          for (int ks = 0; ks < kC / 16; ++ks)
-            umma_f16(tmem + kColS + h * 128, sdesc_sw128(sK + 2 * h * kAtom + ks * 2048, kAtom, 1024),
-                     sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_mm, (c > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(&bar[B_S_FULL]);
-        umma_commit(&bar[B_K_EMPTY]);
+        bool ok = true;
+        for (int h = 0; h < n_half && ok; ++h) {
+          ok = mbar_wait(&bar[B_K_FULL + h], ph, abort_flag, p.err) &&
+               (c == 0 || mbar_wait(&bar[B_S_DONE + h], (c - 1) & 1, abort_flag, p.err));
+          if (!ok) break;
+          tc_fence_after();
+          state_update(h, c > 0);
+        }
+        if (!ok) break;
         umma_commit(&bar[B_V_EMPTY]);
       }
-      // Full pass. The scores of chunk c + 1 are issued right after the A V
-      // product of chunk c, so their conversion overlaps the Qs S' and S' update
-      // products of chunk c + 1, and the o drain and state epilogue of chunk c
-      // overlap the next scores: per chunk the chain is the scores, Qs S' and
-      // the S' update, plus the wait for the next K tile.
-      auto scores = [&](int c) {  // A = Qs Ks^T  (K = d_k)
-        for (int ks = 0; ks < dkp / 16; ++ks)
-          umma_f16(tmem + kColA, sdesc_sw128(sQ + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024),
-                   sdesc_sw128(sK + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024), id_kk, ks > 0);
-        umma_commit(&bar[B_A_FULL]);
-      };
-      if (!state_pass && nch > 0) {
-        if (mbar_wait(&bar[B_Q_FULL], 0, abort_flag, p.err) && mbar_wait(&bar[B_K_FULL], 0, abort_flag, p.err)) {
-          tc_fence_after();
-          scores(0);
-        }
-      }
+      // Full pass, per chunk c in pipe order: the fused scores + Qs S' product
+      // (first d_k half while the second half of Ks may still be loading), the
+      // state update per half, then A V. The score conversion overlaps the
+      // update; the state epilogue of each half overlaps what follows it.
       for (int c = 0; c < nch && !state_pass; ++c) {
-        const uint32_t ph = c & 1, pp = (c - 1) & 1;
+        const uint32_t ph = c & 1;
         const bool carried = c > 0 || has_init;  // a state enters this chunk
-        if (carried) {
-          if (!mbar_wait(&bar[B_S_DONE], (c - 1 + sd0) & 1, abort_flag, p.err)) break;
-          if (c > 0 && !mbar_wait(&bar[B_O_EMPTY], pp, abort_flag, p.err)) break;
+        if (!mbar_wait(&bar[B_Q_FULL], ph, abort_flag, p.err)) break;
+        if (c > 0 && !mbar_wait(&bar[B_O_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
+        bool ok = true;
+        for (int h = 0; h < n_half && ok; ++h) {
+          ok = mbar_wait(&bar[B_K_FULL + h], ph, abort_flag, p.err) &&
+               (!carried || mbar_wait(&bar[B_S_DONE + h], (c - 1 + sd0) & 1, abort_flag, p.err));
+          if (!ok) break;
           tc_fence_after();
-          // o = Qs S'  (K = d_k)
-          for (int ks = 0; ks < dkp / 16; ++ks)
-            umma_f16(tmem + kColO, sdesc_sw128(sQ + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024),
-                     sdesc_sw128(sS + ks * 2048, lbo_s, 1024), id_km, ks > 0);
+          for (int ks = 8 * h; ks < 8 * h + 8; ++ks)
+            umma_f16(tmem + kColA, sdesc_sw128(sQ + (ks >> 2) * kAtom + (ks & 3) * 32, 16, 1024),
+                     sdesc_sw128(sKT + (ks >> 2) * 2 * kAtom + (ks & 3) * 32, 16, 1024),
+                     carried ? id_fused : id_score, ks > 0 ? 1u : 0u);
         }
-        umma_commit(&bar[B_Q_EMPTY]);  // Qs of chunk c: scores and Qs S' issued
+        if (!ok) break;
+        umma_commit(&bar[B_Q_EMPTY]);
+        umma_commit(&bar[B_A_FULL]);
         if (!mbar_wait(&bar[B_V_FULL], ph, abort_flag, p.err)) break;
         tc_fence_after();
-        // S' += Ks^T V per 128-row half of d_k  (K = chunk rows j)
-        for (int h = 0; h < n_half; ++h)
-          for (int ks = 0; ks < kC / 16; ++ks)
-            umma_f16(tmem + kColS + h * 128, sdesc_sw128(sK + 2 * h * kAtom + ks * 2048, kAtom, 1024),
-                     sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_mm, (carried || ks > 0) ? 1u : 0u);
-        umma_commit(&bar[B_S_FULL]);
-        umma_commit(&bar[B_K_EMPTY]);
+        for (int h = 0; h < n_half; ++h) state_update(h, carried);
         if (!mbar_wait(&bar[B_A_READY], ph, abort_flag, p.err)) break;
         tc_fence_after();
         // o += A V  (A fp16 in TMEM, 8 columns per 16 rows j)
@@ -212,12 +225,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
           umma_f16_ts(tmem + kColO, tmem + kColA + ks * 8, sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_km,
                       (carried || ks > 0) ? 1u : 0u);
         umma_commit(&bar[B_O_FULL]);
-        if (c + 1 < nch) {
-          if (!mbar_wait(&bar[B_Q_FULL], ph ^ 1, abort_flag, p.err)) break;
-          if (!mbar_wait(&bar[B_K_FULL], ph ^ 1, abort_flag, p.err)) break;
-          tc_fence_after();
-          scores(c + 1);
-        }
       }
     }
   } else if (warp >= 4 && warp < 8) {
@@ -299,64 +306,72 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
       fence_proxy_async_global();
     }
   } else if (warp >= 8) {
-    // ---------------- state epilogue: S' <- gamma_c mid_{c+1} S', fp16 copy in smem
-    const int g = (warp - 8) >> 2;  // d_k half
+    // ---------------- state epilogue of d_k half g: T <- T Diag(gamma_c mid_{c+1})
+    // for channels [128 g, 128 g + 128) of value row v, and the fp16 copy of
+    // those T entries after the matching Ks atoms
+    const int g = (warp - 8) >> 2;
     const int quad = warp & 3;
     if (g < n_half) {
-      const int a = g * 128 + quad * 32 + lane;  // d_k row
-      uint8_t* sS = smem + kOffS;
+      const int v = quad * 32 + lane;            // value column of the tile (TMEM lane)
+      const int a_own = g * 128 + quad * 32 + lane;  // channel whose factor this thread supplies
+      float* fac = reinterpret_cast<float*>(smem + kOffF);
       const size_t ld_g = static_cast<size_t>(T.heads) * dkp;
-      const float* gp = T.gamma + static_cast<size_t>(b) * nch_all * ld_g + head * dkp + a;
-      const float* mp = T.mid + static_cast<size_t>(b) * nch_all * ld_g + head * dkp + a;
+      const float* gp = T.gamma + static_cast<size_t>(b) * nch_all * ld_g + head * dkp + a_own;
+      const float* mp = T.mid + static_cast<size_t>(b) * nch_all * ld_g + head * dkp + a_own;
       // factor of global chunk cg: gamma_cg * mid_{cg+1} (1 past the sequence's end)
       auto factor = [&](int cg) {
         return __ldg(gp + static_cast<size_t>(cg) * ld_g) *
                (cg + 1 < nch_all ? __ldg(mp + static_cast<size_t>(cg + 1) * ld_g) : 1.f);
       };
-      // fp16 copy of 64 value columns (q2-th MN block) of row a for the o = Qs S' product
-      auto put_f16 = [&](int q2, const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
-        uint8_t* row = sS + q2 * dkp * 128 + a * 128;
+      // fp16 copy of 64 channels (block ka) of row v: the rows 128..255 of the
+      // K-major [Ks ; T] operand, with the 128-byte swizzle of the Ks atoms
+      auto put_f16 = [&](int ka, const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
+        uint8_t* row = smem + kOffKT + ka * 2 * kAtom + kAtom + v * 128;
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           const uint32_t* r = e4 < 4 ? ra + 8 * e4 : rb + 8 * (e4 - 4);
-          st_shared_v4(smem_u32(row + ((e4 ^ (a & 7)) << 4)), pack_half2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+          st_shared_v4(smem_u32(row + ((e4 ^ (v & 7)) << 4)), pack_half2(__uint_as_float(r[0]), __uint_as_float(r[1])),
                        pack_half2(__uint_as_float(r[2]), __uint_as_float(r[3])),
                        pack_half2(__uint_as_float(r[4]), __uint_as_float(r[5])),
                        pack_half2(__uint_as_float(r[6]), __uint_as_float(r[7])));
         }
       };
+      // segment states are stored [channel a][value column v]
+      float* seg_base = state_pass || has_init ? T.seg_state + (seq_slot + seg - (has_init ? 1 : 0)) * dkp * kGlaTile + v
+                                               : nullptr;
       if (has_init) {
         // carried state of this segment (written by the scan) into TMEM and smem
-        const float4* src =
-            reinterpret_cast<const float4*>(T.seg_state + ((seq_slot + seg - 1) * dkp + a) * kGlaTile);
 #pragma unroll 1
         for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t ra[32], rb[32];
+          const float* src = seg_base + static_cast<size_t>(g * 128 + q2 * 64) * kGlaTile;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 x = __ldg(src + q2 * 16 + e), y = __ldg(src + q2 * 16 + 8 + e);
-            ra[4 * e] = __float_as_uint(x.x), ra[4 * e + 1] = __float_as_uint(x.y);
-            ra[4 * e + 2] = __float_as_uint(x.z), ra[4 * e + 3] = __float_as_uint(x.w);
-            rb[4 * e] = __float_as_uint(y.x), rb[4 * e + 1] = __float_as_uint(y.y);
-            rb[4 * e + 2] = __float_as_uint(y.z), rb[4 * e + 3] = __float_as_uint(y.w);
+          for (int e = 0; e < 32; ++e) {
+            ra[e] = __float_as_uint(__ldg(src + e * kGlaTile));
+            rb[e] = __float_as_uint(__ldg(src + (32 + e) * kGlaTile));
           }
           const uint32_t ta = tmem_addr(tmem, quad * 32, kColS + g * 128 + q2 * 64);
           tmem_st32(ta, ra);
           tmem_st32(ta + 32, rb);
-          put_f16(q2, ra, rb);
+          put_f16(2 * g + q2, ra, rb);
         }
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&bar[B_S_DONE]);
+        mbar_arrive(&bar[B_S_DONE + g]);
       }
-      float decay = 1.f;  // product of this segment's factors (state pass)
+      float decay = 1.f;  // product of this segment's factors of channel a_own (state pass)
       float f = factor(c_begin);
-      for (int c = 0; c < nch; ++c) {
+      int c = 0;
+      for (; c < nch; ++c) {
         const float f_next = (c + 1 < nch) ? factor(c_begin + c + 1) : 0.f;
-        if (!mbar_wait(&bar[B_S_FULL], c & 1, abort_flag, p.err)) break;
+        // publish this chunk's factors once every thread of the half has read the last ones
+        if (c > 0 && !mbar_wait(&bar[B_F_FREE + g], (c - 1) & 1, abort_flag, p.err)) break;
+        fac[a_own] = f;
+        mbar_arrive(&bar[B_F_READY + g]);
+        if (!mbar_wait(&bar[B_F_READY + g], c & 1, abort_flag, p.err)) break;
+        if (!mbar_wait(&bar[B_S_FULL + g], c & 1, abort_flag, p.err)) break;
         tc_fence_after();
-        const bool last = c + 1 == nch;
 #pragma unroll 1
         for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t ra[32], rb[32];
@@ -364,35 +379,49 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
           tmem_ld32(ta, ra);
           tmem_ld32(ta + 32, rb);
           tmem_wait_ld();
+          const float4* fr = reinterpret_cast<const float4*>(fac + g * 128 + q2 * 64);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            ra[e] = __float_as_uint(f * __uint_as_float(ra[e]));
-            rb[e] = __float_as_uint(f * __uint_as_float(rb[e]));
+          for (int e = 0; e < 8; ++e) {
+            const float4 x = fr[e], y = fr[8 + e];
+            ra[4 * e] = __float_as_uint(x.x * __uint_as_float(ra[4 * e]));
+            ra[4 * e + 1] = __float_as_uint(x.y * __uint_as_float(ra[4 * e + 1]));
+            ra[4 * e + 2] = __float_as_uint(x.z * __uint_as_float(ra[4 * e + 2]));
+            ra[4 * e + 3] = __float_as_uint(x.w * __uint_as_float(ra[4 * e + 3]));
+            rb[4 * e] = __float_as_uint(y.x * __uint_as_float(rb[4 * e]));
+            rb[4 * e + 1] = __float_as_uint(y.y * __uint_as_float(rb[4 * e + 1]));
+            rb[4 * e + 2] = __float_as_uint(y.z * __uint_as_float(rb[4 * e + 2]));
+            rb[4 * e + 3] = __float_as_uint(y.w * __uint_as_float(rb[4 * e + 3]));
           }
           tmem_st32(ta, ra);
           tmem_st32(ta + 32, rb);
-          if (!state_pass) {
-            put_f16(q2, ra, rb);
-          } else if (last) {
-            // end state of this segment (from zero) for the scan
-            float4* dst = reinterpret_cast<float4*>(T.seg_state + ((seq_slot + seg) * dkp + a) * kGlaTile) + q2 * 16;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              dst[e] = make_float4(__uint_as_float(ra[4 * e]), __uint_as_float(ra[4 * e + 1]),
-                                   __uint_as_float(ra[4 * e + 2]), __uint_as_float(ra[4 * e + 3]));
-              dst[8 + e] = make_float4(__uint_as_float(rb[4 * e]), __uint_as_float(rb[4 * e + 1]),
-                                       __uint_as_float(rb[4 * e + 2]), __uint_as_float(rb[4 * e + 3]));
-            }
-          }
+          if (!state_pass) put_f16(2 * g + q2, ra, rb);
         }
+        mbar_arrive(&bar[B_F_FREE + g]);
         decay *= f;
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&bar[B_S_DONE]);
+        mbar_arrive(&bar[B_S_DONE + g]);
         f = f_next;
       }
-      if (state_pass) T.seg_decay[(seq_slot + seg) * dkp + a] = decay;
+      if (state_pass && c == nch) {
+        // end state of this segment (from zero) and its decay, for the scan
+#pragma unroll 1
+        for (int q2 = 0; q2 < 2; ++q2) {
+          uint32_t ra[32], rb[32];
+          const uint32_t ta = tmem_addr(tmem, quad * 32, kColS + g * 128 + q2 * 64);
+          tmem_ld32(ta, ra);
+          tmem_ld32(ta + 32, rb);
+          tmem_wait_ld();
+          float* dst = seg_base + static_cast<size_t>(g * 128 + q2 * 64) * kGlaTile;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            dst[e * kGlaTile] = __uint_as_float(ra[e]);
+            dst[(32 + e) * kGlaTile] = __uint_as_float(rb[e]);
+          }
+        }
+        T.seg_decay[(seq_slot + seg) * dkp + a_own] = decay;
+      }
     }
   }
   tc_fence_before();
