@@ -482,23 +482,6 @@ __global__ void __launch_bounds__(256) head_norm_kernel(const HeadNormParams p) 
 // kHoldRows rows, block of up to 256 column groups): thread (r, cg) takes 8
 // columns of rows t0 + r, t0 + r + R, ...; no division in the loop (the held
 // row index is a shift for power-of-two scales).
-// Packed fp32 pairs (two IEEE fp32 operations per instruction, round to nearest).
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-
 // One item per (branch, sequence, half of a 128-row chunk, block of 256 key
 // channels), a CTA of 128 threads; thread t owns channels c0 + 2t, c0 + 2t + 1.
 //  1. The half's 64 gate inputs g (rank RP) go to shared memory: a scale-1

@@ -26,7 +26,7 @@
 //   warp 0        TMA loads of Qs, Ks (128 x dkp) and V (128 x 128)
 //   warp 1        TMEM allocation (512 columns) + tcgen05.mma issue
 //   warps 4..7    score epilogue (mask, fp16 back into TMEM) and the o store
-//                 (staged in the V buffer once A V is done, TMA tile stores)
+//                 (staged in the V buffer once V is read, TMA tile stores)
 //   warps 8..15   state epilogue: T <- T * factor in TMEM and its fp16 copy,
 //                 which sits right after each Ks atom in shared memory so that
 //                 [Ks ; T] is one K-major operand (d_k half 0 / half 1)
@@ -57,7 +57,7 @@ constexpr uint32_t kColS = 0, kColA = 256, kColO = 384;
 enum {
   B_Q_FULL = 0, B_Q_EMPTY, B_K_FULL, B_K_FULL1, B_K_EMPTY, B_K_EMPTY1, B_V_FULL, B_V_EMPTY,
   B_A_FULL, B_A_READY, B_O_FULL, B_O_EMPTY, B_S_FULL, B_S_FULL1, B_S_DONE, B_S_DONE1,
-  B_F_READY, B_F_READY1, B_F_FREE, B_F_FREE1, B_COUNT
+  B_F_READY, B_F_READY1, B_F_FREE, B_F_FREE1, B_V_FREE, B_COUNT
 };
 
 // D[tmem] (+)= A[tmem] * B[smem]^T (A K-major in TMEM, 16-bit pairs per column)
@@ -194,8 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
       }
       // Full pass, per chunk c in pipe order: the fused scores + Qs S' product
       // (first d_k half while the second half of Ks may still be loading), the
-      // state update per half, then A V. The score conversion overlaps the
-      // update; the state epilogue of each half overlaps what follows it.
+      // state update of d_k half 0, A V, then the update of half 1. The score
+      // conversion overlaps the first update, the o drain the second, and the
+      // state epilogue of each half what follows it, so the next chunk's fused
+      // product finds its inputs ready.
       for (int c = 0; c < nch && !state_pass; ++c) {
         const uint32_t ph = c & 1;
         const bool carried = c > 0 || has_init;  // a state enters this chunk
@@ -217,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
         umma_commit(&bar[B_A_FULL]);
         if (!mbar_wait(&bar[B_V_FULL], ph, abort_flag, p.err)) break;
         tc_fence_after();
-        for (int h = 0; h < n_half; ++h) state_update(h, carried);
+        state_update(0, carried);
         if (!mbar_wait(&bar[B_A_READY], ph, abort_flag, p.err)) break;
         tc_fence_after();
         // o += A V  (A fp16 in TMEM, 8 columns per 16 rows j)
@@ -225,6 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
           umma_f16_ts(tmem + kColO, tmem + kColA + ks * 8, sdesc_sw128(sV + ks * 2048, kAtom, 1024), id_km,
                       (carried || ks > 0) ? 1u : 0u);
         umma_commit(&bar[B_O_FULL]);
+        for (int h = 1; h < n_half; ++h) state_update(h, carried);
+        umma_commit(&bar[B_V_FREE]);  // V is read: the o rows may be staged there
       }
     }
   } else if (warp >= 4 && warp < 8) {
@@ -261,11 +265,13 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
 
       if (!mbar_wait(&bar[B_O_FULL], c & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      // o rows of this warp, scaled and rounded to fp16, staged in the V buffer
-      // (free: A V has completed) with the 128-byte swizzle of the TMA store,
-      // which writes whole 128-byte rows instead of 16-byte pieces of 32 rows
-      uint8_t* stage = smem + kOffV + quad * 8192;
-#pragma unroll 1
+      // o row i, scaled and rounded to fp16 in registers; the o columns are
+      // released at once, then the rows are staged in the V buffer (once the
+      // state update has read it) with the 128-byte swizzle of the TMA store,
+      // which writes whole 128-byte rows
+      uint32_t po[64];
+      const float qs = p.qk_scale;
+#pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         uint32_t ra[32], rb[32];
         const uint32_t src = tmem_addr(tmem, quad * 32, kColO + h2 * 64);
@@ -273,20 +279,23 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
         tmem_ld32(src + 32, rb);
         tmem_wait_ld(ra);
         tmem_wait_ld(rb);
-        if (h2 == 1) {
-          tc_fence_before();
-          mbar_arrive(&bar[B_O_EMPTY]);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          po[32 * h2 + e] = half2_of_mul(ra[2 * e], ra[2 * e + 1], qs, qs);
+          po[32 * h2 + 16 + e] = half2_of_mul(rb[2 * e], rb[2 * e + 1], qs, qs);
         }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar[B_O_EMPTY]);
+      if (!mbar_wait(&bar[B_V_FREE], c & 1, abort_flag, p.err)) break;
+      uint8_t* stage = smem + kOffV + quad * 8192;
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
         uint8_t* row = stage + h2 * 4096 + lane * 128;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint32_t* r = q < 4 ? ra + 8 * q : rb + 8 * (q - 4);
-          st_shared_v4(smem_u32(row + ((q ^ (lane & 7)) << 4)),
-                       pack_half2(p.qk_scale * __uint_as_float(r[0]), p.qk_scale * __uint_as_float(r[1])),
-                       pack_half2(p.qk_scale * __uint_as_float(r[2]), p.qk_scale * __uint_as_float(r[3])),
-                       pack_half2(p.qk_scale * __uint_as_float(r[4]), p.qk_scale * __uint_as_float(r[5])),
-                       pack_half2(p.qk_scale * __uint_as_float(r[6]), p.qk_scale * __uint_as_float(r[7])));
-        }
+        for (int q = 0; q < 8; ++q)
+          st_shared_v4(smem_u32(row + ((q ^ (lane & 7)) << 4)), po[32 * h2 + 4 * q], po[32 * h2 + 4 * q + 1],
+                       po[32 * h2 + 4 * q + 2], po[32 * h2 + 4 * q + 3]);
       }
       fence_proxy_async_smem();
       __syncwarp();
