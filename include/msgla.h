@@ -262,8 +262,11 @@ int msgla_step(msgla_handle* h, void* cache, const void* x, int B, long long t, 
 
 /* Kernels that msgla_forward launches for a [B, L, d] input, in launch order, as a
  * comma-separated list written to `names` (NUL-terminated, at most `len` bytes):
- * pool_fuse, proj_gemm, gate, [gla_state, gla_scan], gla, [head_norm],
- * [out_gemm_coarse], out_gemm_fused | out_gemm_coarse, hold_fuse. gla_state and
+ * pool_u | (gate_inputs, [pool]), gate, proj_gemm, [gla_state, gla_scan], gla,
+ * [head_norm], [out_gemm_coarse], out_gemm_fused | out_gemm_coarse, hold_fuse.
+ * pool_u (one pass over X for the pooled rows, the fusion logits and the gate
+ * inputs) runs when every coarse scale is a power of two up to 8; otherwise a
+ * GEMM for the gate inputs and a pooling kernel do its work. gla_state and
  * gla_scan appear when long sequences are cut into segments (few sequences: the
  * GLA kernel would fill less than half of the GPU); head_norm when the config
  * enables the head RMS norm. out_gemm_coarse is absent when it runs on the
