@@ -512,6 +512,8 @@ __global__ void __launch_bounds__(kGateThreads) gate_kernel(const __grid_constan
   griddep_wait();
   griddep_launch();
   if (p.clear && blockIdx.x == 0 && threadIdx.x == 0) *p.clear = 0ull;
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < p.n_clear_rows; i += blockDim.x) p.clear_rows[i] = 0ull;
 #pragma unroll 1
   for (int item = blockIdx.x; item < p.total_blocks; item += gridDim.x) {
     gate_item<RP>(p, item, gs);

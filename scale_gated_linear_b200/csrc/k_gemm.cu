@@ -577,6 +577,18 @@ __device__ __forceinline__ bool epilogue_qk(const GemmParams& p, const TileCoord
   return true;
 }
 
+// After a kEpiProjGate tile: once this warp's TMA stores have completed, count
+// the warp's 32 rows in the 128-row block's counter (GemmParams::rows_done), with
+// release order for the GLA kernel's acquire.
+__device__ __forceinline__ void count_rows_done(const GemmParams& p, const TileCoord& tc, int lane) {
+  const GemmTask& T = p.task[tc.task];
+  if (!p.rows_done || T.epi != kEpiProjGate || lane != 0 || tc.m0 >= T.rows) return;
+  bulk_wait0();
+  fence_proxy_async_global();
+  __threadfence();
+  atomicAdd(p.rows_done + T.done_base + static_cast<size_t>(tc.b) * ((T.rows + 127) / 128) + tc.m0 / 128, 1ull);
+}
+
 // Prefetch the output tensor maps of every task (epilogue warps).
 __device__ __forceinline__ void prefetch_out_maps(const GemmParams& p) {
   for (int t = 0; t < p.n_tasks; ++t) {
@@ -728,6 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
+      count_rows_done(p, tc, lane);
     }
     if (lane == 0) bulk_wait0();
   }
@@ -1022,6 +1035,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
       }
       tc_fence_before();
       mbar_arrive_cluster(buf ? lead_empty1 : lead_empty0);
+      if (!kHeld) count_rows_done(p, tc, lane);
     }
     if (lane == 0) bulk_wait0();
   }

@@ -111,7 +111,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_wait();
+  // with per-chunk counters the producer waits for each chunk's operands itself
+  const bool chunk_waits = p.rows_done && !state_pass;
+  if (!chunk_waits) griddep_wait();
   griddep_launch();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
@@ -126,6 +128,13 @@ __global__ void __launch_bounds__(kThreads, 1) gla_chunk_kernel(const __grid_con
       const uint32_t qk_bytes = static_cast<uint32_t>((dkp / 64) * kAtom);
       for (int c = 0; c < nch; ++c) {
         const int row = (c_begin + c) * kC;
+        if (chunk_waits) {
+          // Qs, Ks and v of the chunk's rows are stored by the projection
+          if (!wait_count(p.rows_done + T.done_base + static_cast<size_t>(b) * nch_all + c_begin + c, T.done_target,
+                          abort_flag, p.err))
+            break;
+          fence_proxy_async_global();
+        }
         if (!state_pass) {  // the state pass reads only Ks and V
           if (c > 0 && !mbar_wait(&bar[B_Q_EMPTY], (c - 1) & 1, abort_flag, p.err)) break;
           mbar_arrive_expect_tx(&bar[B_Q_FULL], qk_bytes);

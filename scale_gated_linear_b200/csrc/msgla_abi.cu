@@ -199,6 +199,11 @@ struct BranchWs {
 struct Workspace {
   BranchWs br[MSGLA_MAX_SCALES];
   Region w, u;
+  // the projection's per-chunk completion counters (u64): branch j's at
+  // rows_base[j] + b * n_chunks + c
+  Region rows_done;
+  int rows_base[MSGLA_MAX_SCALES];
+  int n_rows_done = 0;
   size_t total = 0;
 };
 
@@ -263,6 +268,11 @@ Workspace layout(const msgla_handle* h, int B, int L) {
   }
   add(ws.w, cur, BB * L * h->n_scales * 4);
   add(ws.u, cur, BB * L * h->ldu * 4);
+  for (int j = 0; j < h->n_scales; ++j) {
+    ws.rows_base[j] = ws.n_rows_done;
+    ws.n_rows_done += B * ws.br[j].n_chunks;
+  }
+  add(ws.rows_done, cur, static_cast<size_t>(ws.n_rows_done) * 8);
   ws.total = cur;
   return ws;
 }
@@ -621,6 +631,8 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     g.inv_normalizer = 1.f / c.gate_normalizer;
     g.err = h->d_err;
     g.clear = h->d_gla_done + MSGLA_MAX_SCALES + 1;  // GLA exit counter
+    g.clear_rows = static_cast<unsigned long long*>(at(ws.rows_done));
+    g.n_clear_rows = ws.n_rows_done;
     CUDA_TRY(launch_gate(g, st));
     CUDA_TRY(rec->mark(st));
   }
@@ -650,6 +662,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.ab_bf16 = bf ? 1 : 0;
     t.epi = kEpiProjGate;
     t.dkp = h->dkp;
+    t.done_base = ws.rows_base[j];
     t.gd = static_cast<const float*>(at(bw.gd));
     t.mask = bf ? M : nullptr;
     if (!encode_f32_2d_32(&t.tmD, at(bw.gd), t.nq, static_cast<uint64_t>(B) * bw.rows) ||
@@ -661,6 +674,10 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   }
   gp.n_tasks = ns;
   gp.total_tiles = tiles;
+  // an unsegmented GLA starts each chunk once the projection has counted its rows
+  bool any_seg = false;
+  for (int j = 0; j < ns; ++j) any_seg |= ws.br[j].n_segs > 1;
+  if (!any_seg) gp.rows_done = static_cast<unsigned long long*>(at(ws.rows_done));
   CUDA_TRY(launch_gemm(gp, 256, st));
   CUDA_TRY(rec->mark(st));
 
@@ -692,6 +709,8 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
     t.v_tiles = h->dvp / kGlaTile;
     t.seg_chunks = bw.seg_chunks;
     t.n_segs = bw.n_segs;
+    t.done_base = ws.rows_base[j];
+    t.done_target = 8ull * gp.task[j].n_tiles;  // every epilogue warp of every N tile
     if (bw.n_segs > 1) {
       t.seg_state = static_cast<float*>(at(bw.seg_state));
       t.seg_decay = static_cast<float*>(at(bw.seg_decay));
@@ -725,6 +744,7 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   }
   lp.total_ctas = ctas;
   lp.mode = 0;
+  lp.rows_done = gp.rows_done;
   lp.skip_arrival = h->test_skip_arrival;
   h->test_skip_arrival = 0;
   long long gla_ctas = 0;

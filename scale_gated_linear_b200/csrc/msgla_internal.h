@@ -91,6 +91,9 @@ struct alignas(64) GemmTask {
   // columns. Outputs: Qs = q 2^d (tmQK[0]), Ks = k 2^-d (tmQK[1]), v (tmOut[2]).
   int n_qk, dkp;
   const float* gd;        // [B, rows, nq] gate exponents d = b - m (launch_gate)
+  // with GemmParams::rows_done: this task's counters start at rows_done[done_base],
+  // one per (batch element, 128-row block): [done_base + b * ceil(rows / 128) + m0 / 128]
+  int done_base, pad2_;
   // kEpiStoreF32: D -> f32 [B, rows, ldf]; with w set, also the fusion weights
   // w = softmax(D[:, 0:n_scales] + bfuse) (columns 0.. hold the fusion logits)
   float* f32;
@@ -122,6 +125,12 @@ struct GemmParams {
   unsigned int* tile_exit;
   unsigned long long* reset64;
   int n_reset64;
+  // non-null (the forward's projection): after its TMA stores of a kEpiProjGate
+  // tile have completed, every epilogue warp adds 1 (release) to the counter of
+  // the 128-row block it stored (GemmTask::done_base), so a block is complete at
+  // n_tiles * 8 -- the GLA kernel starts on a chunk as soon as its block is
+  // counted, instead of waiting for the whole launch
+  unsigned long long* rows_done;
 };
 
 // Chunkwise GLA over one or more branches.
@@ -138,6 +147,11 @@ struct alignas(64) GlaTask {
   float* seg_decay;    // [B, h, v_tiles, n_segs, dkp]: product of the state factors
   int rows, n_chunks, heads, dkp, dvp, v_tiles, cta_begin, seg_chunks, n_segs;
   int signal_done;  // full pass: this task's CTAs add 1 to GlaParams::done[task] when stored
+  // with GlaParams::rows_done: the projection's counters of this branch (one per
+  // batch element and 128-row chunk, at done_base + b * n_chunks + c) and the
+  // count at which a chunk's Qs, Ks and v are all stored
+  int done_base;
+  unsigned long long done_target;
 };
 
 struct GlaParams {
@@ -154,6 +168,12 @@ struct GlaParams {
   unsigned long long* done;
   unsigned long long* started;
   unsigned long long* exited;
+  // full pass of an unsegmented forward: the projection's per-chunk counters
+  // (GemmParams::rows_done). The kernel then does not wait for the projection
+  // launch to finish (no griddepcontrol.wait): a CTA takes an SM as soon as the
+  // projection's CTA there has left, and loads chunk c once its counter reaches
+  // the task's done_target (bounded wait). Null: wait for the launch.
+  const unsigned long long* rows_done;
 };
 // One warp on a second stream, ordered before a kernel that may only take SMs
 // once every CTA of a running GLA launch is resident: waits (bounded) until
@@ -241,6 +261,10 @@ struct GateParams {
   // set to zero before the forward's GLA launch (the GLA exit counter of the
   // overlapped coarse projection; null: none)
   unsigned long long* clear;
+  // the projection's per-chunk counters (GemmParams::rows_done), zeroed before the
+  // projection launch starts counting (null: none)
+  unsigned long long* clear_rows;
+  int n_clear_rows;
 };
 cudaError_t launch_gate(const GateParams& p, cudaStream_t st);
 
