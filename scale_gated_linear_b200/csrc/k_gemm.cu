@@ -80,7 +80,13 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int tile, 
   for (int t = 1; t < p.n_tasks; ++t)
     if (tile >= p.task[t].tile_begin) ti = t;
   const GemmTask& T = p.task[ti];
-  const int local = tile - T.tile_begin;
+  int local = tile - T.tile_begin;
+  int half = -1;  // >= 0: which 128-column half of a full tile (GemmTask::half_from)
+  if (T.half_from > 0 && local >= T.half_from) {
+    const int hl = local - T.half_from;
+    half = hl & 1;
+    local = T.half_from + (hl >> 1);
+  }
   const int n_tile = local % T.n_tiles;
   const int m_tile = (local / T.n_tiles) % T.m_tiles;
   c.task = ti;
@@ -108,6 +114,10 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int tile, 
   }
   const int n_rem = n_cols - c.n0;
   c.n_eff = n_rem >= bn ? bn : ((n_rem + 15) / 16) * 16;
+  if (half >= 0) {
+    c.n0 += 128 * half;
+    c.n_eff = 128;
+  }
   c.brow0 = b_first + c.n0;
   c.brow1 = c.brow0 + (c.n_eff >> 1);
   return c;
@@ -180,6 +190,10 @@ struct Held {
   uint64_t* empty;
   uint32_t parity;
   volatile int* abort_flag;
+  // a 128-column half tile: the column group of epilogue warps g reads box 2 g
+  // alone, and box 2 g + 1 carries nothing this tile (the loader completes its
+  // round with a plain arrival, the group releases it unread)
+  int half;
 };
 
 // Fusion weights w = softmax(z_t + b_fuse) of this thread's output row
@@ -332,7 +346,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, const TileCoo
       if (held) {
         // held coarse rows from shared memory: 16-byte pieces q of the chunk's
         // 64-column box, swizzled by the row
-        const int box = c0 >> 6, q0 = (c0 & 63) >> 3;
+        const int box = held->half ? (c0 >> 6) * 2 : c0 >> 6, q0 = (c0 & 63) >> 3;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           if (c >= T.n_coarse) break;
@@ -399,8 +413,9 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, const TileCoo
   tmem_wait_ld(va);
   for (int c0 = c_lo; c0 < c_hi; c0 += 64) {
     const bool has_b = c0 + 32 < c_hi, has_next = c0 + 64 < c_hi;
+    const int hb = held && held->half ? (c0 >> 6) * 2 : c0 >> 6;  // held box of these columns
     // held rows: this 64-column box has landed
-    if (held && !mbar_wait(&held->full[c0 >> 6], held->parity, held->abort_flag, p.err)) return false;
+    if (held && !mbar_wait(&held->full[hb], held->parity, held->abort_flag, p.err)) return false;
     if (has_b) tmem_ld32(tmem_addr(tacc, quad * 32, c0 + 32), vb);
     chunk(c0, va, 0, !has_b);
     if (has_b) {
@@ -413,7 +428,12 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, const TileCoo
       // this warp is done with the box: the loader may refill it for the next tile
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&held->empty[c0 >> 6]);
+      if (lane == 0) mbar_arrive(&held->empty[hb]);
+      if (held->half) {
+        // the sibling box of a half tile: complete its round unread
+        if (!mbar_wait(&held->full[hb + 1], held->parity, held->abort_flag, p.err)) return false;
+        if (lane == 0) mbar_arrive(&held->empty[hb + 1]);
+      }
     }
     sel ^= 1;
   }
@@ -968,15 +988,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
         const int m0 = tc.m0 + 128 * static_cast<int>(rank);
         // boxes in the order the epilogue releases them (the first 64 columns of
         // each column half first); each is refilled once its four warps are done
+        const bool half = tc.n_eff == 128;  // a half tile: boxes 0 and 2 hold its two 64-column blocks
         for (int q = 0; q < 4; ++q) {
           const int j = (q >> 1) | ((q & 1) << 1);  // 0, 2, 1, 3
           if (it >= 1 && !mbar_wait(&held_empty[j], (it - 1) & 1, abort_flag, p.err)) {
             ok = false;
             break;
           }
+          if (half && (j & 1)) {
+            mbar_arrive(&held_full[j]);  // nothing to load: complete the box's round
+            continue;
+          }
           mbar_arrive_expect_tx(&held_full[j], bytes);
+          const int col = tc.n0 + 64 * (half ? j >> 1 : j);
           for (int c = 0; c < 2 && c < T.n_coarse; ++c)
-            tma_load_3d(&T.tmOut[1 + c], &held_full[j], held_smem + held_off[c] + j * held_box[c], tc.n0 + 64 * j,
+            tma_load_3d(&T.tmOut[1 + c], &held_full[j], held_smem + held_off[c] + j * held_box[c], col,
                         held_base(m0, T.coarse_scale[c]), tc.b);
         }
       }
@@ -1023,6 +1049,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<kHeld>::k
         h.empty = held_empty;
         h.parity = it & 1;
         h.abort_flag = abort_flag;
+        h.half = tc.n_eff == 128;
         if (!epilogue_tile(p, tc, tmem + buf * kPairBN, quad, lane, lo, hi, padded, stg, sel, fw, &h)) break;
       } else if (!kHeld && tc.qk) {
         if (!epilogue_qk(p, tc, tmem + buf * kPairBN, quad, lane, (warp - 2) >= 4 ? 1 : 0, padded, stg, ge,
@@ -1122,6 +1149,15 @@ cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st, int max_pa
       T.n_tiles = T.epi == kEpiProjGate ? T.n_qk + (T.nv + kPairBN - 1) / kPairBN : (T.N + kPairBN - 1) / kPairBN;
       T.tile_begin = tiles;
       tiles += batches * T.m_tiles * T.n_tiles;
+    }
+    // the fused output launch: a last, partial wave of at most half the pairs runs
+    // as twice as many 128-column half tiles
+    if (held && tiles > pairs) {
+      const int full = tiles / pairs * pairs, rest = tiles - full;
+      if (rest > 0 && 2 * rest <= pairs) {
+        q.task[0].half_from = full;
+        tiles += rest;
+      }
     }
     q.total_tiles = tiles;
     const int grid_pairs = tiles < pairs ? tiles : pairs;

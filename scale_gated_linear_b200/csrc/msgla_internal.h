@@ -97,7 +97,11 @@ struct alignas(64) GemmTask {
   // kEpiStoreF32: D -> f32 [B, rows, ldf]; with w set, also the fusion weights
   // w = softmax(D[:, 0:n_scales] + bfuse) (columns 0.. hold the fusion logits)
   float* f32;
-  int ldf, pad3_;
+  int ldf;
+  // > 0: tiles from this local index on are 128-column halves of the 256-column
+  // tiles that would make up a last, partial wave (two per full tile, half 0
+  // then half 1), so that wave keeps up to twice as many CTA pairs busy
+  int half_from;
 };
 
 // Rows of one 64-column box of held coarse rows staged by the fused output GEMM
