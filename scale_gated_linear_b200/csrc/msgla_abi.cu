@@ -750,8 +750,11 @@ int forward_impl(msgla_handle* h, const void* X, int B, int L, void* O, void* ws
   long long gla_ctas = 0;
   const bool overlap = coarse_overlap(h, ws, B, &gla_ctas);
   if (overlap) {
-    // the second stream starts once the gates are done, alongside the GLA; the
-    // coarse branches' CTAs signal their stored outputs to it
+    // the second stream starts once the projection is done, alongside the GLA; the
+    // coarse branches' CTAs signal their stored outputs to it. It cannot fork
+    // earlier: its first kernel (one warp waiting for the GLA's CTAs) would hold an
+    // SM that one of the projection's CTA pairs needs (they take every SM), and
+    // that pair would run its tiles alone after the GLA had started
     lp.done = h->d_gla_done;
     lp.started = h->d_gla_done + MSGLA_MAX_SCALES;
     lp.exited = h->d_gla_done + MSGLA_MAX_SCALES + 1;
